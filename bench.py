@@ -1,0 +1,422 @@
+"""Benchmark of the AB-Attention hot path on B200.
+
+One step = one pass of the method over one batch of synthetic input: IBCS scoring
+(mean keys, per-block k-means, block scores) -> SIP selection -> HT-weighted block-sparse
+attention. The top-k mode (top-k selection -> unweighted sparse attention) is timed in
+the same run with the same protocol and reported beside it.
+
+Workload (default): Wan2.1-1.3B-shaped 480p clip, B=1, H=12, N=21x30x52=32760 tokens
+(padded to 32768), d=128, bf16, budget 10% of key blocks (26 of 256), 8 clusters, 5
+k-means iterations; synthetic inputs from block_sparse_attention_ab_b200.synth.
+
+Metric: dense-equivalent TFLOPS = 4 B H N^2 d / step time (N valid tokens), plus the
+sparse-attention kernel's ms/call and its tensor-pipe roofline on selected-block FLOPs
+(4 * 128 * 128 * d per kept (query block, key block) pair).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 run under torchrun: every rank runs the same workload on its own data (weak
+scaling, no data-path collective); the step time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+L2_BYTES = 126 * 2**20
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        # start timing only once the sampler is producing lines
+        t0 = time.time()
+        while time.time() - t0 < 5.0:
+            self.fh.flush()
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------------ workload --
+
+def workload(name: str):
+    from block_sparse_attention_ab_b200 import synth
+    return synth.WORKLOADS[name]
+
+
+def dense_equiv_flops(w) -> float:
+    return 4.0 * w.B * w.H * float(w.N) ** 2 * w.d
+
+
+def selected_flops(sum_cnt: int, d: int) -> float:
+    return 4.0 * 128 * 128 * d * sum_cnt
+
+
+# ------------------------------------------------------------------------ our arm ----
+
+def run_ours(args, rank, world, local_rank):
+    import block_sparse_attention_ab_b200 as ab
+    from block_sparse_attention_ab_b200 import build, synth
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workload(args.config)
+    if args.heads:
+        import dataclasses
+        w = dataclasses.replace(w, H=args.heads)
+    if world > 1:
+        import dataclasses
+        w = dataclasses.replace(w, data_seed=w.data_seed + 100 * rank)
+    K = w.budget_blocks(w.budgets[0])
+    q, k, v = synth.make_qkv(w)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    qc, kc, vc = (t.to(dev) for t in (q, k, v))
+    B, H, N_pad, d = qc.shape
+    nb = N_pad // 128
+    shape = ab.make_shape(qc, w.N)
+    ws = torch.empty(ab.score_workspace_bytes(shape, w.n_clusters), device=dev, dtype=torch.uint8)
+    scores = torch.empty(B, H, nb, nb, device=dev, dtype=torch.float32)
+    idx = torch.empty(B, H, nb, nb, device=dev, dtype=torch.int32)
+    cnt = torch.empty(B, H, nb, device=dev, dtype=torch.int32)
+    wt = torch.empty(B, H, nb, nb, device=dev, dtype=torch.float32)
+    out = torch.empty_like(qc)
+    flag = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    def step(events=None, mode="sip"):
+        if events:
+            events[0].record()
+        ab.score(qc, kc, w.N, w.n_clusters, w.iters, workspace=ws, out=scores)
+        if events:
+            events[1].record()
+        ab.select(scores, K, mode, w.sip_seed, dev_flag=flag, out=(idx, cnt, wt))
+        if events:
+            events[2].record()
+        if mode == "sip":
+            ab.attn_fwd(qc, kc, vc, w.N, idx, cnt, wt, dev_flag=flag, out=out)
+        else:
+            ab.attn_topk_fwd(qc, kc, vc, w.N, idx, cnt, dev_flag=flag, out=out)
+        if events:
+            events[3].record()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(mode):
+        for _ in range(args.warmup):
+            step(mode=mode)
+        torch.cuda.synchronize()
+        per = [[ev() for _ in range(4)] for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        t0, t1 = ev(), ev()
+        t0.record()
+        for i in range(args.steps):
+            step(per[i], mode=mode)
+        t1.record()
+        torch.cuda.synchronize()
+        barrier()
+        total = t0.elapsed_time(t1)
+        stage = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]),
+                           e[2].elapsed_time(e[3])] for e in per])
+        return total, stage
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    total_ms, stage_ms = timed("sip")
+    clk = clocks.stop()
+    sum_cnt = int(cnt.sum().item())
+    if ab.check_flag(flag) != 0:
+        raise RuntimeError("device flag raised during the benchmark")
+    topk_total, topk_stage = timed("topk")
+    topk_cnt = int(cnt.sum().item())
+
+    ms_step = max_over_ranks(total_ms / args.steps)
+    attn_ms = float(np.mean(stage_ms[:, 2]))
+    dense = dense_equiv_flops(w)
+    sel = selected_flops(sum_cnt, d)
+    peaks = measured_peaks()
+
+    # end to end through the public API with host buffers: pinned H2D of Q, K, V,
+    # the whole path, D2H of the output; all inside the timed region
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+    def e2e_step():
+        qd = qh.to(dev, non_blocking=True)
+        kd = kh.to(dev, non_blocking=True)
+        vd = vh.to(dev, non_blocking=True)
+        s = ab.score(qd, kd, w.N, w.n_clusters, w.iters, workspace=ws, out=scores)
+        ab.select(s, K, "sip", w.sip_seed, out=(idx, cnt, wt))
+        o = ab.attn_fwd(qd, kd, vd, w.N, idx, cnt, wt, out=out)
+        out_h.copy_(o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(1, min(args.steps, 10))
+    barrier()
+    a, b = ev(), ev()
+    a.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = out_h.numel() * out_h.element_size()
+
+    res = {
+        "metric": "sparse attn ms/call & dense-equiv TFLOPS on 1xB200; % tensor-pipe & HBM roofline",
+        "value": round(world * dense / (ms_step * 1e-3) / 1e12, 2),
+        "unit": "TFLOPS (dense-equivalent, whole step: score + SIP select + sparse attention)",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded generator shaped like Wan2.1-1.3B 480p attention; no weights or prompts)",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} (N_pad={w.N_pad}) d={w.d}, "
+                               f"budget {K}/{nb} key blocks, C={w.n_clusters}, T={w.iters}",
+                   "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world}",
+                   "l2": f"inputs Q+K+V = {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2 (no flush)"},
+        "attn_ms_per_call": round(max_over_ranks(attn_ms), 4),
+        "attn_dense_equiv_tflops": round(dense / (attn_ms * 1e-3) / 1e12, 2),
+        "attn_selected_tflops": round(sel / (attn_ms * 1e-3) / 1e12, 2),
+        "stage_ms": {"score": round(float(np.mean(stage_ms[:, 0])), 4),
+                     "select_sip": round(float(np.mean(stage_ms[:, 1])), 4),
+                     "attn_sip": round(attn_ms, 4)},
+        "sum_cnt": sum_cnt,
+        "topk": {"ms_per_step": round(topk_total / args.steps, 4),
+                 "attn_ms_per_call": round(float(np.mean(topk_stage[:, 2])), 4),
+                 "select_ms": round(float(np.mean(topk_stage[:, 1])), 4),
+                 "attn_selected_tflops": round(selected_flops(topk_cnt, d) /
+                                               (float(np.mean(topk_stage[:, 2])) * 1e-3) / 1e12, 2),
+                 "sum_cnt": topk_cnt},
+        "roofline": {"bound": "tensor",
+                     "kernel": "attn_fwd_kernel<128, weighted, bf16 out>",
+                     "achieved": round(sel / (attn_ms * 1e-3) / 1e12, 2),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(sel / (attn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                     "peak_source": f"{peaks['source']} bf16 dense burst",
+                     "traffic": args.traffic},
+        "score_roofline": {"bound": "hbm",
+                           "achieved": round((2 * q.numel() * 2 + scores.numel() * 4) /
+                                             (float(np.mean(stage_ms[:, 0])) * 1e-3) / 1e9, 1),
+                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": round((2 * q.numel() * 2 + scores.numel() * 4) /
+                                         (float(np.mean(stage_ms[:, 0])) * 1e-3) / 1e9 /
+                                         peaks["hbm_gbs"], 4)},
+        "e2e": {"value": round(world * dense / (e2e_ms * 1e-3) / 1e12, 2),
+                "unit": "TFLOPS (dense-equivalent, host buffers in and out)",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, q, k, v, K, seconds=args.cpu_seconds)
+    return res
+
+
+# ----------------------------------------------------------------- CPU oracle leg ----
+
+def cpu_baseline(w, q, k, v, K, seconds: float = 15.0, max_heads: int = 0):
+    """Time the oracle, as it stands, on a bounded sample of the same workload: whole
+    heads (IBCS scoring, SIP selection and the attention of every query block), one head
+    at a time until `seconds` have been spent; scaled to all B*H heads of one step."""
+    import oracle
+
+    t_heads = []
+    detail = None
+    for h in range(w.H):
+        qs, ks, vs = q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1]
+        t0 = time.perf_counter()
+        cent, wts, _, _, _ = oracle.kmeans(qs, w.N, w.n_clusters, w.iters)
+        s = oracle.score(cent, wts, oracle.mean_key(ks, w.N))
+        t1 = time.perf_counter()
+        idx, cnt, wt, _, _ = oracle.sip(s.astype(np.float32), K, w.sip_seed, with_p=False)
+        t2 = time.perf_counter()
+        oracle.attn_rows(qs, ks, vs, w.N, idx, cnt, wt)
+        t3 = time.perf_counter()
+        t_heads.append(t3 - t0)
+        detail = (t1 - t0, t2 - t1, t3 - t2)
+        if sum(t_heads) >= seconds or (max_heads and len(t_heads) >= max_heads):
+            break
+    per_head = sum(t_heads) / len(t_heads)
+    step_s = w.B * w.H * per_head
+    return {"value": round(dense_equiv_flops(w) / step_s / 1e12, 6),
+            "unit": "TFLOPS (dense-equivalent, whole step)",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"{len(t_heads)} of {w.B * w.H} (batch, head) slices of the workload, each "
+                       f"complete: scoring {detail[0]:.2f} s, SIP {detail[1]:.3f} s, attention of "
+                       f"all {w.n_blocks} query blocks {detail[2]:.2f} s (last slice); "
+                       f"{sum(t_heads):.1f} s of CPU time, scaled by {w.B * w.H}/{len(t_heads)}"),
+            "est_step_s": round(step_s, 2)}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle on the same workload and metric, each step a bounded
+    sample scaled to one whole step."""
+    if rank != 0:
+        return None
+    w = workload(args.config)
+    from block_sparse_attention_ab_b200 import synth
+    q, k, v = synth.make_qkv(w, heads=[0])
+    K = w.budget_blocks(w.budgets[0])
+    # each step: one complete (batch, head) slice, scaled to the whole step
+    for _ in range(args.warmup):
+        cpu_baseline(w, q, k, v, K, seconds=0.0, max_heads=1)
+    vals = []
+    last = None
+    for _ in range(args.steps):
+        last = cpu_baseline(w, q, k, v, K, seconds=0.0, max_heads=1)
+        vals.append(last["est_step_s"])
+    ms = statistics.median(vals) * 1e3
+    value = dense_equiv_flops(w) / (ms * 1e-3) / 1e12
+    return {
+        "impl": "reference",
+        "metric": "sparse attn ms/call & dense-equiv TFLOPS on 1xB200; % tensor-pipe & HBM roofline",
+        "value": round(value, 6),
+        "unit": "TFLOPS (dense-equivalent, whole step: score + SIP select + sparse attention)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} budget {K}/{w.n_blocks}",
+                   "global_batch": w.B, "seq_len": w.N, "parallelism": "dp1"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS (dense-equivalent, whole step)",
+                         "cores": last["cores"], "kind": "oracle", "sample": last["sample"]},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPS (dense-equivalent, whole step)",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="wan13b")
+    ap.add_argument("--heads", type=int, default=0, help="override head count (profiling)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per attention launch from an ncu capture of this kernel")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,228 @@
+"""AB-Attention block-sparse attention on NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C ABI in ``include/ab_attn.h`` (``libab_attn.so``, built
+in-tree by ``build.py``). Every function here only checks and marshals arguments:
+all work runs in the library's CUDA kernels on the current torch stream. There is no
+fallback: if the library is missing or no CUDA device is present, calls raise.
+
+Steps (AB-Attention news page, section «Три приёма AB-Attention»):
+  score()          IBCS block scores from per-block k-means centroids and mean keys
+  select()         SIP sampling with inclusion-probability weights, or top-k
+  attn_fwd()       block-sparse attention with Horvitz-Thompson weights (logit shift)
+  attn_topk_fwd()  the same with all weights 1 (top-k baseline)
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import synth  # noqa: F401  (seeded input generators)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libab_attn.so")
+BLOCK = 128
+
+AB_F32 = 0
+AB_BF16 = 1
+MODE_SIP = 0
+MODE_TOPK = 1
+FLAG_BAD_SCORE = 1
+FLAG_BAD_INDEX = 2
+FLAG_BAD_WEIGHT = 4
+FLAG_TIMEOUT = 8
+
+STATUS = {
+    0: "AB_OK", 1: "AB_ERR_NULL", 2: "AB_ERR_SHAPE", 3: "AB_ERR_DTYPE",
+    4: "AB_ERR_UNSUPPORTED", 5: "AB_ERR_RANGE", 6: "AB_ERR_CUDA", 7: "AB_ERR_DEVICE_FLAG",
+    8: "AB_ERR_TIMEOUT", 9: "AB_ERR_ALIGN", 10: "AB_ERR_WORKSPACE",
+}
+
+
+class AbError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = f"{where}: {STATUS.get(code, code)}"
+        if code == 6 and _lib is not None:
+            msg += f" ({_lib.ab_last_cuda_error().decode()})"
+        super().__init__(msg)
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("N_pad", ctypes.c_int32), ("d", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libab_attn.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m block_sparse_attention_ab_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, Shape
+        L.ab_score_workspace_size.argtypes = [S, I, ctypes.POINTER(ctypes.c_size_t)]
+        L.ab_score.argtypes = [P, P, S, I, I, P, P, P, P, P, P, ctypes.c_size_t, P, P]
+        L.ab_select.argtypes = [P, I, I, I, I, I, I, ctypes.c_uint64, P, P, P, P, P, P]
+        L.ab_attn_fwd.argtypes = [P, P, P, S, P, P, P, P, I, P, P, P]
+        L.ab_attn_topk_fwd.argtypes = [P, P, P, S, P, P, P, I, P, P, P]
+        L.ab_check_flag.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
+        L.ab_status_str.argtypes = [I]
+        L.ab_status_str.restype = ctypes.c_char_p
+        L.ab_version.argtypes = []
+        L.ab_last_cuda_error.argtypes = []
+        L.ab_last_cuda_error.restype = ctypes.c_char_p
+        for name in ("ab_score_workspace_size", "ab_score", "ab_select", "ab_attn_fwd",
+                     "ab_attn_topk_fwd", "ab_check_flag", "ab_version"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise AbError(code, where)
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def make_shape(q: torch.Tensor, N: int) -> Shape:
+    B, H, N_pad, d = q.shape
+    return Shape(B, H, int(N), N_pad, d, AB_BF16)
+
+
+def score_workspace_bytes(shape: Shape, n_clusters: int = 8) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().ab_score_workspace_size(shape, n_clusters, ctypes.byref(n)), "ab_score_workspace_size")
+    return int(n.value)
+
+
+def score(q: torch.Tensor, k: torch.Tensor, N: int, n_clusters: int = 8, iters: int = 5,
+          intermediates: bool = False, workspace: Optional[torch.Tensor] = None,
+          out: Optional[torch.Tensor] = None):
+    """IBCS block scores [B,H,nqb,nkb] fp32. With intermediates=True also returns
+    (kbar, centroids, cluster weights, assignment)."""
+    _need(q, torch.bfloat16, "q")
+    _need(k, torch.bfloat16, "k")
+    B, H, N_pad, d = q.shape
+    nb = N_pad // BLOCK
+    shape = make_shape(q, N)
+    dev = q.device
+    scores = out if out is not None else torch.empty(B, H, nb, nb, device=dev, dtype=torch.float32)
+    kbar = cent = cw = assign = None
+    if intermediates:
+        kbar = torch.empty(B, H, nb, d, device=dev, dtype=torch.float32)
+        cent = torch.empty(B, H, nb, n_clusters, d, device=dev, dtype=torch.float32)
+        cw = torch.empty(B, H, nb, n_clusters, device=dev, dtype=torch.float32)
+        assign = torch.empty(B, H, N_pad, device=dev, dtype=torch.uint8)
+    if workspace is None:
+        workspace = torch.empty(score_workspace_bytes(shape, n_clusters), device=dev, dtype=torch.uint8)
+    _check(lib().ab_score(_ptr(q), _ptr(k), shape, n_clusters, iters, _ptr(scores), _ptr(kbar),
+                          _ptr(cent), _ptr(cw), _ptr(assign), _ptr(workspace),
+                          workspace.numel(), None, _stream()), "ab_score")
+    if intermediates:
+        return scores, kbar, cent, cw, assign
+    return scores
+
+
+def select(scores: torch.Tensor, budget: int, mode: str = "sip", seed: int = 0,
+           want_p: bool = False, dev_flag: Optional[torch.Tensor] = None, out=None):
+    """Returns (idx int32, cnt int32, w fp32[, p fp64]) for SIP or top-k."""
+    _need(scores, torch.float32, "scores")
+    B, H, nqb, nkb = scores.shape
+    dev = scores.device
+    if out is not None:
+        idx, cnt, w = out[:3]
+    else:
+        idx = torch.empty(B, H, nqb, nkb, device=dev, dtype=torch.int32)
+        cnt = torch.empty(B, H, nqb, device=dev, dtype=torch.int32)
+        w = torch.empty(B, H, nqb, nkb, device=dev, dtype=torch.float32)
+    p = torch.empty(B, H, nqb, nkb, device=dev, dtype=torch.float64) if want_p else None
+    m = {"sip": MODE_SIP, "topk": MODE_TOPK}[mode]
+    _check(lib().ab_select(_ptr(scores), B, H, nqb, nkb, int(budget), m,
+                           ctypes.c_uint64(int(seed) & (2**64 - 1)), _ptr(idx), _ptr(cnt), _ptr(w),
+                           _ptr(p), _ptr(dev_flag), _stream()), "ab_select")
+    return (idx, cnt, w, p) if want_p else (idx, cnt, w)
+
+
+def _out_buffer(q, out, out_dtype):
+    if out is not None:
+        _need(out, out_dtype, "out")
+        return out
+    return torch.empty(q.shape, device=q.device, dtype=out_dtype)
+
+
+def _out_code(out_dtype):
+    return {torch.bfloat16: AB_BF16, torch.float32: AB_F32}[out_dtype]
+
+
+def attn_fwd(q, k, v, N: int, idx, cnt, w, want_lse: bool = False,
+             dev_flag: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+             out_dtype=torch.bfloat16):
+    """Block-sparse HT-weighted attention; returns out (bf16 or fp32) [and lse fp32]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    _need(idx, torch.int32, "idx")
+    _need(cnt, torch.int32, "cnt")
+    _need(w, torch.float32, "w")
+    o = _out_buffer(q, out, out_dtype)
+    lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32) if want_lse else None
+    _check(lib().ab_attn_fwd(_ptr(q), _ptr(k), _ptr(v), make_shape(q, N), _ptr(idx), _ptr(cnt),
+                             _ptr(w), _ptr(o), _out_code(out_dtype), _ptr(lse), _ptr(dev_flag),
+                             _stream()), "ab_attn_fwd")
+    return (o, lse) if want_lse else o
+
+
+def attn_topk_fwd(q, k, v, N: int, idx, cnt, want_lse: bool = False,
+                  dev_flag: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                  out_dtype=torch.bfloat16):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    _need(idx, torch.int32, "idx")
+    _need(cnt, torch.int32, "cnt")
+    o = _out_buffer(q, out, out_dtype)
+    lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32) if want_lse else None
+    _check(lib().ab_attn_topk_fwd(_ptr(q), _ptr(k), _ptr(v), make_shape(q, N), _ptr(idx),
+                                  _ptr(cnt), _ptr(o), _out_code(out_dtype), _ptr(lse),
+                                  _ptr(dev_flag), _stream()), "ab_attn_topk_fwd")
+    return (o, lse) if want_lse else o
+
+
+def check_flag(dev_flag: torch.Tensor) -> int:
+    """Synchronise the current stream and return the device flag bits."""
+    host = ctypes.c_int(0)
+    code = lib().ab_check_flag(_ptr(dev_flag), ctypes.byref(host), _stream())
+    if code not in (0, 7, 8):
+        raise AbError(code, "ab_check_flag")
+    return int(host.value)
+
+
+def ab_attention(q, k, v, N: int, budget: int, mode: str = "sip", seed: int = 0,
+                 n_clusters: int = 8, iters: int = 5):
+    """One pass of the whole path: score -> select -> sparse attention (device tensors)."""
+    s = score(q, k, N, n_clusters, iters)
+    idx, cnt, w = select(s, budget, mode, seed)
+    if mode == "sip":
+        return attn_fwd(q, k, v, N, idx, cnt, w)
+    return attn_topk_fwd(q, k, v, N, idx, cnt)

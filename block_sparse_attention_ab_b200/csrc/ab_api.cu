@@ -1,0 +1,203 @@
+// ab_api.cu -- the C ABI declared in include/ab_attn.h: host-side argument checks,
+// workspace carving, and kernel launches on the caller's stream. No device memory is
+// allocated here and no state is kept between calls.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/ab_attn.h"
+#include "ab_kernels.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ab_status check_shape(const ab_shape &s)
+{
+    if (s.B <= 0 || s.H <= 0 || s.N <= 0 || s.N_pad <= 0 || s.d <= 0) return AB_ERR_SHAPE;
+    if (s.N_pad % AB_BLOCK != 0 || s.N > s.N_pad || s.N_pad - s.N >= AB_BLOCK) return AB_ERR_SHAPE;
+    if (s.dtype != AB_BF16) return AB_ERR_DTYPE;
+    if (s.d != 64 && s.d != 128) return AB_ERR_UNSUPPORTED;
+    if (s.N_pad / AB_BLOCK > AB_MAX_BLOCKS) return AB_ERR_RANGE;
+    // grid and index arithmetic stay in int / size_t ranges
+    if ((long long)s.B * s.H > 65535LL) return AB_ERR_RANGE;
+    return AB_OK;
+}
+
+struct ScoreLayout {
+    size_t kbar, cent, cw, total;
+};
+
+ScoreLayout score_layout(const ab_shape &s, int C)
+{
+    const size_t BH = (size_t)s.B * s.H, nb = (size_t)s.N_pad / AB_BLOCK;
+    ScoreLayout L;
+    L.kbar = 0;
+    L.cent = round_up(L.kbar + BH * nb * s.d * sizeof(float), kAlign);
+    L.cw = round_up(L.cent + BH * nb * C * s.d * sizeof(float), kAlign);
+    L.total = round_up(L.cw + BH * nb * C * sizeof(float), kAlign);
+    return L;
+}
+
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+ab_status cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return AB_OK;
+    g_last_cuda_error = e;
+    return AB_ERR_CUDA;
+}
+
+ab_status attn_common(const void *q, const void *k, const void *v, ab_shape s, const int32_t *idx,
+                      const int32_t *cnt, const float *w, void *out, ab_dtype out_dtype,
+                      float *lse, int *dev_flag, void *stream)
+{
+    if (!q || !k || !v || !idx || !cnt || !out) return AB_ERR_NULL;
+    ab_status st = check_shape(s);
+    if (st != AB_OK) return st;
+    if (out_dtype != AB_BF16 && out_dtype != AB_F32) return AB_ERR_DTYPE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(idx) ||
+        !aligned16(cnt) || (w && !aligned16(w)) || (lse && !aligned16(lse)))
+        return AB_ERR_ALIGN;
+    ab::AttnLaunch a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.w = w;
+    a.out = out;
+    a.out_f32 = out_dtype == AB_F32;
+    a.lse = lse;
+    a.flag = dev_flag;
+    a.B = s.B;
+    a.H = s.H;
+    a.N = s.N;
+    a.N_pad = s.N_pad;
+    a.d = s.d;
+    a.grid_override = 0;
+    return cuda_status(ab::launch_attn(a, (cudaStream_t)stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+ab_status ab_score_workspace_size(ab_shape s, int n_clusters, size_t *bytes)
+{
+    if (!bytes) return AB_ERR_NULL;
+    *bytes = 0;
+    ab_status st = check_shape(s);
+    if (st != AB_OK) return st;
+    if (n_clusters < 1 || n_clusters > 8) return AB_ERR_UNSUPPORTED;
+    *bytes = score_layout(s, n_clusters).total;
+    return AB_OK;
+}
+
+ab_status ab_score(const void *q, const void *k, ab_shape s, int n_clusters, int iters,
+                   float *scores, float *kbar, float *centroids, float *cweights,
+                   uint8_t *assign, void *workspace, size_t workspace_bytes, int *dev_flag,
+                   void *stream)
+{
+    (void)dev_flag;  // the scoring kernels have no device-detected failure mode
+    if (!q || !k || !scores) return AB_ERR_NULL;
+    ab_status st = check_shape(s);
+    if (st != AB_OK) return st;
+    if (n_clusters < 1 || n_clusters > 8) return AB_ERR_UNSUPPORTED;
+    if (iters < 1 || iters > 1000) return AB_ERR_RANGE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(scores) || (kbar && !aligned16(kbar)) ||
+        (centroids && !aligned16(centroids)) || (cweights && !aligned16(cweights)) ||
+        !aligned16(workspace))
+        return AB_ERR_ALIGN;
+    const ScoreLayout L = score_layout(s, n_clusters);
+    if (!workspace || workspace_bytes < L.total) return AB_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *kb = kbar ? kbar : reinterpret_cast<float *>(ws + L.kbar);
+    float *ce = centroids ? centroids : reinterpret_cast<float *>(ws + L.cent);
+    float *cw = cweights ? cweights : reinterpret_cast<float *>(ws + L.cw);
+    const int BH = s.B * s.H, nb = s.N_pad / AB_BLOCK;
+    cudaStream_t cs = (cudaStream_t)stream;
+    cudaError_t e = ab::launch_meankey(k, kb, BH, s.N, s.N_pad, s.d, cs);
+    if (e == cudaSuccess)
+        e = ab::launch_kmeans(q, ce, cw, assign, BH, s.N, s.N_pad, s.d, n_clusters, iters, cs);
+    if (e == cudaSuccess) e = ab::launch_score(ce, cw, kb, scores, BH, nb, nb, s.d, n_clusters, cs);
+    return cuda_status(e);
+}
+
+ab_status ab_select(const float *scores, int B, int H, int nqb, int nkb, int budget,
+                    ab_mode mode, uint64_t seed, int32_t *idx, int32_t *cnt, float *w, double *p,
+                    int *dev_flag, void *stream)
+{
+    if (!scores || !idx || !cnt) return AB_ERR_NULL;
+    if (mode == AB_MODE_SIP && !w) return AB_ERR_NULL;
+    if (mode != AB_MODE_SIP && mode != AB_MODE_TOPK) return AB_ERR_UNSUPPORTED;
+    if (B <= 0 || H <= 0 || nqb <= 0 || nkb <= 0) return AB_ERR_SHAPE;
+    if (nkb > AB_MAX_BLOCKS || budget < 1) return AB_ERR_RANGE;
+    if ((long long)B * H * nqb > 2147483647LL) return AB_ERR_RANGE;
+    if (!aligned16(scores) || !aligned16(idx) || !aligned16(cnt) || (w && !aligned16(w)) ||
+        (p && !aligned16(p)))
+        return AB_ERR_ALIGN;
+    const int K = budget < nkb ? budget : nkb;
+    cudaStream_t cs = (cudaStream_t)stream;
+    cudaError_t e;
+    if (mode == AB_MODE_SIP)
+        e = ab::launch_sip(scores, B, H, nqb, nkb, K, seed, idx, cnt, w, p, dev_flag, cs);
+    else
+        e = ab::launch_topk(scores, B, H, nqb, nkb, K, idx, cnt, w, dev_flag, cs);
+    return cuda_status(e);
+}
+
+ab_status ab_attn_fwd(const void *q, const void *k, const void *v, ab_shape s, const int32_t *idx,
+                      const int32_t *cnt, const float *w, void *out, ab_dtype out_dtype,
+                      float *lse, int *dev_flag, void *stream)
+{
+    if (!w) return AB_ERR_NULL;
+    return attn_common(q, k, v, s, idx, cnt, w, out, out_dtype, lse, dev_flag, stream);
+}
+
+ab_status ab_attn_topk_fwd(const void *q, const void *k, const void *v, ab_shape s,
+                           const int32_t *idx, const int32_t *cnt, void *out, ab_dtype out_dtype,
+                           float *lse, int *dev_flag, void *stream)
+{
+    return attn_common(q, k, v, s, idx, cnt, nullptr, out, out_dtype, lse, dev_flag, stream);
+}
+
+ab_status ab_check_flag(const int *dev_flag, int *host_flag, void *stream)
+{
+    if (!dev_flag || !host_flag) return AB_ERR_NULL;
+    cudaError_t e = cudaMemcpyAsync(host_flag, dev_flag, sizeof(int), cudaMemcpyDeviceToHost,
+                                    (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (*host_flag == 0) return AB_OK;
+    if (*host_flag & AB_FLAG_TIMEOUT) return AB_ERR_TIMEOUT;
+    return AB_ERR_DEVICE_FLAG;
+}
+
+const char *ab_status_str(ab_status s)
+{
+    switch (s) {
+    case AB_OK: return "AB_OK";
+    case AB_ERR_NULL: return "AB_ERR_NULL";
+    case AB_ERR_SHAPE: return "AB_ERR_SHAPE";
+    case AB_ERR_DTYPE: return "AB_ERR_DTYPE";
+    case AB_ERR_UNSUPPORTED: return "AB_ERR_UNSUPPORTED";
+    case AB_ERR_RANGE: return "AB_ERR_RANGE";
+    case AB_ERR_CUDA: return "AB_ERR_CUDA";
+    case AB_ERR_DEVICE_FLAG: return "AB_ERR_DEVICE_FLAG";
+    case AB_ERR_TIMEOUT: return "AB_ERR_TIMEOUT";
+    case AB_ERR_ALIGN: return "AB_ERR_ALIGN";
+    case AB_ERR_WORKSPACE: return "AB_ERR_WORKSPACE";
+    }
+    return "AB_ERR_UNKNOWN";
+}
+
+const char *ab_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+
+int ab_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,640 @@
+// attn_kernel.cu -- block-sparse flash-attention forward with Horvitz-Thompson block
+// weights on sm_100a (AB-Attention news page, section «Три приёма AB-Attention»: each
+// sampled block counts with weight 1/p in the numerator and the softmax normaliser,
+// which keeps the computation ordinary softmax attention with a logit shift; the
+// kernel gathers the chosen key/value blocks by index, tokens stay in order).
+//
+// One persistent CTA per SM walks work items (b, h, query block) in head-major order
+// (CTA c takes items c, c + grid, ...), so concurrently running CTAs share a head's
+// K/V in L2. Per CTA, 320 threads in three roles:
+//   warps 0-7  softmax: warps q and q+4 own query rows 32q..32q+31 (TMEM lanes), warp
+//              q the first 64 key columns of each S row and warp q+4 the last 64; they
+//              read S from TMEM, run the online softmax in the log2 domain with the
+//              block's log2(w) added, write P (bf16) back over S, lazily rescale their
+//              half of O, and normalise and store their half of each output row;
+//   warp 8     TMA producer: Q tile (double buffered) and a ring of K / V tiles
+//              fetched by block index with 3-D tensor maps whose row extent is N, so
+//              rows past the sequence end arrive as zeros;
+//   warp 9     TMEM owner and MMA issuer: S = Q K^T (both operands from shared
+//              memory) into one of two S buffers, O += P V (P from TMEM).
+// Issue order of the MMA warp over the CTA's whole block stream g = 0, 1, ...:
+//   S(0), S(1), PV(0), S(2), PV(1), ...  so S(g+1) runs while block g is in softmax.
+// Every wait is bounded (2 s); on a timeout the roles unwind, drain their own
+// asynchronous work and the CTA frees its TMEM before returning.
+#include <cmath>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ab_device.cuh"
+#include "ab_kernels.h"
+
+namespace ab {
+
+constexpr int kAttnThreads = 320;  // 8 softmax warps, 1 TMA warp, 1 MMA warp
+constexpr int kWarpTma = 8, kWarpMma = 9;
+constexpr int kTmemCols = 512;
+constexpr int kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 256 without a rescale
+
+struct AttnParams {
+    const int32_t *idx;
+    const int32_t *cnt;
+    const float *w;  // nullptr: all weights 1 (top-k)
+    void *out;       // bf16 or fp32 [B*H, N_pad, D]
+    float *lse;
+    int *flag;
+    int H, N, N_pad, nqb, nkb;
+    int n_items;
+    float scale_log2;  // log2(e) / sqrt(d)
+};
+
+template <int D>
+struct AttnSmem {
+    static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
+    static constexpr int kBoxes = D / 64;           // 64-column (128-byte) TMA boxes per tile
+    static constexpr int kStages = D == 128 ? 4 : 8;
+    static constexpr int kQOff = 0;
+    static constexpr int kKVOff = 2 * kTileBytes;
+    static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2],
+    // o_full, drain
+    static constexpr int kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 1 + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kXchOff = kMiscOff + 16;  // softmax exchange: float [2][2][128] + [2][128]
+    static constexpr int kBytes = kXchOff + (2 * 2 * 128 + 2 * 128) * 4;
+    static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
+};
+
+// The per-CTA stream of (item, block) pairs shared by the three roles.
+struct Cursor {
+    int r;    // work item (flat (b*H + h)*nqb + qb); >= n_items when done
+    int i;    // block position within the item
+    int n;    // selected-block count of the item (clamped to [0, nkb])
+    int seq;  // index of the item among this CTA's non-empty items
+};
+
+__device__ __forceinline__ int load_cnt(const AttnParams &p, int r)
+{
+    const int c = __ldg(p.cnt + r);
+    return c < 0 ? 0 : (c > p.nkb ? p.nkb : c);
+}
+
+__device__ __forceinline__ void cursor_seek(Cursor &c, const AttnParams &p)
+{
+    while (c.r < p.n_items && c.i >= c.n) {
+        if (c.n > 0) ++c.seq;
+        c.r += gridDim.x;
+        c.i = 0;
+        c.n = c.r < p.n_items ? load_cnt(p, c.r) : 0;
+    }
+}
+
+__device__ __forceinline__ Cursor cursor_first(const AttnParams &p)
+{
+    Cursor c;
+    c.r = blockIdx.x;
+    c.i = 0;
+    c.seq = 0;
+    c.n = c.r < p.n_items ? load_cnt(p, c.r) : 0;
+    cursor_seek(c, p);
+    return c;
+}
+
+__device__ __forceinline__ void cursor_next(Cursor &c, const AttnParams &p)
+{
+    ++c.i;
+    cursor_seek(c, p);
+}
+
+__device__ __forceinline__ int block_index(const AttnParams &p, int r, int i, bool report)
+{
+    int j = __ldg(p.idx + (size_t)r * p.nkb + i);
+    if (j < 0 || j >= p.nkb) {
+        if (report) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
+        j = j < 0 ? 0 : p.nkb - 1;
+    }
+    return j;
+}
+
+// bounded wait that ignores the abort flag (used only to drain in-flight work)
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > 200000000ull) return;
+    }
+}
+
+template <int D, bool kWeighted, bool kOutF32>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const AttnParams p)
+{
+    using L = AttnSmem<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+    uint64_t *q_full = bars;
+    uint64_t *q_empty = bars + 2;
+    uint64_t *kv_full = bars + 4;
+    uint64_t *kv_empty = kv_full + L::kStages;
+    uint64_t *s_full = kv_empty + L::kStages;
+    uint64_t *p_full = s_full + 2;
+    uint64_t *o_full = p_full + 2;
+    uint64_t *drain = o_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&q_full[b], 1);
+            mbar_init(&q_empty[b], 1);
+            mbar_init(&s_full[b], 1);
+            mbar_init(&p_full[b], 256);
+        }
+        for (int s = 0; s < L::kStages; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(o_full, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kWarpTma) {
+        // ------------------------------ TMA producer ------------------------------
+        // The whole warp runs the control flow (warp-uniform values); one elected lane
+        // issues each copy.
+        if (elect_one()) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+        }
+        __syncwarp();
+        int kv_pos = 0;
+        int q_loads = 0;
+        bool ok = true;
+        auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag));
+        };
+        auto load_q = [&](const Cursor &c) -> bool {
+            const int b = c.seq & 1;
+            if (!wait(&q_empty[b], ((c.seq >> 1) & 1) ^ 1)) return false;
+            uint8_t *dst = smem + L::kQOff + b * L::kTileBytes;
+            const int bh = c.r / p.nqb, qb = c.r % p.nqb;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&q_full[b], L::kTileBytes);
+#pragma unroll
+                for (int x = 0; x < L::kBoxes; ++x)
+                    tma_load_3d(dst + x * 16384, &tmQ, &q_full[b], x * 64, qb * 128, bh);
+            }
+            __syncwarp();
+            ++q_loads;
+            return true;
+        };
+        auto load_kv = [&](const Cursor &c, const CUtensorMap *tm) -> bool {
+            const int s = kv_pos % L::kStages;
+            if (!wait(&kv_empty[s], ((kv_pos / L::kStages) & 1) ^ 1)) return false;
+            const int j = block_index(p, c.r, c.i, tm == &tmK && lane == 0);
+            uint8_t *dst = smem + L::kKVOff + s * L::kTileBytes;
+            const int bh = c.r / p.nqb;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&kv_full[s], L::kTileBytes);
+#pragma unroll
+                for (int x = 0; x < L::kBoxes; ++x)
+                    tma_load_3d(dst + x * 16384, tm, &kv_full[s], x * 64, j * 128, bh);
+            }
+            __syncwarp();
+            ++kv_pos;
+            return true;
+        };
+        Cursor cur = cursor_first(p);
+        if (cur.r < p.n_items) {
+            ok = load_q(cur) && load_kv(cur, &tmK);
+            while (ok) {
+                Cursor nxt = cur;
+                cursor_next(nxt, p);
+                const bool more = nxt.r < p.n_items;
+                if (more) {
+                    if (nxt.i == 0) ok = load_q(nxt);
+                    ok = ok && load_kv(nxt, &tmK);
+                }
+                ok = ok && load_kv(cur, &tmV);
+                if (!more) break;
+                cur = nxt;
+            }
+        }
+        if (!ok) {
+            // drain: the last loads issued may still be in flight
+            for (int k = kv_pos - L::kStages; k < kv_pos; ++k)
+                if (k >= 0) drain_wait(&kv_full[k % L::kStages], (k / L::kStages) & 1);
+            for (int k = q_loads - 2; k < q_loads; ++k)
+                if (k >= 0) drain_wait(&q_full[k & 1], (k >> 1) & 1);
+        }
+    } else if (warp == kWarpMma) {
+        // ------------------------------- MMA issuer -------------------------------
+        // The whole warp runs the control flow, so descriptors and addresses are
+        // warp-uniform values; one elected lane issues each tcgen05.mma / commit.
+        // Per MMA only a constant is added to a precomputed descriptor's start-address
+        // field (addresses stay below 256 KB, so the 14-bit field never carries): a
+        // lean issue path lets one thread keep up with the tensor core.
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+        constexpr uint64_t kTileDesc = L::kTileBytes >> 4;
+        const uint64_t q_desc0 = smem_desc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+        const uint64_t k_desc0 = smem_desc_sw128(smem_u32(smem + L::kKVOff), 16, 1024);
+        const uint64_t v_desc0 = smem_desc_sw128(smem_u32(smem + L::kKVOff), 16384, 1024);
+        int kv_pos = 0;
+        bool ok = true;
+        auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag));
+        };
+        auto issue_s = [&](const Cursor &c, int g) -> bool {
+            const int qbuf = c.seq & 1;
+            if (c.i == 0 && !wait(&q_full[qbuf], (c.seq >> 1) & 1)) return false;
+            const int s = kv_pos % L::kStages;
+            if (!wait(&kv_full[s], (kv_pos / L::kStages) & 1)) return false;
+            tc_fence_after();
+            const uint64_t qd = q_desc0 + (uint64_t)qbuf * kTileDesc;
+            const uint64_t kd = k_desc0 + (uint64_t)s * kTileDesc;
+            const uint32_t d_tmem = tmem + ((g & 1) ? kColS1 : kColS0);
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                    mma_ss(d_tmem, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&s_full[g & 1]);
+                mma_commit(&kv_empty[s]);
+                if (c.i == c.n - 1) mma_commit(&q_empty[qbuf]);
+            }
+            __syncwarp();
+            ++kv_pos;
+            return true;
+        };
+        Cursor cur = cursor_first(p);
+        int g = 0;
+        if (cur.r < p.n_items) {
+            ok = issue_s(cur, 0);
+            while (ok) {
+                Cursor nxt = cur;
+                cursor_next(nxt, p);
+                const bool more = nxt.r < p.n_items;
+                if (more && !issue_s(nxt, g + 1)) {
+                    ok = false;
+                    break;
+                }
+                // O (+)= P(g) V(g)
+                if (!wait(&p_full[g & 1], (g >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const int s = kv_pos % L::kStages;
+                if (!wait(&kv_full[s], (kv_pos / L::kStages) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t vd = v_desc0 + (uint64_t)s * kTileDesc;
+                const uint32_t p_tmem = tmem + ((g & 1) ? kColS1 : kColS0);
+                const uint32_t acc0 = cur.i > 0 ? 1u : 0u;
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < 128 / 16; ++kk)
+                        mma_ts(tmem + kColO, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)),
+                               idesc_pv, kk > 0 ? 1u : acc0);
+                    mma_commit(&kv_empty[s]);
+                    mma_commit(o_full);
+                }
+                __syncwarp();
+                ++kv_pos;
+                if (!more) break;
+                cur = nxt;
+                ++g;
+            }
+        }
+        if (!ok) {
+            if (elect_one()) {
+                mma_commit(drain);
+                drain_wait(drain, 0);
+            }
+            __syncwarp();
+        }
+    } else {
+        // -------------------------------- softmax ---------------------------------
+        // Warps q and q + 4 share TMEM lanes 32q..32q+31 (query rows); warp q takes S
+        // columns 0..63 of those rows, warp q + 4 columns 64..127. The row max is
+        // exchanged through shared memory across a 64-thread named barrier; warp q + 4
+        // writes P into columns 32..63, which warp q reads as S, only after it.
+        // These warps never leave their loops early: after a failed (timed-out) wait
+        // they skip the remaining waits but keep the same sequence of named barriers,
+        // so a pair can never be left waiting for its partner.
+        const int quad = warp & 3, half = warp >> 2;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        float *xmax_sh = reinterpret_cast<float *>(smem + L::kXchOff);  // [2][2][128]
+        float *xl_sh = xmax_sh + 2 * 2 * 128;                            // [2][128]
+        auto pair_sync = [&]() {
+            tc_fence_before();
+            asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
+            tc_fence_after();
+        };
+        int g = 0;
+        int o_seen = 0;  // PV completions observed so far
+        bool ok = true;
+        auto wait_bar = [&](uint64_t *bar, uint32_t parity) {
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag));
+        };
+        auto wait_o = [&](int k) {  // wait until PV(k) is complete
+            if (o_seen > k) return;
+            wait_bar(o_full, k & 1);
+            o_seen = k + 1;
+        };
+        auto block_lw = [&](float wj) -> float {
+            if (!kWeighted) return 0.f;
+            if (wj > 0.f && wj < INFINITY) return log2f(wj);
+            if (warp == 0 && lane == 0) raise_flag(p.flag, AB_FLAG_BAD_WEIGHT);
+            return 0.f;
+        };
+        constexpr int kHalfD = D / 2;
+        constexpr int kSoftPairs = 6;  // of 32 pairs per block: exp2 on the FMA pipe
+        const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+        for (int r = blockIdx.x; r < p.n_items; r += gridDim.x) {
+            const int n = load_cnt(p, r);
+            const int bh = r / p.nqb, qb = r % p.nqb;
+            const int tok = qb * 128 + row;
+            const size_t orow_off = ((size_t)bh * p.N_pad + tok) * D + half * kHalfD;
+            // this thread's half output row: D/2 bf16 (D/16 uint4) or D/2 fp32 (D/8 uint4)
+            uint4 *o4 = kOutF32 ? reinterpret_cast<uint4 *>(static_cast<float *>(p.out) + orow_off)
+                                : reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow_off);
+            constexpr int kRowVecs = kOutF32 ? kHalfD / 4 : kHalfD / 8;
+            if (warp == 0 && lane == 0) {
+                const int c = __ldg(p.cnt + r);
+                if (c < 0 || c > p.nkb) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
+            }
+            if (n == 0) {
+#pragma unroll
+                for (int e = 0; e < kRowVecs; ++e) o4[e] = make_uint4(0, 0, 0, 0);
+                if (p.lse && half == 0) p.lse[(size_t)bh * p.N_pad + tok] = tok < p.N ? -INFINITY : 0.f;
+                continue;
+            }
+            const int32_t *idx_row = p.idx + (size_t)r * p.nkb;
+            const float *w_row = kWeighted ? p.w + (size_t)r * p.nkb : nullptr;
+            int j_next = __ldg(idx_row);
+            float w_next = kWeighted ? __ldg(w_row) : 1.f;
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int i = 0; i < n; ++i, ++g) {
+                int j = j_next;
+                if (j < 0 || j >= p.nkb) j = j < 0 ? 0 : p.nkb - 1;
+                const float lw = block_lw(w_next);
+                if (i + 1 < n) {  // prefetch the next block's index and weight
+                    j_next = __ldg(idx_row + i + 1);
+                    if (kWeighted) w_next = __ldg(w_row + i + 1);
+                }
+                const int nvalid = min(128, p.N - j * 128) - half * 64;  // valid columns here
+                const uint32_t s_col = (g & 1) ? kColS1 : kColS0;
+                wait_bar(&s_full[g & 1], (g >> 1) & 1);
+                tc_fence_after();
+                // the destination registers are only read after tcgen05.wait::ld
+                uint32_t su[64];
+                tmem_ld32(tmem + lane_off + s_col + half * 64,
+                          *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
+                tmem_ld32(tmem + lane_off + s_col + half * 64 + 32,
+                          *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
+                tmem_wait_ld();
+                float sv[64];
+#pragma unroll
+                for (int e = 0; e < 64; ++e) sv[e] = __uint_as_float(su[e]);
+                if (nvalid < 64) {
+#pragma unroll
+                    for (int e = 0; e < 64; ++e)
+                        if (e >= nvalid) sv[e] = -INFINITY;
+                }
+                // row max: 8 independent chains, then a tree; the two halves exchange theirs
+                float mx[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) mx[t] = sv[t];
+#pragma unroll
+                for (int e = 8; e < 64; e += 8)
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) mx[t] = fmaxf(mx[t], sv[e + t]);
+                mx[0] = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                xmax_sh[((g & 1) * 2 + half) * 128 + row] = mx[0];
+                pair_sync();
+                const float smax = fmaxf(mx[0], xmax_sh[((g & 1) * 2 + (half ^ 1)) * 128 + row]);
+                const float xmax = smax * p.scale_log2 + lw;
+                const float m_new = fmaxf(m_run, xmax);
+                bool rescale = false;
+                if (i == 0) {
+                    m_run = m_new;
+                } else if (m_new > m_run + kRescaleThreshold) {
+                    rescale = true;
+                }
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // O *= 2^(m_run - m_new) on the rows that need it; PV(g-1) must be done
+                    wait_o(g - 1);
+                    tc_fence_after();
+                    const float f = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+#pragma unroll 1
+                    for (int ch = 0; ch < kHalfD / 32; ++ch) {
+                        uint32_t r32[32];
+                        const uint32_t oc = kColO + half * kHalfD + ch * 32;
+                        tmem_ld32(tmem + lane_off + oc, r32);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            r32[e] = __float_as_uint(__uint_as_float(r32[e]) * f);
+                        tmem_st32(tmem + lane_off + oc, r32);
+                    }
+                    if (rescale) {
+                        l_run *= f;
+                        m_run = m_new;
+                    }
+                }
+                // P = 2^(s * scale_log2 + lw - m_run) in fp32 pairs, packed to bf16 over
+                // the S columns; the first kSoftPairs pairs use the FMA-pipe exp2
+                const float bias = lw - m_run;
+                const uint64_t bias2 = f2_pack(bias, bias);
+                uint64_t ls2[4] = {0, 0, 0, 0};
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const uint64_t x2 = f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), scale2, bias2);
+                    float2 pr;
+                    if (e < kSoftPairs) {
+                        pr = soft_exp2_pair(x2);
+                    } else {
+                        const float2 xv = f2_unpack(x2);
+                        pr.x = fast_exp2(xv.x);
+                        pr.y = fast_exp2(xv.y);
+                    }
+                    ls2[e & 3] = f2_add(ls2[e & 3], f2_pack(pr.x, pr.y));
+                    pk[e] = pack_bf16x2(pr.x, pr.y);
+                }
+                tmem_st32(tmem + lane_off + s_col + half * 32, pk);
+                {
+                    const float2 a = f2_unpack(f2_add(f2_add(ls2[0], ls2[1]), f2_add(ls2[2], ls2[3])));
+                    l_run += a.x + a.y;
+                }
+                tmem_wait_st();
+                if (g > 0) wait_o(g - 1);
+                tc_fence_before();
+                mbar_arrive(&p_full[g & 1]);
+
+                if (i == n - 1) {
+                    // epilogue: O / l (l summed over both halves), straight to global memory
+                    wait_o(g);
+                    xl_sh[half * 128 + row] = l_run;
+                    pair_sync();
+                    const float l_tot = l_run + xl_sh[(half ^ 1) * 128 + row];
+                    const float inv = tok < p.N ? 1.0f / l_tot : 0.f;
+#pragma unroll 1
+                    for (int ch = 0; ch < kHalfD / 32; ++ch) {
+                        uint32_t r32[32];
+                        tmem_ld32(tmem + lane_off + kColO + half * kHalfD + ch * 32, r32);
+                        tmem_wait_ld();
+                        if (kOutF32) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                uint4 v;
+                                v.x = __float_as_uint(__uint_as_float(r32[4 * e + 0]) * inv);
+                                v.y = __float_as_uint(__uint_as_float(r32[4 * e + 1]) * inv);
+                                v.z = __float_as_uint(__uint_as_float(r32[4 * e + 2]) * inv);
+                                v.w = __float_as_uint(__uint_as_float(r32[4 * e + 3]) * inv);
+                                o4[ch * 8 + e] = v;
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                uint4 v;
+                                v.x = pack_bf16x2(__uint_as_float(r32[8 * e + 0]) * inv,
+                                                  __uint_as_float(r32[8 * e + 1]) * inv);
+                                v.y = pack_bf16x2(__uint_as_float(r32[8 * e + 2]) * inv,
+                                                  __uint_as_float(r32[8 * e + 3]) * inv);
+                                v.z = pack_bf16x2(__uint_as_float(r32[8 * e + 4]) * inv,
+                                                  __uint_as_float(r32[8 * e + 5]) * inv);
+                                v.w = pack_bf16x2(__uint_as_float(r32[8 * e + 6]) * inv,
+                                                  __uint_as_float(r32[8 * e + 7]) * inv);
+                                o4[ch * 4 + e] = v;
+                            }
+                        }
+                    }
+                    if (p.lse && half == 0)
+                        p.lse[(size_t)bh * p.N_pad + tok] =
+                            tok < p.N ? (m_run + log2f(l_tot)) * 0.69314718055994531f : 0.f;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 3-D map over a [B*H, N_pad, d] bf16 tensor with row extent N (rows >= N read as 0),
+// box 64 columns x 128 rows, 128-byte swizzle.
+static bool make_tmap(CUtensorMap *tm, const void *base, int BH, int N, int N_pad, int d)
+{
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N_pad * d * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool W, bool F32>
+static cudaError_t launch_attn_t(const AttnLaunch &a, cudaStream_t st)
+{
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, a.q, a.B * a.H, a.N, a.N_pad, D) ||
+        !make_tmap(&tk, a.k, a.B * a.H, a.N, a.N_pad, D) ||
+        !make_tmap(&tv, a.v, a.B * a.H, a.N, a.N_pad, D))
+        return cudaErrorInvalidValue;
+    AttnParams p;
+    p.idx = a.idx;
+    p.cnt = a.cnt;
+    p.w = a.w;
+    p.out = a.out;
+    p.lse = a.lse;
+    p.flag = a.flag;
+    p.H = a.H;
+    p.N = a.N;
+    p.N_pad = a.N_pad;
+    p.nqb = a.N_pad / 128;
+    p.nkb = a.N_pad / 128;
+    p.n_items = a.B * a.H * p.nqb;
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    const int smem = AttnSmem<D>::kAlloc;
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, W, F32>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = a.grid_override > 0 ? a.grid_override : (p.n_items < sms ? p.n_items : sms);
+    attn_fwd_kernel<D, W, F32><<<grid, kAttnThreads, smem, st>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+template <int D, bool W>
+static cudaError_t launch_attn_o(const AttnLaunch &a, cudaStream_t st)
+{
+    return a.out_f32 ? launch_attn_t<D, W, true>(a, st) : launch_attn_t<D, W, false>(a, st);
+}
+
+cudaError_t launch_attn(const AttnLaunch &a, cudaStream_t st)
+{
+    const bool weighted = a.w != nullptr;
+    if (a.d == 128) return weighted ? launch_attn_o<128, true>(a, st) : launch_attn_o<128, false>(a, st);
+    return weighted ? launch_attn_o<64, true>(a, st) : launch_attn_o<64, false>(a, st);
+}
+
+}  // namespace ab

@@ -1,0 +1,347 @@
+// select_kernels.cu -- key-block selection per query block on sm_100a.
+//
+// SIP (AB-Attention news page, section «Три приёма AB-Attention», second technique):
+// inclusion probability p_j = min(1, c s_j) with sum p_j = K, the top blocks always
+// kept, each kept block weighted by 1/p_j. Solved exactly in integers on the fixed
+// point u_j = floor(s_j 2^50) so every implementation reproduces the same bits; draws
+// from Philox4x32-10 (Salmon et al., SC'11) keyed by the seed, counter (j, qb, h, b).
+// Top-k (section «Где ломаются прежние разреженные схемы»): the K largest scores, ties
+// to the lower index, found by an MSB-first radix select on the score bits.
+// One CTA of 256 threads per (b, h, qb) row; kept blocks are compacted in ascending
+// order with warp ballots and a block-wide prefix.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "ab_device.cuh"
+#include "ab_kernels.h"
+
+namespace ab {
+
+constexpr int kSelThreads = 256;
+constexpr int kSelWarps = kSelThreads / 32;
+
+// Philox4x32-10: ten rounds of the 4x32 S-box, key bumped by the Weyl constants
+// 0x9E3779B9 / 0xBB67AE85 between rounds, round multipliers 0xD2511F53 / 0xCD9E8D57.
+__device__ __forceinline__ uint4 philox_4x32_10(uint4 c, uint32_t k0, uint32_t k1)
+{
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+        const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return c;
+}
+
+__device__ __forceinline__ bool score_ok(float v) { return v >= 0.f && v <= 2.f; }
+
+// exact: v in [0, 2] -> floor(v * 2^50) < 2^52
+__device__ __forceinline__ uint64_t fixed50(float v)
+{
+    return __double2ull_rz((double)v * 1125899906842624.0);
+}
+
+// k * u >= R with a 128-bit product
+__device__ __forceinline__ bool mul_ge(uint64_t k, uint64_t u, uint64_t R)
+{
+    return __umul64hi(k, u) != 0ull || k * u >= R;
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Block-wide sums of (a, b, c); every thread gets the totals.
+struct Sum3 {
+    unsigned long long a, b, c;
+};
+
+__device__ Sum3 block_sum3(unsigned long long a, unsigned long long b, unsigned long long c,
+                           unsigned long long (*red)[3])
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    a = warp_sum(a);
+    b = warp_sum(b);
+    c = warp_sum(c);
+    __syncthreads();
+    if (lane == 0) {
+        red[warp][0] = a;
+        red[warp][1] = b;
+        red[warp][2] = c;
+    }
+    __syncthreads();
+    Sum3 s{0, 0, 0};
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) {
+        s.a += red[w][0];
+        s.b += red[w][1];
+        s.c += red[w][2];
+    }
+    return s;
+}
+
+// Ordered compaction step: returns the exclusive position of this thread's element
+// among the kept elements of the current chunk and writes the chunk total to *total.
+__device__ __forceinline__ int chunk_prefix(bool keep, int *wtot, int *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned m = __ballot_sync(0xffffffffu, keep);
+    __syncthreads();
+    if (lane == 0) wtot[warp] = __popc(m);
+    __syncthreads();
+    int before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) {
+        const int t = wtot[w];
+        before += (w < warp) ? t : 0;
+        all += t;
+    }
+    *total = all;
+    return before + __popc(m & ((1u << lane) - 1u));
+}
+
+__global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restrict__ scores,
+                                                         int H, int nqb, int nkb, int K,
+                                                         uint32_t key0, uint32_t key1,
+                                                         int32_t *__restrict__ idx,
+                                                         int32_t *__restrict__ cnt,
+                                                         float *__restrict__ w,
+                                                         double *__restrict__ p_out, int *flag)
+{
+    extern __shared__ uint8_t inS[];  // nkb bytes: 0 = out, 1 = saturated, 2 = joining
+    __shared__ unsigned long long red[kSelWarps][3];
+    __shared__ int wtot[kSelWarps];
+
+    const size_t row = blockIdx.x;
+    const int b = (int)(row / ((size_t)H * nqb));
+    const int h = (int)((row / nqb) % H);
+    const int qb = (int)(row % nqb);
+    const float *s = scores + row * nkb;
+    const int tid = threadIdx.x;
+
+    // pass 0: validate, U = sum u_j, number of positive u_j
+    unsigned long long U = 0, npos = 0, nbad = 0;
+    for (int j = tid; j < nkb; j += kSelThreads) {
+        const float v = s[j];
+        inS[j] = 0;
+        if (!score_ok(v)) {
+            ++nbad;
+            continue;
+        }
+        const uint64_t u = fixed50(v);
+        U += u;
+        npos += u > 0;
+    }
+    Sum3 t = block_sum3(U, npos, nbad, red);
+    U = t.a;
+    npos = t.b;
+    if (t.c != 0) {
+        for (int j = tid; j < nkb; j += kSelThreads) {
+            idx[row * nkb + j] = -1;
+            w[row * nkb + j] = 0.f;
+            if (p_out) p_out[row * nkb + j] = 0.0;
+        }
+        if (tid == 0) {
+            cnt[row] = 0;
+            raise_flag(flag, AB_FLAG_BAD_SCORE);
+        }
+        return;
+    }
+
+    // saturated set S by the fixed point S <- S + {j : (K-|S|) u_j >= U - sum_S u}
+    const bool all_positive_kept = npos <= (unsigned long long)K;
+    uint64_t k_rest = 0, R = 0;
+    if (all_positive_kept) {
+        for (int j = tid; j < nkb; j += kSelThreads) inS[j] = fixed50(s[j]) > 0 ? 1 : 0;
+        __syncthreads();
+    } else {
+        unsigned long long sizeS = 0, sumS = 0;
+        for (;;) {
+            k_rest = (uint64_t)K - sizeS;
+            R = U - sumS;
+            unsigned long long add_n = 0, add_u = 0;
+            for (int j = tid; j < nkb; j += kSelThreads) {
+                if (inS[j]) continue;
+                const uint64_t u = fixed50(s[j]);
+                if (mul_ge(k_rest, u, R)) {
+                    inS[j] = 2;
+                    ++add_n;
+                    add_u += u;
+                }
+            }
+            t = block_sum3(add_n, add_u, 0, red);
+            if (t.a == 0) break;
+            sizeS += t.a;
+            sumS += t.b;
+            for (int j = tid; j < nkb; j += kSelThreads)
+                if (inS[j] == 2) inS[j] = 1;
+            __syncthreads();
+        }
+    }
+
+    // probabilities, draws, ordered compaction
+    const double Rd = __ull2double_rn(R);
+    int base = 0;
+    for (int j0 = 0; j0 < nkb; j0 += kSelThreads) {
+        const int j = j0 + tid;
+        bool keep = false;
+        double pj = 0.0;
+        if (j < nkb) {
+            if (inS[j] == 1) {
+                pj = 1.0;
+            } else if (!all_positive_kept) {
+                const uint64_t u = fixed50(s[j]);
+                if (u > 0) pj = __ull2double_rn(k_rest * u) / Rd;
+            }
+            if (p_out) p_out[row * nkb + j] = pj;
+            const uint4 x = philox_4x32_10(make_uint4((uint32_t)j, (uint32_t)qb, (uint32_t)h,
+                                                      (uint32_t)b),
+                                           key0, key1);
+            const uint64_t r53 = ((((uint64_t)x.x) << 32) | x.y) >> 11;
+            keep = __ull2double_rn(r53) < pj * 9007199254740992.0;
+        }
+        int total;
+        const int pos = chunk_prefix(keep, wtot, &total);
+        if (keep) {
+            idx[row * nkb + base + pos] = j;
+            w[row * nkb + base + pos] = __double2float_rn(1.0 / pj);
+        }
+        base += total;
+    }
+    for (int c = base + tid; c < nkb; c += kSelThreads) {
+        idx[row * nkb + c] = -1;
+        w[row * nkb + c] = 0.f;
+    }
+    if (tid == 0) cnt[row] = base;
+}
+
+__global__ void __launch_bounds__(kSelThreads) topk_kernel(const float *__restrict__ scores,
+                                                          int nkb, int K,
+                                                          int32_t *__restrict__ idx,
+                                                          int32_t *__restrict__ cnt,
+                                                          float *__restrict__ w, int *flag)
+{
+    extern __shared__ uint32_t keys[];  // nkb score bit patterns (order-preserving for s >= 0)
+    __shared__ unsigned long long red[kSelWarps][3];
+    __shared__ int hist[256];
+    __shared__ int wtot[kSelWarps];
+    __shared__ uint32_t sel_digit;
+    __shared__ int sel_rem;
+
+    const size_t row = blockIdx.x;
+    const float *s = scores + row * nkb;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    unsigned long long nbad = 0;
+    for (int j = tid; j < nkb; j += kSelThreads) {
+        const float v = s[j];
+        if (!score_ok(v)) ++nbad;
+        keys[j] = __float_as_uint(v + 0.0f);  // -0 -> +0
+    }
+    const Sum3 t = block_sum3(nbad, 0, 0, red);
+    if (t.a != 0) {
+        for (int j = tid; j < nkb; j += kSelThreads) {
+            idx[row * nkb + j] = -1;
+            if (w) w[row * nkb + j] = 0.f;
+        }
+        if (tid == 0) {
+            cnt[row] = 0;
+            raise_flag(flag, AB_FLAG_BAD_SCORE);
+        }
+        return;
+    }
+
+    // K-th largest key by MSB-first radix select, 8-bit digits
+    uint32_t prefix = 0, mask = 0;
+    int rem = K;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int e = tid; e < 256; e += kSelThreads) hist[e] = 0;
+        __syncthreads();
+        for (int j = tid; j < nkb; j += kSelThreads) {
+            const uint32_t key = keys[j];
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // lane l owns digits 255-8l .. 248-8l (descending)
+            int local = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) local += hist[255 - 8 * lane - e];
+            int incl = local;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const int excl = incl - local;
+            if (excl < rem && incl >= rem) {
+                int acc = excl;
+                for (int e = 0; e < 8; ++e) {
+                    const int dgt = 255 - 8 * lane - e;
+                    if (acc + hist[dgt] >= rem) {
+                        sel_digit = (uint32_t)dgt;
+                        sel_rem = rem - acc;
+                        break;
+                    }
+                    acc += hist[dgt];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= sel_digit << shift;
+        mask |= 255u << shift;
+        rem = sel_rem;
+        __syncthreads();
+    }
+    // keep key > T, plus the first `rem` keys equal to T in index order
+    const uint32_t T = prefix;
+    int base = 0, eq_base = 0;
+    for (int j0 = 0; j0 < nkb; j0 += kSelThreads) {
+        const int j = j0 + tid;
+        const uint32_t key = j < nkb ? keys[j] : 0u;
+        const bool eq = j < nkb && key == T;
+        int eq_total;
+        const int eq_pos = chunk_prefix(eq, wtot, &eq_total);
+        const bool keep = j < nkb && (key > T || (eq && eq_base + eq_pos < rem));
+        eq_base += eq_total;
+        int total;
+        const int pos = chunk_prefix(keep, wtot, &total);
+        if (keep) {
+            idx[row * nkb + base + pos] = j;
+            if (w) w[row * nkb + base + pos] = 1.0f;
+        }
+        base += total;
+    }
+    for (int c = base + tid; c < nkb; c += kSelThreads) {
+        idx[row * nkb + c] = -1;
+        if (w) w[row * nkb + c] = 0.f;
+    }
+    if (tid == 0) cnt[row] = base;
+}
+
+cudaError_t launch_sip(const float *scores, int B, int H, int nqb, int nkb, int K, uint64_t seed,
+                       int32_t *idx, int32_t *cnt, float *w, double *p, int *flag, cudaStream_t st)
+{
+    const unsigned rows = (unsigned)((size_t)B * H * nqb);
+    sip_kernel<<<rows, kSelThreads, (size_t)nkb, st>>>(scores, H, nqb, nkb, K, (uint32_t)seed,
+                                                       (uint32_t)(seed >> 32), idx, cnt, w, p,
+                                                       flag);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const float *scores, int B, int H, int nqb, int nkb, int K, int32_t *idx,
+                        int32_t *cnt, float *w, int *flag, cudaStream_t st)
+{
+    const unsigned rows = (unsigned)((size_t)B * H * nqb);
+    topk_kernel<<<rows, kSelThreads, (size_t)nkb * sizeof(uint32_t), st>>>(scores, nkb, K, idx,
+                                                                            cnt, w, flag);
+    return cudaGetLastError();
+}
+
+}  // namespace ab

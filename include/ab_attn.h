@@ -1,0 +1,196 @@
+/*
+ * ab_attn.h -- C ABI of the AB-Attention hot path on NVIDIA B200 (sm_100a).
+ *
+ * The method is described on the news page "AB-Attention ускорил генерацию видео до
+ * 2,23× и пропускает 92% внимания" (app.hamidun.com), section «Три приёма AB-Attention»:
+ * score key blocks (IBCS), sample them (SIP), and run softmax attention over the
+ * sampled blocks, gathered by index, with a logit shift. The page's section «Где
+ * ломаются прежние разреженные схемы» describes the top-k baseline.
+ *
+ * Conventions shared by every call
+ *   - Token tensors Q, K, V, O are contiguous bf16 arrays [B, H, N_pad, d] (BHND,
+ *     row-major). N is the number of valid tokens, N_pad = N rounded up to a multiple
+ *     of 128 (the block size). Rows t >= N are never read as data (the kernels treat
+ *     them as absent) and are written as 0 on output.
+ *   - n_qb = n_kb = N_pad / 128 query / key blocks of 128 tokens each.
+ *   - Every pointer argument except `stream` is a DEVICE pointer on the current
+ *     device, allocated and owned by the caller, 16-byte aligned. The library
+ *     allocates no device memory and keeps no state between calls; the only
+ *     host-side work is argument validation and building TMA tensor maps.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
+ *     enqueues work on it and returns; results are ready when the stream is.
+ *   - Argument errors are reported synchronously by the return value and nothing is
+ *     enqueued. Problems only the device can see (a bad score, an out-of-range block
+ *     index, a bounded wait that gave up) are OR-ed as AB_FLAG_* bits into the
+ *     optional `dev_flag` int (caller-allocated, caller-zeroed); read it back with
+ *     ab_check_flag().
+ */
+#ifndef AB_ATTN_H
+#define AB_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AB_OK = 0,
+    AB_ERR_NULL = 1,        /* a required pointer is NULL */
+    AB_ERR_SHAPE = 2,       /* inconsistent or non-positive sizes */
+    AB_ERR_DTYPE = 3,       /* token tensors must be AB_BF16 */
+    AB_ERR_UNSUPPORTED = 4, /* head dim other than 64 / 128, clusters outside 1..8, ... */
+    AB_ERR_RANGE = 5,       /* budget < 1, iters < 1, too many blocks */
+    AB_ERR_CUDA = 6,        /* a CUDA runtime / driver call or launch failed */
+    AB_ERR_DEVICE_FLAG = 7, /* ab_check_flag: the device flag is non-zero */
+    AB_ERR_TIMEOUT = 8,     /* ab_check_flag: a kernel's bounded wait gave up */
+    AB_ERR_ALIGN = 9,       /* a pointer is not 16-byte aligned */
+    AB_ERR_WORKSPACE = 10   /* workspace NULL or smaller than ab_score_workspace_size */
+} ab_status;
+
+typedef enum { AB_F32 = 0, AB_BF16 = 1 } ab_dtype;
+
+typedef enum {
+    AB_MODE_SIP = 0, /* sampling with inclusion-probability weights */
+    AB_MODE_TOPK = 1 /* deterministic top-k, all weights 1 */
+} ab_mode;
+
+/* Shape of the token tensors (BHND, contiguous). dtype must be AB_BF16. */
+typedef struct {
+    int32_t B, H, N, N_pad, d;
+    int32_t dtype; /* ab_dtype */
+} ab_shape;
+
+/* Bits OR-ed into *dev_flag by the kernels. */
+#define AB_FLAG_BAD_SCORE 1u  /* ab_select: a score is NaN, infinite, < 0 or > 2 */
+#define AB_FLAG_BAD_INDEX 2u  /* ab_attn_*: a cnt or idx entry outside its range */
+#define AB_FLAG_BAD_WEIGHT 4u /* ab_attn_fwd: a weight is NaN, infinite or <= 0 */
+#define AB_FLAG_TIMEOUT 8u    /* a bounded in-kernel wait gave up (pipeline stalled) */
+
+/* Limits: head dim d in {64, 128}; 1 <= n_kb <= 8192 (N_pad <= 1,048,576). */
+#define AB_BLOCK 128
+#define AB_MAX_BLOCKS 8192
+
+/*
+ * ab_score_workspace_size -- bytes of device scratch ab_score() needs for shape `s`
+ * and `n_clusters`: the mean keys [B,H,n_kb,d] fp32, the centroids [B,H,n_qb,C,d] fp32
+ * and the cluster weights [B,H,n_qb,C] fp32, each region 256-byte aligned.
+ * Returns AB_ERR_* for an invalid shape; *bytes is then 0.
+ */
+ab_status ab_score_workspace_size(ab_shape s, int n_clusters, size_t *bytes);
+
+/*
+ * ab_score -- IBCS block scores (page section «Три приёма AB-Attention», first
+ * technique). For every query block qb of 128 tokens:
+ *   1. kbar_j = mean of the valid keys of key block j;
+ *   2. k-means of the block's valid queries into C = n_clusters clusters, `iters`
+ *      Lloyd iterations (assign to the nearest centroid in squared Euclidean
+ *      distance, ties to the lowest cluster; update to the member mean, an empty
+ *      cluster keeps its centroid); the initial centroid c is the query at
+ *      block-local index c*floor(n_v/C) (min(c, n_v-1) when n_v < C); the weight of a
+ *      cluster is its share of the block's valid queries;
+ *   3. scores[qb][j] = sum_c w_c softmax_j(cent_c . kbar_j / sqrt(d)), the softmax
+ *      taken over all n_kb key blocks.
+ * q, k       : bf16 [B,H,N_pad,d], s.dtype == AB_BF16, d in {64,128}.
+ * n_clusters : 1..8 (8 is the method's value; 1 gives mean-pooled block scores).
+ * iters      : >= 1 Lloyd iterations (5 in the method's configuration).
+ * scores     : out, fp32 [B,H,n_qb,n_kb]; each row sums to 1.
+ * kbar, centroids, cweights, assign : optional outputs (NULL to skip): fp32
+ *              [B,H,n_kb,d], fp32 [B,H,n_qb,C,d], fp32 [B,H,n_qb,C], uint8 [B,H,N_pad]
+ *              (cluster of each query after the last assignment, 255 on padding rows).
+ * workspace  : device scratch of at least ab_score_workspace_size() bytes, owned by
+ *              the caller, contents need not be initialised, not read after return.
+ * dev_flag   : optional (see above).
+ * Errors: AB_ERR_NULL, AB_ERR_SHAPE, AB_ERR_DTYPE, AB_ERR_UNSUPPORTED, AB_ERR_RANGE,
+ * AB_ERR_ALIGN, AB_ERR_WORKSPACE, AB_ERR_CUDA.
+ */
+ab_status ab_score(const void *q, const void *k, ab_shape s, int n_clusters, int iters,
+                   float *scores, float *kbar, float *centroids, float *cweights,
+                   uint8_t *assign, void *workspace, size_t workspace_bytes, int *dev_flag,
+                   void *stream);
+
+/*
+ * ab_select -- choose key blocks per query block (page section «Три приёма
+ * AB-Attention», second technique SIP; section «Где ломаются прежние разреженные
+ * схемы» for top-k).
+ * AB_MODE_SIP: inclusion probabilities p_j = min(1, c s_j) with sum p_j = K =
+ *   min(budget, n_kb), solved exactly in integers on u_j = floor(s_j 2^50): the
+ *   saturated set S grows from empty by S <- S + {j : (K-|S|) u_j >= U - sum_S u} until
+ *   stable (if at most K blocks have u_j > 0, exactly those are kept with p = 1);
+ *   p_j = 1 on S, else (double)((K-|S|) u_j) / (double)(U - sum_S u). Block j is kept
+ *   iff (double)R < p_j 2^53, where R = ((x0 << 32) | x1) >> 11 and (x0, x1) are the
+ *   first two words of Philox4x32-10 with key (seed & 0xffffffff, seed >> 32) and
+ *   counter (j, qb, h, b). Kept blocks carry w = (float)(1 / p_j), so a block drawn
+ *   with p = 1/4 counts four times.
+ * AB_MODE_TOPK: the K blocks with the largest scores (ties to the lower index),
+ *   weights 1.
+ * scores : fp32 [B,H,nqb,nkb], every entry finite and in [0, 2].
+ * idx    : out, int32 [B,H,nqb,nkb]: kept block indices in ascending order in the
+ *          first cnt entries of each row, -1 after them.
+ * cnt    : out, int32 [B,H,nqb].
+ * w      : out, fp32 [B,H,nqb,nkb] aligned with idx (0 after cnt); required for SIP,
+ *          optional (NULL) for top-k.
+ * p      : optional out, fp64 [B,H,nqb,nkb]: p_j by block index (SIP only).
+ * A row with an invalid score sets AB_FLAG_BAD_SCORE and gets cnt = 0, idx = -1.
+ * Errors: AB_ERR_NULL, AB_ERR_SHAPE, AB_ERR_RANGE (budget < 1, nkb > AB_MAX_BLOCKS),
+ * AB_ERR_ALIGN, AB_ERR_CUDA.
+ */
+ab_status ab_select(const float *scores, int B, int H, int nqb, int nkb, int budget,
+                    ab_mode mode, uint64_t seed, int32_t *idx, int32_t *cnt, float *w,
+                    double *p, int *dev_flag, void *stream);
+
+/*
+ * ab_attn_fwd -- block-sparse softmax attention over the selected key blocks with
+ * Horvitz-Thompson weights (page section «Три приёма AB-Attention», SIP and the third
+ * technique: the kernel gathers the chosen blocks by index, tokens stay in order, the
+ * weights enter as a logit shift). For query i of block qb, over the kept blocks j and
+ * their valid keys t < N:
+ *   O_i = sum_j w_j sum_t e^{q_i.k_t/sqrt(d)} v_t / sum_j w_j sum_t e^{q_i.k_t/sqrt(d)}
+ * computed as online softmax of q_i.k_t/sqrt(d) + ln w_j.
+ * q, k, v : bf16 [B,H,N_pad,d], d in {64,128}.
+ * idx, cnt, w : the plan from ab_select (row stride n_kb); every w_j must be > 0.
+ * out     : [B,H,N_pad,d] in `out_dtype` (AB_BF16 or AB_F32); rows t >= N and rows of
+ *           an empty selection are 0.
+ * lse     : optional fp32 [B,H,N_pad]: ln of the denominator (0 on padding rows,
+ *           -inf for an empty selection).
+ * Device-side: an idx/cnt outside range sets AB_FLAG_BAD_INDEX (the block is clamped
+ * into range), a bad weight sets AB_FLAG_BAD_WEIGHT.
+ * Errors: AB_ERR_NULL, AB_ERR_SHAPE, AB_ERR_DTYPE (inputs not bf16, or out_dtype not
+ * AB_BF16 / AB_F32), AB_ERR_UNSUPPORTED, AB_ERR_ALIGN, AB_ERR_CUDA.
+ */
+ab_status ab_attn_fwd(const void *q, const void *k, const void *v, ab_shape s,
+                      const int32_t *idx, const int32_t *cnt, const float *w, void *out,
+                      ab_dtype out_dtype, float *lse, int *dev_flag, void *stream);
+
+/*
+ * ab_attn_topk_fwd -- the same attention with every weight 1 (no logit shift): the
+ * top-k baseline, where a dropped block leaves both the numerator and the softmax
+ * normaliser (page section «Где ломаются прежние разреженные схемы»). Takes the
+ * idx / cnt of ab_select(..., AB_MODE_TOPK, ...). Arguments and errors as ab_attn_fwd.
+ */
+ab_status ab_attn_topk_fwd(const void *q, const void *k, const void *v, ab_shape s,
+                           const int32_t *idx, const int32_t *cnt, void *out, ab_dtype out_dtype,
+                           float *lse, int *dev_flag, void *stream);
+
+/*
+ * ab_check_flag -- synchronise `stream`, copy *dev_flag to *host_flag and map it to a
+ * status: AB_OK (0), AB_ERR_TIMEOUT (AB_FLAG_TIMEOUT set) or AB_ERR_DEVICE_FLAG.
+ */
+ab_status ab_check_flag(const int *dev_flag, int *host_flag, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *ab_status_str(ab_status s);
+
+/* The CUDA error string behind the calling thread's most recent AB_ERR_CUDA (static
+ * storage; "no error" if the thread has seen none). */
+const char *ab_last_cuda_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int ab_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AB_ATTN_H */

@@ -1,0 +1,137 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point that
+include/ab_attn.h declares, and rejects bad arguments synchronously with the documented
+status codes. Nothing here launches a kernel, so it runs without a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_ab_b200 as ab
+from block_sparse_attention_ab_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ab_attn.h")
+
+FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: every call below fails first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ab.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ab_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert {"ab_score", "ab_select", "ab_attn_fwd", "ab_attn_topk_fwd"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code, name in ab.STATUS.items():
+        assert L.ab_status_str(code).decode() == name
+    assert L.ab_version() >= 100
+
+
+def shape(B=1, H=2, N=1000, N_pad=1024, d=64, dtype=ab.AB_BF16):
+    return ab.Shape(B, H, N, N_pad, d, dtype)
+
+
+def test_workspace_size(L):
+    n = ctypes.c_size_t(0)
+    assert L.ab_score_workspace_size(shape(), 8, ctypes.byref(n)) == 0
+    nb = 8
+    need = 2 * nb * 64 * 4 + 2 * nb * 8 * 64 * 4 + 2 * nb * 8 * 4
+    assert need <= n.value <= need + 3 * 256
+    assert L.ab_score_workspace_size(shape(), 9, ctypes.byref(n)) == 4
+    assert n.value == 0
+    assert L.ab_score_workspace_size(shape(N=1024, N_pad=1000), 8, ctypes.byref(n)) == 2
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(B=0), 2), (dict(N=0), 2), (dict(N_pad=1000), 2), (dict(N=1025), 2),
+    (dict(N=800), 2),  # N_pad - N >= 128
+    (dict(dtype=0), 3), (dict(d=96), 4), (dict(d=256), 4),
+    (dict(N=128 * 8193, N_pad=128 * 8193), 5),
+])
+def test_shape_rejections(L, bad, code):
+    s = shape(**bad)
+    assert L.ab_attn_topk_fwd(FAKE, FAKE, FAKE, s, FAKE, FAKE, FAKE, ab.AB_BF16, None, None,
+                              None) == code
+    assert L.ab_attn_fwd(FAKE, FAKE, FAKE, s, FAKE, FAKE, FAKE, FAKE, ab.AB_F32, None, None,
+                         None) == code
+    assert L.ab_score(FAKE, FAKE, s, 8, 5, FAKE, None, None, None, None, FAKE, 1 << 40, None,
+                      None) == code
+
+
+def test_null_and_alignment(L):
+    s = shape()
+    B16 = ab.AB_BF16
+    assert L.ab_attn_fwd(None, FAKE, FAKE, s, FAKE, FAKE, FAKE, FAKE, B16, None, None, None) == 1
+    assert L.ab_attn_fwd(FAKE, FAKE, FAKE, s, FAKE, FAKE, None, FAKE, B16, None, None, None) == 1
+    assert L.ab_attn_fwd(FAKE, MISALIGNED, FAKE, s, FAKE, FAKE, FAKE, FAKE, B16, None, None,
+                         None) == 9
+    assert L.ab_attn_fwd(FAKE, FAKE, FAKE, s, FAKE, FAKE, FAKE, FAKE, 7, None, None, None) == 3
+    assert L.ab_attn_topk_fwd(FAKE, FAKE, FAKE, s, FAKE, FAKE, FAKE, 2, None, None, None) == 3
+    assert L.ab_score(FAKE, FAKE, s, 8, 5, None, None, None, None, None, FAKE, 1 << 40, None,
+                      None) == 1
+    assert L.ab_score(FAKE, FAKE, s, 8, 5, MISALIGNED, None, None, None, None, FAKE, 1 << 40,
+                      None, None) == 9
+
+
+def test_score_argument_checks(L):
+    s = shape()
+    n = ctypes.c_size_t(0)
+    L.ab_score_workspace_size(s, 8, ctypes.byref(n))
+    assert L.ab_score(FAKE, FAKE, s, 0, 5, FAKE, None, None, None, None, FAKE, n.value, None,
+                      None) == 4
+    assert L.ab_score(FAKE, FAKE, s, 8, 0, FAKE, None, None, None, None, FAKE, n.value, None,
+                      None) == 5
+    assert L.ab_score(FAKE, FAKE, s, 8, 5, FAKE, None, None, None, None, None, n.value, None,
+                      None) == 10
+    assert L.ab_score(FAKE, FAKE, s, 8, 5, FAKE, None, None, None, None, FAKE, n.value - 1,
+                      None, None) == 10
+
+
+def test_select_argument_checks(L):
+    u = ctypes.c_uint64(0)
+    assert L.ab_select(None, 1, 1, 8, 8, 3, 0, u, FAKE, FAKE, FAKE, None, None, None) == 1
+    assert L.ab_select(FAKE, 1, 1, 8, 8, 3, 0, u, FAKE, FAKE, None, None, None, None) == 1
+    assert L.ab_select(FAKE, 1, 1, 8, 8, 3, 7, u, FAKE, FAKE, FAKE, None, None, None) == 4
+    assert L.ab_select(FAKE, 0, 1, 8, 8, 3, 0, u, FAKE, FAKE, FAKE, None, None, None) == 2
+    assert L.ab_select(FAKE, 1, 1, 8, 8, 0, 0, u, FAKE, FAKE, FAKE, None, None, None) == 5
+    assert L.ab_select(FAKE, 1, 1, 8, 8193, 3, 1, u, FAKE, FAKE, None, None, None, None) == 5
+    assert L.ab_select(MISALIGNED, 1, 1, 8, 8, 3, 1, u, FAKE, FAKE, None, None, None, None) == 9
+
+
+def test_check_flag_null(L):
+    host = ctypes.c_int(0)
+    assert L.ab_check_flag(None, ctypes.byref(host), None) == 1
+
+
+def test_product_path_has_no_fallback(monkeypatch, tmp_path):
+    """Without the shared library the binding raises instead of computing on the CPU."""
+    monkeypatch.setattr(ab, "_lib", None)
+    monkeypatch.setattr(ab, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        ab.lib()
+
+
+def test_product_package_does_not_reference_the_oracle():
+    pkg = os.path.join(ROOT, "block_sparse_attention_ab_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", text, re.M), f
+                assert "liboracle" not in text and "ab_oracle" not in text, f
