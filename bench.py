@@ -27,6 +27,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +37,24 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 L2_BYTES = 126 * 2**20
+
+
+def attn_traffic_from_profile():
+    """DRAM bytes per attention launch recorded in profiles/attn_fwd_wan13b.md, or None
+    when the kernel source changed since that capture (hash mismatch)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "attn_fwd_wan13b.md")
+    csrc = os.path.join(ROOT, "block_sparse_attention_ab_b200", "csrc")
+    try:
+        rec = dict(line.split(":", 1) for line in open(path) if line.startswith(("traffic_bytes", "kernel_source")))
+        h = hashlib.sha256()
+        for f in ("attn_kernel.cu", "ab_device.cuh"):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+        if h.hexdigest()[:16] != rec["kernel_source_sha256_16"].strip():
+            return None
+        return float(rec["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def measured_peaks():
@@ -60,11 +79,10 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"ab_bench_clocks_{os.getpid()}_{device_index}.csv")
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
@@ -284,7 +302,8 @@ def run_ours(args, rank, world, local_rank):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(sel / (attn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} bf16 dense burst",
-                     "traffic": args.traffic},
+                     "traffic": args.traffic if args.traffic is not None else attn_traffic_from_profile(),
+                     "algorithmic_bytes": 4 * q.numel() * 2},
         "score_roofline": {"bound": "hbm",
                            "achieved": round((2 * q.numel() * 2 + scores.numel() * 4) /
                                              (float(np.mean(stage_ms[:, 0])) * 1e-3) / 1e9, 1),

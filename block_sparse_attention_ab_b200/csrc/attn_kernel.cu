@@ -364,12 +364,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             wait_bar(o_full, k & 1);
             o_seen = k + 1;
         };
-        auto block_lw = [&](float wj) -> float {
+        auto lw_of = [&](float wj) -> float {  // log2 of a block weight (0 for top-k)
             if (!kWeighted) return 0.f;
-            if (wj > 0.f && wj < INFINITY) return log2f(wj);
+            if (wj > 0.f && wj < INFINITY) return fast_log2(wj);
             if (warp == 0 && lane == 0) raise_flag(p.flag, AB_FLAG_BAD_WEIGHT);
             return 0.f;
         };
+        auto clamp_j = [&](int j) { return j < 0 ? 0 : (j >= p.nkb ? p.nkb - 1 : j); };
         constexpr int kHalfD = D / 2;
         constexpr int kSoftPairs = 6;  // of 32 pairs per block: exp2 on the FMA pipe
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
@@ -394,14 +395,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             const int32_t *idx_row = p.idx + (size_t)r * p.nkb;
             const float *w_row = kWeighted ? p.w + (size_t)r * p.nkb : nullptr;
-            int j_next = __ldg(idx_row);
-            float w_next = kWeighted ? __ldg(w_row) : 1.f;
+            // the block's index and log2 weight are ready before the block starts: the
+            // next block's are loaded during this one and converted after its P is out
+            int j = clamp_j(__ldg(idx_row));
+            float lw = lw_of(kWeighted ? __ldg(w_row) : 1.f);
             float m_run = -INFINITY, l_run = 0.f;
             for (int i = 0; i < n; ++i, ++g) {
-                int j = j_next;
-                if (j < 0 || j >= p.nkb) j = j < 0 ? 0 : p.nkb - 1;
-                const float lw = block_lw(w_next);
-                if (i + 1 < n) {  // prefetch the next block's index and weight
+                int j_next = 0;
+                float w_next = 1.f;
+                if (i + 1 < n) {
                     j_next = __ldg(idx_row + i + 1);
                     if (kWeighted) w_next = __ldg(w_row + i + 1);
                 }
@@ -495,6 +497,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (g > 0) wait_o(g - 1);
                 tc_fence_before();
                 mbar_arrive(&p_full[g & 1]);
+                if (i + 1 < n) {
+                    j = clamp_j(j_next);
+                    lw = lw_of(w_next);
+                }
 
                 if (i == n - 1) {
                     // epilogue: O / l (l summed over both halves), straight to global memory
