@@ -69,6 +69,7 @@ def lib():
         P, I, S = ctypes.c_void_p, ctypes.c_int, Shape
         L.ab_score_workspace_size.argtypes = [S, I, ctypes.POINTER(ctypes.c_size_t)]
         L.ab_score.argtypes = [P, P, S, I, I, P, P, P, P, P, P, ctypes.c_size_t, P, P]
+        L.ab_score_noalloc.argtypes = [P, P, S, I, I, P, P, P]
         L.ab_select.argtypes = [P, I, I, I, I, I, I, ctypes.c_uint64, P, P, P, P, P, P]
         L.ab_attn_fwd.argtypes = [P, P, P, S, P, P, P, P, I, P, P, P]
         L.ab_attn_topk_fwd.argtypes = [P, P, P, S, P, P, P, I, P, P, P]
@@ -78,7 +79,7 @@ def lib():
         L.ab_version.argtypes = []
         L.ab_last_cuda_error.argtypes = []
         L.ab_last_cuda_error.restype = ctypes.c_char_p
-        for name in ("ab_score_workspace_size", "ab_score", "ab_select", "ab_attn_fwd",
+        for name in ("ab_score_workspace_size", "ab_score", "ab_score_noalloc", "ab_select", "ab_attn_fwd",
                      "ab_attn_topk_fwd", "ab_check_flag", "ab_version"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -143,6 +144,20 @@ def score(q: torch.Tensor, k: torch.Tensor, N: int, n_clusters: int = 8, iters: 
                           workspace.numel(), None, _stream()), "ab_score")
     if intermediates:
         return scores, kbar, cent, cw, assign
+    return scores
+
+
+def score_noalloc(q: torch.Tensor, k: torch.Tensor, N: int, n_clusters: int = 8, iters: int = 5,
+                  out: Optional[torch.Tensor] = None):
+    """IBCS block scores through ab_score_noalloc: no workspace argument; the library's
+    fixed device scratch is used (see include/ab_attn.h for its size limit)."""
+    _need(q, torch.bfloat16, "q")
+    _need(k, torch.bfloat16, "k")
+    B, H, N_pad, d = q.shape
+    nb = N_pad // BLOCK
+    scores = out if out is not None else torch.empty(B, H, nb, nb, device=q.device, dtype=torch.float32)
+    _check(lib().ab_score_noalloc(_ptr(q), _ptr(k), make_shape(q, N), n_clusters, iters,
+                                  _ptr(scores), None, _stream()), "ab_score_noalloc")
     return scores
 
 

@@ -111,6 +111,32 @@ ab_status ab_score(const void *q, const void *k, ab_shape s, int n_clusters, int
                    void *stream);
 
 /*
+ * ab_score_noalloc -- ab_score for callers that cannot allocate device memory. The
+ * method's pages have no counterpart to this call; it exists for integration only.
+ * Some callers cannot call cudaMalloc or hand the library a workspace: a plugin or
+ * custom operator running inside a host framework that owns all device memory and
+ * forbids allocation on its execution path, or code that has no allocator of its own.
+ * This call computes exactly what ab_score computes (scores only; no optional
+ * outputs), with its scratch (mean keys, centroids, cluster weights) in a fixed array
+ * of AB_NOALLOC_SCRATCH_BYTES bytes in the library's own device memory. That array
+ * exists once on every GPU that loads the library and stays allocated until the
+ * process exits. The call itself allocates nothing.
+ *   - Scratch needed = ab_score_workspace_size(s, n_clusters); larger problems are
+ *     rejected with AB_ERR_WORKSPACE (e.g. 12 heads x 32768 tokens, d = 128, C = 8
+ *     needs 14.3 MB and fits; 24 heads x 118912 tokens does not).
+ *   - The first call on each device looks up the array's device address (with that
+ *     device current) and caches it; make that first call before any stream capture.
+ *   - Every call uses the same array and leaves its contents behind; every region is
+ *     rewritten before it is read, so no clearing is needed. Calls that overlap on the
+ *     GPU (different streams, or different host threads) race on the array: serialise
+ *     them, e.g. on one stream.
+ * Other arguments, conventions and errors as ab_score.
+ */
+#define AB_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, int n_clusters, int iters,
+                           float *scores, int *dev_flag, void *stream);
+
+/*
  * ab_select -- choose key blocks per query block (page section «Три приёма
  * AB-Attention», second technique SIP; section «Где ломаются прежние разреженные
  * схемы» for top-k).
