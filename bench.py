@@ -133,6 +133,27 @@ def workload(name: str):
     return synth.WORKLOADS[name]
 
 
+def rank_workload(name: str, rank: int, world: int, heads: int = 0):
+    """The workload a rank runs: every rank gets the same shape on its own data (weak
+    scaling over independent batches; the method has no cross-rank exchange)."""
+    import dataclasses
+    w = workload(name)
+    if heads:
+        w = dataclasses.replace(w, H=heads)
+    if world > 1:
+        w = dataclasses.replace(w, data_seed=w.data_seed + 100 * rank)
+    return w
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world == 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dense_equiv_flops(w) -> float:
     return 4.0 * w.B * w.H * float(w.N) ** 2 * w.d
 
@@ -150,13 +171,7 @@ def run_ours(args, rank, world, local_rank):
     build.build()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = workload(args.config)
-    if args.heads:
-        import dataclasses
-        w = dataclasses.replace(w, H=args.heads)
-    if world > 1:
-        import dataclasses
-        w = dataclasses.replace(w, data_seed=w.data_seed + 100 * rank)
+    w = rank_workload(args.config, rank, world, args.heads)
     K = w.budget_blocks(w.budgets[0])
     q, k, v = synth.make_qkv(w)
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
@@ -195,12 +210,6 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
 
     def timed(mode):
         for _ in range(args.warmup):
@@ -231,7 +240,7 @@ def run_ours(args, rank, world, local_rank):
     topk_total, topk_stage = timed("topk")
     topk_cnt = int(cnt.sum().item())
 
-    ms_step = max_over_ranks(total_ms / args.steps)
+    ms_step = max_over_ranks(total_ms / args.steps, world, dev)
     attn_ms = float(np.mean(stage_ms[:, 2]))
     dense = dense_equiv_flops(w)
     sel = selected_flops(sum_cnt, d)
@@ -262,7 +271,7 @@ def run_ours(args, rank, world, local_rank):
     b.record()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps)
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world, dev)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = out_h.numel() * out_h.element_size()
 
@@ -283,7 +292,7 @@ def run_ours(args, rank, world, local_rank):
                                f"budget {K}/{nb} key blocks, C={w.n_clusters}, T={w.iters}",
                    "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world}",
                    "l2": f"inputs Q+K+V = {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2 (no flush)"},
-        "attn_ms_per_call": round(max_over_ranks(attn_ms), 4),
+        "attn_ms_per_call": round(max_over_ranks(attn_ms, world, dev), 4),
         "attn_dense_equiv_tflops": round(dense / (attn_ms * 1e-3) / 1e12, 2),
         "attn_selected_tflops": round(sel / (attn_ms * 1e-3) / 1e12, 2),
         "stage_ms": {"score": round(float(np.mean(stage_ms[:, 0])), 4),
