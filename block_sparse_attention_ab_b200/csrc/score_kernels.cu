@@ -63,13 +63,63 @@ __global__ void __launch_bounds__(256) meankey_kernel(const __nv_bfloat16 *__res
 }
 
 // ---------------------------------------------------------------------------------
-// Per-block k-means: one CTA of 128 threads per (b, h, query block), thread t owns
-// query t (kept in fp32 registers); centroids live in shared memory.
-//   assign: argmin_c |c|^2 - 2 q.c (the |q|^2 term is common), strict < so ties go
-//           to the lowest cluster;
-//   update: members gathered per cluster in index order (warp ballots), summed in
-//           that order by one thread per dimension; an empty cluster keeps its centroid.
+// Per-block k-means on the tensor cores (warp-level mma.sync m16n8k16, bf16 inputs,
+// fp32 accumulation). One CTA of 128 threads (4 warps) per (b, h, query block); the
+// block's queries stay in shared memory for all T iterations.
+//   assign: q.c for every (query, centroid) as one small GEMM; each fp32 centroid is
+//           split exactly into three bf16 terms (hi + mid + lo), so the products are
+//           those of fp32 centroids with the bf16 queries, accumulated in fp32;
+//           distance |c|^2 - 2 q.c (|q|^2 is common); argmin with ties to the lowest
+//           cluster (compared as (distance, index) pairs across the 4 lanes that hold
+//           a row's 8 centroids);
+//   update: member sums as onehot[c][t] x Q[t][d] (exact 0/1 and bf16 operands, fp32
+//           accumulation), divided by the member counts; an empty cluster keeps its
+//           centroid.
+// The GEMMs are 128 x 24 x d and 16 x d x 128: far below one tcgen05 tile, and each
+// iteration needs the previous one's result, so warp-level MMAs in registers are used.
 // ---------------------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t &r0, uint32_t &r1)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t &r0, uint32_t &r1)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int D>
+struct KmSmem {
+    static constexpr int kStride = D + 8;                      // bf16 row stride (ldmatrix conflict-free)
+    static constexpr int kQ = 0;                               // Q     [128][kStride] bf16
+    static constexpr int kCB = kQ + 128 * kStride * 2;         // splits [24][kStride] bf16
+    static constexpr int kOH = kCB + 24 * kStride * 2;         // onehot [16][136] bf16
+    static constexpr int kCS = kOH + 16 * 136 * 2;             // fp32 centroids [8][D]
+    static constexpr int kBytes = kCS + 8 * D * 4;
+};
+
 template <int D>
 __global__ void __launch_bounds__(128) kmeans_kernel(const __nv_bfloat16 *__restrict__ q, int N,
                                                      int N_pad, int nqb, int C, int T,
@@ -77,14 +127,16 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __nv_bfloat16 *__rest
                                                      float *__restrict__ w_out,
                                                      uint8_t *__restrict__ assign_out)
 {
-    constexpr int CMAX = 8;
-    __shared__ __align__(16) __nv_bfloat16 qs[128][D];
-    __shared__ __align__(16) float cs[CMAX][D];
+    using L = KmSmem<D>;
+    constexpr int CMAX = 8, S = L::kStride;
+    extern __shared__ __align__(16) uint8_t km_smem[];
+    __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(km_smem + L::kQ);
+    __nv_bfloat16 *cb = reinterpret_cast<__nv_bfloat16 *>(km_smem + L::kCB);
+    __nv_bfloat16 *oh = reinterpret_cast<__nv_bfloat16 *>(km_smem + L::kOH);
+    float *cs = reinterpret_cast<float *>(km_smem + L::kCS);
     __shared__ float cn[CMAX];
     __shared__ int wcount[4][CMAX];
-    __shared__ int cstart[CMAX + 1];
     __shared__ int ccount[CMAX];
-    __shared__ uint8_t order[128];
     __shared__ uint8_t lab[128];
 
     const int blk = blockIdx.x;
@@ -92,114 +144,163 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __nv_bfloat16 *__rest
     const int t0 = qb * 128;
     const int nv = min(128, N - t0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = lane >> 2, tig = lane & 3;
 
-    // Stage the block's queries (padding rows as zero) with 16-byte loads.
+    // Stage the block's queries (padding rows as zero) with 16-byte loads; clear the
+    // one-hot matrix (its rows 8..15 stay zero).
     {
-        const uint4 *src = reinterpret_cast<const uint4 *>(q + ((size_t)bh * N_pad + t0) * D);
-        uint4 *dst = reinterpret_cast<uint4 *>(&qs[0][0]);
         constexpr int VEC = D / 8;
+        const uint4 *src = reinterpret_cast<const uint4 *>(q + ((size_t)bh * N_pad + t0) * D);
         for (int v = tid; v < 128 * VEC; v += 128) {
-            const int r = v / VEC;
-            dst[v] = r < nv ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+            const int r = v / VEC, c8 = v % VEC;
+            *reinterpret_cast<uint4 *>(qs + r * S + c8 * 8) =
+                r < nv ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
         }
+        for (int v = tid; v < 16 * 136 / 8; v += 128)
+            reinterpret_cast<uint4 *>(oh)[v] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
-
-    float qr[D];
-#pragma unroll
-    for (int i = 0; i < D; i += 2) {
-        const uint32_t x = *reinterpret_cast<const uint32_t *>(&qs[tid][i]);
-        qr[i] = bf16_lo(x);
-        qr[i + 1] = bf16_hi(x);
-    }
-    for (int e = tid; e < C * D; e += 128) {
+    for (int e = tid; e < CMAX * D; e += 128) {
         const int c = e / D, i = e % D;
-        const int src = nv >= C ? c * (nv / C) : min(c, nv - 1);
-        cs[c][i] = __bfloat162float(qs[src][i]);
+        float v = 0.f;
+        if (c < C) {
+            const int src = nv >= C ? c * (nv / C) : min(c, nv - 1);
+            v = __bfloat162float(qs[src * S + i]);
+        }
+        cs[c * D + i] = v;
     }
     __syncthreads();
 
+    const uint32_t qs_a = smem_u32(qs), cb_a = smem_u32(cb), oh_a = smem_u32(oh);
     for (int it = 0; it < T; ++it) {
-        // squared norms of the centroids
-        for (int c = warp; c < C; c += 4) {
-            float s = 0.f;
-            for (int i = lane; i < D; i += 32) s = fmaf(cs[c][i], cs[c][i], s);
+        // fp32 centroids -> exact three-term bf16 split; squared norms
+        for (int e = tid; e < CMAX * D; e += 128) {
+            const int c = e / D, i = e % D;
+            const float x = cs[c * D + i];
+            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+            const float r1 = x - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+            cb[c * S + i] = hi;
+            cb[(8 + c) * S + i] = mid;
+            cb[(16 + c) * S + i] = lo;
+        }
+        for (int c = warp; c < CMAX; c += 4) {
+            float sq = 0.f;
+            for (int i = lane; i < D; i += 32) sq = fmaf(cs[c * D + i], cs[c * D + i], sq);
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            if (lane == 0) cn[c] = s;
+            for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            if (lane == 0) cn[c] = sq;
         }
         __syncthreads();
-        // assignment
-        int a = CMAX;  // padding rows belong to no cluster
-        if (tid < nv) {
-            float best = 0.f;
+
+        // assignment: warp w owns queries 32w..32w+31 (two 16-row tiles)
 #pragma unroll
-            for (int c = 0; c < CMAX; ++c) {
-                if (c < C) {
-                    const float4 *cv = reinterpret_cast<const float4 *>(&cs[c][0]);
-                    float dot = 0.f;
+        for (int mt = 0; mt < 2; ++mt) {
+            const int r_base = warp * 32 + mt * 16;
+            float acc[3][4];
 #pragma unroll
-                    for (int i4 = 0; i4 < D / 4; ++i4) {
-                        const float4 cc = cv[i4];
-                        dot = fmaf(qr[4 * i4 + 0], cc.x, dot);
-                        dot = fmaf(qr[4 * i4 + 1], cc.y, dot);
-                        dot = fmaf(qr[4 * i4 + 2], cc.z, dot);
-                        dot = fmaf(qr[4 * i4 + 3], cc.w, dot);
-                    }
-                    const float dist = fmaf(-2.f, dot, cn[c]);
-                    if (c == 0 || dist < best) {
-                        best = dist;
-                        a = c;
-                    }
+            for (int nt = 0; nt < 3; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(qs_a + ((r_base + (lane & 15)) * S + kk * 16 + (lane >> 4) * 8) * 2, a0, a1,
+                        a2, a3);
+#pragma unroll
+                for (int nt = 0; nt < 3; ++nt) {
+                    uint32_t b0, b1;
+                    ldsm_x2(cb_a + ((nt * 8 + (lane & 7)) * S + kk * 16 + ((lane >> 3) & 1) * 8) * 2,
+                            b0, b1);
+                    mma_16816(acc[nt], a0, a1, a2, a3, b0, b1);
                 }
             }
-        }
-        lab[tid] = (uint8_t)a;
-        // stable counting sort of the members by cluster (warp ballots)
-        int rank = 0;
+            // rows r_base+grp (acc[.][0..1]) and r_base+grp+8 (acc[.][2..3]);
+            // columns (centroids) 2*tig and 2*tig+1
 #pragma unroll
-        for (int c = 0; c < CMAX; ++c) {
-            const unsigned m = __ballot_sync(0xffffffffu, a == c);
-            if (a == c) rank = __popc(m & ((1u << lane) - 1u));
-            if (lane == 0) wcount[warp][c] = __popc(m);
-        }
-        __syncthreads();
-        if (tid == 0) {
-            int s = 0;
-            for (int c = 0; c < CMAX; ++c) {
-                cstart[c] = s;
-                int n = 0;
-                for (int w = 0; w < 4; ++w) n += wcount[w][c];
-                ccount[c] = n;
-                s += n;
+            for (int h = 0; h < 2; ++h) {
+                float best = INFINITY;
+                int arg = CMAX;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int c = 2 * tig + e;
+                    const float dot = acc[0][2 * h + e] + acc[1][2 * h + e] + acc[2][2 * h + e];
+                    const float dist = c < C ? fmaf(-2.f, dot, cn[c]) : INFINITY;
+                    if (dist < best) {
+                        best = dist;
+                        arg = c;
+                    }
+                }
+#pragma unroll
+                for (int o = 1; o <= 2; o <<= 1) {
+                    const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+                    const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+                    if (ob < best || (ob == best && oa < arg)) {
+                        best = ob;
+                        arg = oa;
+                    }
+                }
+                const int r = r_base + grp + 8 * h;
+                if (tig == 0) lab[r] = r < nv ? (uint8_t)arg : (uint8_t)255;
             }
-            cstart[CMAX] = s;
         }
         __syncthreads();
-        if (a < CMAX) {
-            int pos = cstart[a] + rank;
-            for (int w = 0; w < warp; ++w) pos += wcount[w][a];
-            order[pos] = (uint8_t)tid;
+
+        // one-hot matrix [c][t] and member counts
+        {
+            const int a = lab[tid];
+#pragma unroll
+            for (int c = 0; c < CMAX; ++c) {
+                oh[c * 136 + tid] = __float2bfloat16_rn(a == c ? 1.f : 0.f);
+                const unsigned m = __ballot_sync(0xffffffffu, a == c);
+                if (lane == 0) wcount[warp][c] = __popc(m);
+            }
         }
         __syncthreads();
-        // update: thread i sums dimension i of each cluster's members in index order
-        for (int i = tid; i < D; i += 128) {
-            for (int c = 0; c < C; ++c) {
-                const int n = ccount[c];
-                if (n == 0) continue;
-                float s = 0.f;
-                const int st = cstart[c];
-                for (int m = 0; m < n; ++m) s += __bfloat162float(qs[order[st + m]][i]);
-                cs[c][i] = s / (float)n;
+        if (tid < CMAX) ccount[tid] = wcount[0][tid] + wcount[1][tid] + wcount[2][tid] + wcount[3][tid];
+
+        // update: sums[c][d] = onehot[c][.] x Q[.][d]; warp w owns columns w*D/4..
+        constexpr int NT = D / 32;  // n-tiles of 8 columns per warp
+        float sacc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(oh_a + ((lane & 15) * 136 + kk * 16 + (lane >> 4) * 8) * 2, a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int n0 = warp * (D / 4) + nt * 8;
+                uint32_t b0, b1;
+                ldsm_x2_trans(qs_a + ((kk * 16 + (lane & 15)) * S + n0) * 2, b0, b1);
+                mma_16816(sacc[nt], a0, a1, a2, a3, b0, b1);
+            }
+        }
+        __syncthreads();  // ccount visible; all reads of cs done
+        // rows 0..7 of the product are the clusters: this thread holds cluster grp,
+        // columns n0 + 2*tig + {0, 1}
+        {
+            const int c = grp;
+            const int n = ccount[c];
+            if (c < C && n > 0) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int col = warp * (D / 4) + nt * 8 + 2 * tig;
+                    cs[c * D + col] = sacc[nt][0] / (float)n;
+                    cs[c * D + col + 1] = sacc[nt][1] / (float)n;
+                }
             }
         }
         __syncthreads();
     }
 
     const size_t rowc = (size_t)blk * C;
-    for (int e = tid; e < C * D; e += 128) cent_out[rowc * D + e] = cs[e / D][e % D];
+    for (int e = tid; e < C * D; e += 128) cent_out[rowc * D + e] = cs[(e / D) * D + (e % D)];
     if (tid < C) w_out[rowc + tid] = (float)ccount[tid] / (float)nv;
-    if (assign_out) assign_out[(size_t)bh * N_pad + t0 + tid] = tid < nv ? lab[tid] : (uint8_t)255;
+    if (assign_out) assign_out[(size_t)bh * N_pad + t0 + tid] = lab[tid];
 }
 
 // ---------------------------------------------------------------------------------
@@ -353,12 +454,21 @@ cudaError_t launch_kmeans(const void *q, float *cent, float *cw, uint8_t *assign
 {
     const int nqb = N_pad / 128;
     const dim3 grid((unsigned)(BH * nqb));
-    if (d == 128)
-        kmeans_kernel<128><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)q, N, N_pad, nqb, C, T,
-                                                 cent, cw, assign);
-    else
-        kmeans_kernel<64><<<grid, 128, 0, st>>>((const __nv_bfloat16 *)q, N, N_pad, nqb, C, T,
-                                                cent, cw, assign);
+    if (d == 128) {
+        const int smem = KmSmem<128>::kBytes;
+        cudaError_t e = cudaFuncSetAttribute(kmeans_kernel<128>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        kmeans_kernel<128><<<grid, 128, smem, st>>>((const __nv_bfloat16 *)q, N, N_pad, nqb, C, T,
+                                                    cent, cw, assign);
+    } else {
+        const int smem = KmSmem<64>::kBytes;
+        cudaError_t e = cudaFuncSetAttribute(kmeans_kernel<64>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        kmeans_kernel<64><<<grid, 128, smem, st>>>((const __nv_bfloat16 *)q, N, N_pad, nqb, C, T,
+                                                   cent, cw, assign);
+    }
     return cudaGetLastError();
 }
 
