@@ -10,10 +10,6 @@
 
 namespace {
 
-constexpr size_t kAlign = 256;
-
-size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 ab_status check_shape(const ab_shape &s)
@@ -28,19 +24,9 @@ ab_status check_shape(const ab_shape &s)
     return AB_OK;
 }
 
-struct ScoreLayout {
-    size_t kbar, cent, cw, total;
-};
-
-ScoreLayout score_layout(const ab_shape &s, int C)
+ab::ScoreLayout score_layout(const ab_shape &s, int C)
 {
-    const size_t BH = (size_t)s.B * s.H, nb = (size_t)s.N_pad / AB_BLOCK;
-    ScoreLayout L;
-    L.kbar = 0;
-    L.cent = round_up(L.kbar + BH * nb * s.d * sizeof(float), kAlign);
-    L.cw = round_up(L.cent + BH * nb * C * s.d * sizeof(float), kAlign);
-    L.total = round_up(L.cw + BH * nb * C * sizeof(float), kAlign);
-    return L;
+    return ab::score_layout((size_t)s.B * s.H, (size_t)s.N_pad / AB_BLOCK, (size_t)s.d, (size_t)C);
 }
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
@@ -103,7 +89,6 @@ ab_status ab_score(const void *q, const void *k, ab_shape s, int n_clusters, int
                    uint8_t *assign, void *workspace, size_t workspace_bytes, int *dev_flag,
                    void *stream)
 {
-    (void)dev_flag;  // the scoring kernels have no device-detected failure mode
     if (!q || !k || !scores) return AB_ERR_NULL;
     ab_status st = check_shape(s);
     if (st != AB_OK) return st;
@@ -113,7 +98,7 @@ ab_status ab_score(const void *q, const void *k, ab_shape s, int n_clusters, int
         (centroids && !aligned16(centroids)) || (cweights && !aligned16(cweights)) ||
         !aligned16(workspace))
         return AB_ERR_ALIGN;
-    const ScoreLayout L = score_layout(s, n_clusters);
+    const ab::ScoreLayout L = score_layout(s, n_clusters);
     if (!workspace || workspace_bytes < L.total) return AB_ERR_WORKSPACE;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     float *kb = kbar ? kbar : reinterpret_cast<float *>(ws + L.kbar);
@@ -121,10 +106,13 @@ ab_status ab_score(const void *q, const void *k, ab_shape s, int n_clusters, int
     float *cw = cweights ? cweights : reinterpret_cast<float *>(ws + L.cw);
     const int BH = s.B * s.H, nb = s.N_pad / AB_BLOCK;
     cudaStream_t cs = (cudaStream_t)stream;
-    cudaError_t e = ab::launch_meankey(k, kb, BH, s.N, s.N_pad, s.d, cs);
+    void *kt = ws + L.kbar_terms;
+    cudaError_t e = ab::launch_meankey(k, kb, kt, BH, s.N, s.N_pad, s.d, cs);
     if (e == cudaSuccess)
-        e = ab::launch_kmeans(q, ce, cw, assign, BH, s.N, s.N_pad, s.d, n_clusters, iters, cs);
-    if (e == cudaSuccess) e = ab::launch_score(ce, cw, kb, scores, BH, nb, nb, s.d, n_clusters, cs);
+        e = ab::launch_kmeans(q, ce, cw, assign, BH, s.N, s.N_pad, s.d, n_clusters, iters,
+                              dev_flag, cs);
+    if (e == cudaSuccess)
+        e = ab::launch_score(ce, cw, kt, scores, BH, nb, nb, s.d, n_clusters, dev_flag, cs);
     return cuda_status(e);
 }
 

@@ -89,6 +89,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// Bounded wait that ignores the abort flag: used only while unwinding, to let copies
+// and MMAs already in flight land before the CTA releases its memory.
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > 200000000ull) return;
+    }
+}
+
+// Make this thread's ordinary shared-memory stores visible to the async proxy (TMA,
+// tcgen05.mma operand reads); issued by the writers before the barrier that hands the
+// data to the MMA thread.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Base of the dynamic shared memory rounded up to 1024 bytes (the 128-byte swizzle
+// atoms assume 1024-byte aligned tiles); launches reserve 1024 bytes of slack.
+__device__ __forceinline__ uint8_t *align_smem_1024(uint8_t *raw)
+{
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(raw) + 1023) &
+                                       ~static_cast<uintptr_t>(1023));
+}
+
 // ---------------------------------------------------------------------------------
 // TMA: 3-D tiled load global -> shared, completion counted on an mbarrier.
 // ---------------------------------------------------------------------------------

@@ -1,6 +1,7 @@
 // ab_noalloc.cu -- ab_score_noalloc: the IBCS scoring call for callers that cannot
-// allocate device memory (see include/ab_attn.h). Its scratch -- mean keys, centroids
-// and cluster weights -- lives in a fixed array in the library's own device memory.
+// allocate device memory (see include/ab_attn.h). Its scratch -- mean keys, centroids,
+// cluster weights and the bf16 terms of the mean keys -- lives in a fixed array in the
+// library's own device memory.
 #include <cstdint>
 #include <mutex>
 #include <cuda_runtime.h>
@@ -11,7 +12,6 @@
 namespace {
 
 constexpr size_t kScratchBytes = (size_t)AB_NOALLOC_SCRATCH_BYTES;
-constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
 
 // One copy per device that loads the library, resident until the process exits.
@@ -19,8 +19,6 @@ static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 std::mutex g_setup_mutex;
 void *g_scratch_addr[kMaxDevices] = {};
-
-size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -46,7 +44,6 @@ ab_status scratch_on_current_device(void **out)
 extern "C" ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, int n_clusters,
                                       int iters, float *scores, int *dev_flag, void *stream)
 {
-    (void)dev_flag;
     if (!q || !k || !scores) return AB_ERR_NULL;
     if (s.B <= 0 || s.H <= 0 || s.N <= 0 || s.N_pad <= 0 || s.d <= 0) return AB_ERR_SHAPE;
     if (s.N_pad % AB_BLOCK != 0 || s.N > s.N_pad || s.N_pad - s.N >= AB_BLOCK) return AB_ERR_SHAPE;
@@ -57,12 +54,9 @@ extern "C" ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, 
     if (iters < 1 || iters > 1000) return AB_ERR_RANGE;
     if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return AB_ERR_ALIGN;
 
-    const size_t BH = (size_t)s.B * s.H, nb = (size_t)s.N_pad / AB_BLOCK;
-    const size_t off_kbar = 0;
-    const size_t off_cent = round_up(off_kbar + BH * nb * s.d * sizeof(float), kAlign);
-    const size_t off_cw = round_up(off_cent + BH * nb * n_clusters * s.d * sizeof(float), kAlign);
-    const size_t total = round_up(off_cw + BH * nb * n_clusters * sizeof(float), kAlign);
-    if (total > kScratchBytes) return AB_ERR_WORKSPACE;
+    const ab::ScoreLayout L = ab::score_layout((size_t)s.B * s.H, (size_t)s.N_pad / AB_BLOCK,
+                                               (size_t)s.d, (size_t)n_clusters);
+    if (L.total > kScratchBytes) return AB_ERR_WORKSPACE;
 
     void *base = nullptr;
     ab_status st = scratch_on_current_device(&base);
@@ -70,14 +64,17 @@ extern "C" ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, 
     // Every region below is fully written by a kernel before any kernel reads it, so
     // nothing left by an earlier call needs clearing.
     uint8_t *ws = static_cast<uint8_t *>(base);
-    float *kb = reinterpret_cast<float *>(ws + off_kbar);
-    float *ce = reinterpret_cast<float *>(ws + off_cent);
-    float *cw = reinterpret_cast<float *>(ws + off_cw);
-    const int nbi = (int)nb;
+    float *kb = reinterpret_cast<float *>(ws + L.kbar);
+    float *ce = reinterpret_cast<float *>(ws + L.cent);
+    float *cw = reinterpret_cast<float *>(ws + L.cw);
+    void *kt = ws + L.kbar_terms;
+    const int BH = s.B * s.H, nb = s.N_pad / AB_BLOCK;
     cudaStream_t cs = (cudaStream_t)stream;
-    cudaError_t e = ab::launch_meankey(k, kb, (int)BH, s.N, s.N_pad, s.d, cs);
+    cudaError_t e = ab::launch_meankey(k, kb, kt, BH, s.N, s.N_pad, s.d, cs);
     if (e == cudaSuccess)
-        e = ab::launch_kmeans(q, ce, cw, nullptr, (int)BH, s.N, s.N_pad, s.d, n_clusters, iters, cs);
-    if (e == cudaSuccess) e = ab::launch_score(ce, cw, kb, scores, (int)BH, nbi, nbi, s.d, n_clusters, cs);
+        e = ab::launch_kmeans(q, ce, cw, nullptr, BH, s.N, s.N_pad, s.d, n_clusters, iters,
+                              dev_flag, cs);
+    if (e == cudaSuccess)
+        e = ab::launch_score(ce, cw, kt, scores, BH, nb, nb, s.d, n_clusters, dev_flag, cs);
     return e == cudaSuccess ? AB_OK : AB_ERR_CUDA;
 }

@@ -29,6 +29,7 @@
 
 #include "ab_device.cuh"
 #include "ab_kernels.h"
+#include "tmap_host.h"
 
 namespace ab {
 
@@ -118,15 +119,6 @@ __device__ __forceinline__ int block_index(const AttnParams &p, int r, int i, bo
     return j;
 }
 
-// bounded wait that ignores the abort flag (used only to drain in-flight work)
-__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)
-{
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > 200000000ull) return;
-    }
-}
-
 template <int D, bool kWeighted, bool kOutF32>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -134,8 +126,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 {
     using L = AttnSmem<D>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *smem = align_smem_1024(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
     uint64_t *q_full = bars;
     uint64_t *q_empty = bars + 2;
@@ -560,40 +551,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // ---------------------------------------------------------------------------------
 // Host side: tensor maps and launch
 // ---------------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
 // 3-D map over a [B*H, N_pad, d] bf16 tensor with row extent N (rows >= N read as 0),
 // box 64 columns x 128 rows, 128-byte swizzle.
 static bool make_tmap(CUtensorMap *tm, const void *base, int BH, int N, int N_pad, int d)
 {
-    EncodeTiledFn enc = get_encode_fn();
-    if (!enc) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
-    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N_pad * d * 2};
-    const cuuint32_t box[3] = {64, 128, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return make_tmap_bf16_3d(tm, base, (uint64_t)d, (uint64_t)N, (uint64_t)BH, (uint64_t)d * 2,
+                             (uint64_t)N_pad * d * 2, 64, 128);
 }
 
 template <int D, bool W, bool F32>

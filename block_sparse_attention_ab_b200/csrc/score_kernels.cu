@@ -8,20 +8,62 @@
 
 #include "ab_device.cuh"
 #include "ab_kernels.h"
+#include "tmap_host.h"
 
 namespace ab {
 
 __device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 
+// Exact three-term bf16 split of fp32 values: x = hi + mid + lo with every term a bf16
+// (each subtraction is exact: the remainder of rounding to 8 significant bits has at
+// most 16, then at most 8). Products of two such splits with the terms of total
+// order <= 4 reproduce an fp32 product to about 2^-24 relative.
+__device__ __forceinline__ void split3(float x, __nv_bfloat16 &a, __nv_bfloat16 &b,
+                                       __nv_bfloat16 &c)
+{
+    a = __float2bfloat16_rn(x);
+    const float r = x - __bfloat162float(a);
+    b = __float2bfloat16_rn(r);
+    c = __float2bfloat16_rn(r - __bfloat162float(b));
+}
+
+// The same for 8 consecutive values, packed as three 16-byte rows (hi, mid, lo).
+__device__ __forceinline__ void split3x8(const float (&x)[8], uint4 (&t)[3])
+{
+    uint32_t a[4], b[4], c[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float x0 = x[2 * e], x1 = x[2 * e + 1];
+        a[e] = pack_bf16x2(x0, x1);
+        const float r0 = x0 - bf16_lo(a[e]), r1 = x1 - bf16_hi(a[e]);
+        b[e] = pack_bf16x2(r0, r1);
+        c[e] = pack_bf16x2(r0 - bf16_lo(b[e]), r1 - bf16_hi(b[e]));
+    }
+    t[0] = make_uint4(a[0], a[1], a[2], a[3]);
+    t[1] = make_uint4(b[0], b[1], b[2], b[3]);
+    t[2] = make_uint4(c[0], c[1], c[2], c[3]);
+}
+
+// Byte offset of the 16-byte chunk holding element (row, col) of a K-major tile stored
+// as 64-column (128-byte) panels of `panel_bytes` each, with the 128-byte swizzle that
+// TMA and the tcgen05 descriptors use (chunk index XOR row mod 8; tiles 1024-aligned).
+__device__ __forceinline__ int sw128_chunk(int row, int col, int panel_bytes)
+{
+    return (col >> 6) * panel_bytes + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4);
+}
+
 // ---------------------------------------------------------------------------------
 // Mean key: one CTA of 256 threads per (b, h, key block); 16-byte coalesced loads,
-// fp32 sums in a fixed order, divided by the block's valid-key count.
+// fp32 sums in a fixed order, divided by the block's valid-key count. Also writes the
+// three bf16 terms of each mean key (split3) for the tensor-core block score:
+// kbs[t][bh][j][i], t = 0 (hi), 1 (mid), 2 (lo).
 // ---------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) meankey_kernel(const __nv_bfloat16 *__restrict__ k,
-                                                      float *__restrict__ kbar, int N, int N_pad,
-                                                      int nkb)
+                                                      float *__restrict__ kbar,
+                                                      __nv_bfloat16 *__restrict__ kbs, int N,
+                                                      int N_pad, int nkb)
 {
     constexpr int VEC = D / 8;         // 16-byte vectors per row
     constexpr int GROUPS = 256 / VEC;  // row groups
@@ -54,442 +96,648 @@ __global__ void __launch_bounds__(256) meankey_kernel(const __nv_bfloat16 *__res
     dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     __syncthreads();
     const float inv = 1.0f / (float)nv;
+    const size_t term = (size_t)gridDim.x * D;
     for (int col = tid; col < D; col += 256) {
         float s = 0.f;
 #pragma unroll 8
         for (int g = 0; g < GROUPS; ++g) s += part[g][col];
-        kbar[(size_t)blk * D + col] = s * inv;
+        const float m = s * inv;
+        kbar[(size_t)blk * D + col] = m;
+        __nv_bfloat16 a, b, c;
+        split3(m, a, b, c);
+        kbs[(size_t)blk * D + col] = a;
+        kbs[term + (size_t)blk * D + col] = b;
+        kbs[2 * term + (size_t)blk * D + col] = c;
     }
 }
 
 // ---------------------------------------------------------------------------------
-// Per-block k-means on the tensor cores (warp-level mma.sync m16n8k16, bf16 inputs,
-// fp32 accumulation). One CTA of 128 threads (4 warps) per (b, h, query block); the
-// block's queries stay in shared memory for all T iterations.
-//   assign: q.c for every (query, centroid) as one small GEMM; each fp32 centroid is
-//           split exactly into three bf16 terms (hi + mid + lo), so the products are
-//           those of fp32 centroids with the bf16 queries, accumulated in fp32;
-//           distance |c|^2 - 2 q.c (|q|^2 is common); argmin with ties to the lowest
-//           cluster (compared as (distance, index) pairs across the 4 lanes that hold
-//           a row's 8 centroids);
-//   update: member sums as onehot[c][t] x Q[t][d] (exact 0/1 and bf16 operands, fp32
-//           accumulation), divided by the member counts; an empty cluster keeps its
+// Per-block k-means on the 5th-generation tensor cores. One CTA of 128 threads per
+// (b, h, query block). The block's queries arrive by TMA (128-byte swizzle; rows past
+// N read as zero) and stay in shared memory for all T iterations. Each iteration runs
+// two single-CTA tcgen05 GEMMs with fp32 accumulators in TMEM:
+//   assign: G = Q B^T (M = 128 queries, N = 32, K = d): rows 8t + c of B hold term t
+//           (split3) of fp32 centroid c, rows 24..31 are zero, so q . c =
+//           G[q][c] + G[q][8 + c] + G[q][16 + c] is the bf16 query times the fp32
+//           centroid; distance |c|^2 - 2 q.c (|q|^2 is common), argmin with ties to
+//           the lowest cluster; thread t reads TMEM lane t = query t;
+//   update: S = Q^T H (M = 128 features, Q read feature-major from the same tile;
+//           N = 16 clusters, one-hot rows 8..15 zero; K = 128 queries): member sums,
+//           exact 0/1 and bf16 operands with fp32 accumulation, divided by the member
+//           counts; thread i reads TMEM lane i = feature i; an empty cluster keeps its
 //           centroid.
-// The GEMMs are 128 x 24 x d and 16 x d x 128: far below one tcgen05 tile, and each
-// iteration needs the previous one's result, so warp-level MMAs in registers are used.
+// All 128 threads stage the operands; one elected thread of warp 0 issues the MMAs.
+// Every wait is bounded; a timed-out CTA drains its in-flight work and exits.
 // ---------------------------------------------------------------------------------
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
-                                        uint32_t &r3)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t &r0, uint32_t &r1)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
-                 : "=r"(r0), "=r"(r1)
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t &r0, uint32_t &r1)
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-                 : "=r"(r0), "=r"(r1)
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                          uint32_t a3, uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 template <int D>
 struct KmSmem {
-    static constexpr int kStride = D + 8;                      // bf16 row stride (ldmatrix conflict-free)
-    static constexpr int kQ = 0;                               // Q     [128][kStride] bf16
-    static constexpr int kCB = kQ + 128 * kStride * 2;         // splits [24][kStride] bf16
-    static constexpr int kOH = kCB + 24 * kStride * 2;         // onehot [16][136] bf16
-    static constexpr int kCS = kOH + 16 * 136 * 2;             // fp32 centroids [8][D]
-    static constexpr int kBytes = kCS + 8 * D * 4;
+    static constexpr int kQ = 0;                        // queries: 2 panels [128][64] bf16
+    static constexpr int kBA = kQ + 2 * 16384;          // centroid terms: (D/64) x [32][64]
+    static constexpr int kBU = kBA + (D / 64) * 4096;   // one-hot: 2 panels [16][64]
+    static constexpr int kCS = kBU + 2 * 2048;          // fp32 centroids [8][D]
+    static constexpr int kBar = kCS + 8 * D * 4;        // q_full, mma_done, drain
+    static constexpr int kMisc = kBar + 3 * 8;          // TMEM base, abort flag
+    static constexpr int kBytes = kMisc + 8;
+    static constexpr int kAlloc = kBytes + 1024;        // slack to align the base to 1024 B
 };
 
+constexpr int kKmTmemCols = 64;  // G in columns 0..31, S in columns 32..47
+
 template <int D>
-__global__ void __launch_bounds__(128) kmeans_kernel(const __nv_bfloat16 *__restrict__ q, int N,
-                                                     int N_pad, int nqb, int C, int T,
+__global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                     int N, int N_pad, int nqb, int C, int T,
                                                      float *__restrict__ cent_out,
                                                      float *__restrict__ w_out,
-                                                     uint8_t *__restrict__ assign_out)
+                                                     uint8_t *__restrict__ assign_out, int *flag)
 {
     using L = KmSmem<D>;
-    constexpr int CMAX = 8, S = L::kStride;
-    extern __shared__ __align__(16) uint8_t km_smem[];
-    __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(km_smem + L::kQ);
-    __nv_bfloat16 *cb = reinterpret_cast<__nv_bfloat16 *>(km_smem + L::kCB);
-    __nv_bfloat16 *oh = reinterpret_cast<__nv_bfloat16 *>(km_smem + L::kOH);
-    float *cs = reinterpret_cast<float *>(km_smem + L::kCS);
+    constexpr int CMAX = 8;
+    extern __shared__ uint8_t km_raw[];
+    uint8_t *smem = align_smem_1024(km_raw);
     __shared__ float cn[CMAX];
     __shared__ int wcount[4][CMAX];
-    __shared__ int ccount[CMAX];
     __shared__ uint8_t lab[128];
+    uint64_t *q_full = reinterpret_cast<uint64_t *>(smem + L::kBar);
+    uint64_t *mma_done = q_full + 1;
+    uint64_t *drain = q_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+    float *cs = reinterpret_cast<float *>(smem + L::kCS);
 
     const int blk = blockIdx.x;
     const int bh = blk / nqb, qb = blk % nqb;
     const int t0 = qb * 128;
     const int nv = min(128, N - t0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int grp = lane >> 2, tig = lane & 3;
 
-    // Stage the block's queries (padding rows as zero) with 16-byte loads; clear the
-    // one-hot matrix (its rows 8..15 stay zero).
-    {
-        constexpr int VEC = D / 8;
-        const uint4 *src = reinterpret_cast<const uint4 *>(q + ((size_t)bh * N_pad + t0) * D);
-        for (int v = tid; v < 128 * VEC; v += 128) {
-            const int r = v / VEC, c8 = v % VEC;
-            *reinterpret_cast<uint4 *>(qs + r * S + c8 * 8) =
-                r < nv ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
-        }
-        for (int v = tid; v < 16 * 136 / 8; v += 128)
-            reinterpret_cast<uint4 *>(oh)[v] = make_uint4(0, 0, 0, 0);
+    if (tid == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(mma_done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
     }
-    __syncthreads();
-    for (int e = tid; e < CMAX * D; e += 128) {
-        const int c = e / D, i = e % D;
-        float v = 0.f;
-        if (c < C) {
-            const int src = nv >= C ? c * (nv / C) : min(c, nv - 1);
-            v = __bfloat162float(qs[src * S + i]);
-        }
-        cs[c * D + i] = v;
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, kKmTmemCols);
+        tmem_relinquish();
     }
+    // constant zero rows: centroid-term rows 24..31, one-hot rows 8..15
+    for (int e = tid; e < (D / 64) * 64; e += 128)
+        *reinterpret_cast<uint4 *>(smem + L::kBA + (e >> 6) * 4096 + (24 + ((e >> 3) & 7)) * 128 +
+                                   (e & 7) * 16) = make_uint4(0, 0, 0, 0);
+    if (tid < 128)
+        *reinterpret_cast<uint4 *>(smem + L::kBU + (tid >> 6) * 2048 + (8 + ((tid >> 3) & 7)) * 128 +
+                                   (tid & 7) * 16) = make_uint4(0, 0, 0, 0);
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
 
-    const uint32_t qs_a = smem_u32(qs), cb_a = smem_u32(cb), oh_a = smem_u32(oh);
-    for (int it = 0; it < T; ++it) {
-        // fp32 centroids -> exact three-term bf16 split; squared norms
+    if (warp == 0) {
+        if (elect_one()) {
+            prefetch_tmap(&tmQ);
+            mbar_arrive_expect_tx(q_full, (D / 64) * 16384);
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+                tma_load_3d(smem + L::kQ + h * 16384, &tmQ, q_full, h * 64, t0, bh);
+        }
+        __syncwarp();
+    }
+    bool ok = __syncthreads_and(mbar_wait(q_full, 0, abort_flag, flag));
+
+    const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(smem + L::kQ);
+    if (ok) {
+        // initial centroid c: the query at block-local index c*floor(nv/C) (min(c, nv-1)
+        // when nv < C)
         for (int e = tid; e < CMAX * D; e += 128) {
             const int c = e / D, i = e % D;
-            const float x = cs[c * D + i];
-            const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-            const float r1 = x - __bfloat162float(hi);
-            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-            cb[c * S + i] = hi;
-            cb[(8 + c) * S + i] = mid;
-            cb[(16 + c) * S + i] = lo;
-        }
-        for (int c = warp; c < CMAX; c += 4) {
-            float sq = 0.f;
-            for (int i = lane; i < D; i += 32) sq = fmaf(cs[c * D + i], cs[c * D + i], sq);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-            if (lane == 0) cn[c] = sq;
+            float v = 0.f;
+            if (c < C) {
+                const int src = nv >= C ? c * (nv / C) : min(c, nv - 1);
+                v = __bfloat162float(qs[(sw128_chunk(src, i, 16384) >> 1) + (i & 7)]);
+            }
+            cs[c * D + i] = v;
         }
         __syncthreads();
+    }
 
-        // assignment: warp w owns queries 32w..32w+31 (two 16-row tiles)
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-            const int r_base = warp * 32 + mt * 16;
-            float acc[3][4];
-#pragma unroll
-            for (int nt = 0; nt < 3; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4(qs_a + ((r_base + (lane & 15)) * S + kk * 16 + (lane >> 4) * 8) * 2, a0, a1,
-                        a2, a3);
-#pragma unroll
-                for (int nt = 0; nt < 3; ++nt) {
-                    uint32_t b0, b1;
-                    ldsm_x2(cb_a + ((nt * 8 + (lane & 7)) * S + kk * 16 + ((lane >> 3) & 1) * 8) * 2,
-                            b0, b1);
-                    mma_16816(acc[nt], a0, a1, a2, a3, b0, b1);
-                }
-            }
-            // rows r_base+grp (acc[.][0..1]) and r_base+grp+8 (acc[.][2..3]);
-            // columns (centroids) 2*tig and 2*tig+1
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float best = INFINITY;
-                int arg = CMAX;
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int c = 2 * tig + e;
-                    const float dot = acc[0][2 * h + e] + acc[1][2 * h + e] + acc[2][2 * h + e];
-                    const float dist = c < C ? fmaf(-2.f, dot, cn[c]) : INFINITY;
-                    if (dist < best) {
-                        best = dist;
-                        arg = c;
-                    }
-                }
-#pragma unroll
-                for (int o = 1; o <= 2; o <<= 1) {
-                    const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-                    const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
-                    if (ob < best || (ob == best && oa < arg)) {
-                        best = ob;
-                        arg = oa;
-                    }
-                }
-                const int r = r_base + grp + 8 * h;
-                if (tig == 0) lab[r] = r < nv ? (uint8_t)arg : (uint8_t)255;
-            }
-        }
-        __syncthreads();
+    const uint32_t q_addr = smem_u32(smem + L::kQ);
+    const uint64_t a_asg = smem_desc_sw128(q_addr, 16, 1024);
+    const uint64_t b_asg = smem_desc_sw128(smem_u32(smem + L::kBA), 16, 1024);
+    const uint64_t a_upd = smem_desc_sw128(q_addr, 16384, 1024);  // feature-major view of Q
+    const uint64_t b_upd = smem_desc_sw128(smem_u32(smem + L::kBU), 16, 1024);
+    constexpr uint32_t idesc_asg = idesc_bf16_f32(128, 32, 0, 0);
+    constexpr uint32_t idesc_upd = idesc_bf16_f32(128, 16, 1, 0);
+    const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+    uint32_t phase = 0;
 
-        // one-hot matrix [c][t] and member counts
+    for (int it = 0; it < T && ok; ++it) {
+        // (1) centroid terms (B of the assignment GEMM) and squared norms
         {
-            const int a = lab[tid];
+            constexpr int CH = D / 8;
+            if (tid < CMAX * CH) {
+                const int c = tid / CH, k0 = (tid % CH) * 8;
+                const float4 x0 = *reinterpret_cast<const float4 *>(cs + c * D + k0);
+                const float4 x1 = *reinterpret_cast<const float4 *>(cs + c * D + k0 + 4);
+                const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                uint4 t[3];
+                split3x8(xs, t);
+#pragma unroll
+                for (int s = 0; s < 3; ++s)
+                    *reinterpret_cast<uint4 *>(smem + L::kBA + sw128_chunk(8 * s + c, k0, 4096)) = t[s];
+            }
+            for (int c = warp; c < CMAX; c += 4) {
+                float sq = 0.f;
+                for (int i = lane; i < D; i += 32) sq = fmaf(cs[c * D + i], cs[c * D + i], sq);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                if (lane == 0) cn[c] = sq;
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // (2) assignment GEMM
+        if (warp == 0) {
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    mma_ss(tmem, a_asg + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                           b_asg + (uint64_t)(((kk >> 2) * 4096 + (kk & 3) * 32) >> 4), idesc_asg,
+                           kk > 0 ? 1u : 0u);
+                mma_commit(mma_done);
+            }
+            __syncwarp();
+        }
+        bool good = __all_sync(0xffffffffu, mbar_wait(mma_done, phase, abort_flag, flag));
+        phase ^= 1;
+        tc_fence_after();
+        {
+            uint32_t g[32];
+            if (good) {
+                tmem_ld32(t_lane, g);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) g[e] = 0u;
+            }
+            float best = INFINITY;
+            int arg = 0;
 #pragma unroll
             for (int c = 0; c < CMAX; ++c) {
-                oh[c * 136 + tid] = __float2bfloat16_rn(a == c ? 1.f : 0.f);
+                const float dot = (__uint_as_float(g[c]) + __uint_as_float(g[8 + c])) +
+                                  __uint_as_float(g[16 + c]);
+                const float dist = fmaf(-2.f, dot, cn[c]);
+                if (c < C && dist < best) {
+                    best = dist;
+                    arg = c;
+                }
+            }
+            const int a = tid < nv ? arg : 255;
+            lab[tid] = (uint8_t)a;
+            // (3) one-hot column of this query (B of the update GEMM) and member counts
+            __nv_bfloat16 *oh = reinterpret_cast<__nv_bfloat16 *>(smem + L::kBU);
+#pragma unroll
+            for (int c = 0; c < CMAX; ++c) {
+                oh[(sw128_chunk(c, tid, 2048) >> 1) + (tid & 7)] =
+                    __ushort_as_bfloat16(a == c ? (unsigned short)0x3F80u : (unsigned short)0u);
                 const unsigned m = __ballot_sync(0xffffffffu, a == c);
                 if (lane == 0) wcount[warp][c] = __popc(m);
             }
         }
-        __syncthreads();
-        if (tid < CMAX) ccount[tid] = wcount[0][tid] + wcount[1][tid] + wcount[2][tid] + wcount[3][tid];
+        fence_proxy_async_smem();
+        tc_fence_before();
+        ok = __syncthreads_and(good);
+        if (!ok) break;
+        tc_fence_after();
 
-        // update: sums[c][d] = onehot[c][.] x Q[.][d]; warp w owns columns w*D/4..
-        constexpr int NT = D / 32;  // n-tiles of 8 columns per warp
-        float sacc[NT][4];
+        // (4) update GEMM
+        if (warp == 0) {
+            if (elect_one()) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(oh_a + ((lane & 15) * 136 + kk * 16 + (lane >> 4) * 8) * 2, a0, a1, a2, a3);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int n0 = warp * (D / 4) + nt * 8;
-                uint32_t b0, b1;
-                ldsm_x2_trans(qs_a + ((kk * 16 + (lane & 15)) * S + n0) * 2, b0, b1);
-                mma_16816(sacc[nt], a0, a1, a2, a3, b0, b1);
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + 32, a_upd + (uint64_t)((kk * 2048) >> 4),
+                           b_upd + (uint64_t)(((kk >> 2) * 2048 + (kk & 3) * 32) >> 4), idesc_upd,
+                           kk > 0 ? 1u : 0u);
+                mma_commit(mma_done);
             }
+            __syncwarp();
         }
-        __syncthreads();  // ccount visible; all reads of cs done
-        // rows 0..7 of the product are the clusters: this thread holds cluster grp,
-        // columns n0 + 2*tig + {0, 1}
-        {
-            const int c = grp;
-            const int n = ccount[c];
-            if (c < C && n > 0) {
+        good = __all_sync(0xffffffffu, mbar_wait(mma_done, phase, abort_flag, flag));
+        phase ^= 1;
+        tc_fence_after();
+        if (good) {
+            uint32_t sv[16];
+            tmem_ld16(t_lane + 32, sv);
+            tmem_wait_ld();
+            if (tid < D) {
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const int col = warp * (D / 4) + nt * 8 + 2 * tig;
-                    cs[c * D + col] = sacc[nt][0] / (float)n;
-                    cs[c * D + col + 1] = sacc[nt][1] / (float)n;
+                for (int c = 0; c < CMAX; ++c) {
+                    const int n = wcount[0][c] + wcount[1][c] + wcount[2][c] + wcount[3][c];
+                    if (c < C && n > 0) cs[c * D + tid] = __uint_as_float(sv[c]) / (float)n;
                 }
             }
         }
-        __syncthreads();
+        tc_fence_before();
+        ok = __syncthreads_and(good);
     }
 
-    const size_t rowc = (size_t)blk * C;
-    for (int e = tid; e < C * D; e += 128) cent_out[rowc * D + e] = cs[(e / D) * D + (e % D)];
-    if (tid < C) w_out[rowc + tid] = (float)ccount[tid] / (float)nv;
-    if (assign_out) assign_out[(size_t)bh * N_pad + t0 + tid] = lab[tid];
+    if (ok) {
+        const size_t rowc = (size_t)blk * C;
+        for (int e = tid; e < C * D; e += 128) cent_out[rowc * D + e] = cs[e];
+        if (tid < C) {
+            const int n = wcount[0][tid] + wcount[1][tid] + wcount[2][tid] + wcount[3][tid];
+            w_out[rowc + tid] = (float)n / (float)nv;
+        }
+        if (assign_out) assign_out[(size_t)bh * N_pad + t0 + tid] = lab[tid];
+    } else if (warp == 0) {
+        // unwind: let the query copy and the last MMAs land before releasing memory
+        if (elect_one()) {
+            mma_commit(drain);
+            drain_wait(drain, 0);
+            drain_wait(q_full, 0);
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kKmTmemCols);
+    }
 }
 
 // ---------------------------------------------------------------------------------
-// Block score: one CTA of 8 warps per (b, h, 8 query blocks); warp w owns query block
-// qb0 + w and its C <= 8 centroids; lane l owns key-block columns 2l, 2l+1 of each
-// 64-wide tile of mean keys. Pass 1 accumulates each centroid's softmax max and sum
-// over all key blocks (online, merged across lanes); pass 2 recomputes the logits and
-// writes s_j = sum_c (w_c / Z_c) exp(L_cj - m_c).
+// Block score on the 5th-generation tensor cores. One CTA per (b, h, 16 query
+// blocks); its 128 TMEM lanes are the centroid rows r = 8 * (query block) + c
+// (clusters c >= C and query blocks past the end are zero rows with weight 0).
+// Logits L[r][j] = cent_r . kbar_j are computed as 128 x 64 x d tcgen05 GEMMs over
+// tiles of 64 key blocks, with both fp32 operands split exactly into three bf16 terms
+// (split3) and the six term products of total order <= 4 accumulated in fp32: the
+// omitted terms are below 2^-24 relative, so the logits carry fp32 accuracy. The
+// centroid terms are built once in shared memory by all threads; the key terms are
+// written by the mean-key kernel and arrive by TMA.
+// Key blocks are processed in chunks of 256 (one TMEM buffer of 256 columns; two
+// buffers). With n_kb <= 256 one pass suffices: each row's softmax max and sum and
+// then the scores come from the logits held in TMEM. With more chunks, a first pass
+// accumulates each row's max and sum online and a second pass recomputes the logits
+// and writes s_j = sum_c (w_c / Z_c) 2^(L'_cj - m_c) (L' in log2 units), the sum over
+// a query block's 8 centroid rows taken across 8 lanes (butterfly reduce-scatter).
+// Warp 0: TMA producer; warp 1: TMEM owner and MMA issuer; warps 2..5: epilogue
+// (warp w reads TMEM lanes 32 (w mod 4) .. +31).
 // ---------------------------------------------------------------------------------
+constexpr int kScThreads = 192;
+constexpr int kScChunk = 256;
+constexpr int kScTmemCols = 512;
+
 template <int D>
-__global__ void __launch_bounds__(256) score_kernel(const float *__restrict__ cent,
-                                                    const float *__restrict__ cw,
-                                                    const float *__restrict__ kbar, int nqb,
-                                                    int nkb, int C, float scale,
-                                                    float *__restrict__ scores)
+struct ScSmem {
+    static constexpr int kPanels = D / 64;
+    static constexpr int kATerm = kPanels * 16384;           // one term of the 128 centroid rows
+    static constexpr int kBTerm = kPanels * 8192;            // one term of 64 mean keys
+    static constexpr int kStageBytes = 3 * kBTerm;
+    static constexpr int kStages = D == 128 ? 2 : 4;
+    static constexpr int kA = 0;
+    static constexpr int kB = kA + 3 * kATerm;
+    static constexpr int kBar = kB + kStages * kStageBytes;
+    // barriers: full[S], empty[S], tfull[2], tempty[2], drain
+    static constexpr int kNumBars = 2 * kStages + 5;
+    static constexpr int kMisc = kBar + kNumBars * 8;       // TMEM base, abort flag
+    static constexpr int kBytes = kMisc + 8;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+
+// the six term products (a, b) of total order <= 4, terms numbered 0 (hi), 1, 2 (lo):
+// (0,0) (0,1) (1,0) (0,2) (1,1) (2,0)
+__host__ __device__ constexpr int prod_term_a(int pr) { return pr == 2 || pr == 4 ? 1 : (pr == 5 ? 2 : 0); }
+__host__ __device__ constexpr int prod_term_b(int pr) { return pr == 1 || pr == 4 ? 1 : (pr == 3 ? 2 : 0); }
+
+template <int D>
+__global__ void __launch_bounds__(kScThreads, 1)
+    score_kernel(const __grid_constant__ CUtensorMap tmKB, const float *__restrict__ cent,
+                 const float *__restrict__ cw, int BH, int nqb, int nkb, int C, float scale_log2,
+                 float *__restrict__ scores, int *flag)
 {
-    constexpr int CMAX = 8, TJ = 64, BS = TJ + 2;
-    extern __shared__ __align__(16) float smem_f[];
-    float *As = smem_f;                 // [8 warps][D][CMAX]
-    float *Bt = smem_f + 8 * D * CMAX;  // [D][BS]
+    using L = ScSmem<D>;
+    extern __shared__ uint8_t sc_raw[];
+    uint8_t *smem = align_smem_1024(sc_raw);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBar);
+    uint64_t *empty = full + L::kStages;
+    uint64_t *tfull = empty + L::kStages;
+    uint64_t *tempty = tfull + 2;
+    uint64_t *drain = tempty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
 
-    const int bh = blockIdx.y;
+    const int g = blockIdx.x, bh = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qb = blockIdx.x * 8 + warp;
-    const bool row_ok = qb < nqb;
 
-    // centroids of this warp's query block, transposed to [i][c]; absent ones are 0
-    for (int e = lane; e < D * CMAX; e += 32) {
-        const int i = e / CMAX, c = e % CMAX;
-        float v = 0.f;
-        if (row_ok && c < C) v = cent[(((size_t)bh * nqb + qb) * C + c) * D + i];
-        As[(warp * D + i) * CMAX + c] = v;
-    }
-    float wc[CMAX];
+    // centroid terms (A operand), all threads
+    {
+        constexpr int CH = D / 8;
+        for (int pi = tid; pi < 128 * CH; pi += kScThreads) {
+            const int row = pi / CH, k0 = (pi % CH) * 8;
+            const int qb = g * 16 + (row >> 3), c = row & 7;
+            float x[8];
+            if (qb < nqb && c < C) {
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    cent + (((size_t)bh * nqb + qb) * C + c) * D + k0);
+                const float4 u = __ldg(src), v = __ldg(src + 1);
+                x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+                x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+            } else {
 #pragma unroll
-    for (int c = 0; c < CMAX; ++c)
-        wc[c] = (row_ok && c < C) ? cw[((size_t)bh * nqb + qb) * C + c] : 0.f;
-
-    const float *kb = kbar + (size_t)bh * nkb * D;
-    const int ntiles = (nkb + TJ - 1) / TJ;
-    float m[CMAX], z[CMAX];
+                for (int e = 0; e < 8; ++e) x[e] = 0.f;
+            }
+            uint4 t[3];
+            split3x8(x, t);
 #pragma unroll
-    for (int c = 0; c < CMAX; ++c) {
-        m[c] = -INFINITY;
-        z[c] = 0.f;
-    }
-
-    for (int pass = 0; pass < 2; ++pass) {
-        float coef[CMAX];
-        if (pass == 1) {
-#pragma unroll
-            for (int c = 0; c < CMAX; ++c) coef[c] = (c < C && z[c] > 0.f) ? wc[c] / z[c] : 0.f;
+            for (int s = 0; s < 3; ++s)
+                *reinterpret_cast<uint4 *>(smem + L::kA + s * L::kATerm + sw128_chunk(row, k0, 16384)) = t[s];
         }
-        for (int tj = 0; tj < ntiles; ++tj) {
-            const int j0 = tj * TJ;
-            __syncthreads();
-            for (int e = tid; e < TJ * D; e += 256) {
-                const int jj = e / D, i = e % D;
-                Bt[i * BS + jj] = (j0 + jj < nkb) ? kb[(size_t)(j0 + jj) * D + i] : 0.f;
-            }
-            __syncthreads();
-            float L0[CMAX], L1[CMAX];
-#pragma unroll
-            for (int c = 0; c < CMAX; ++c) L0[c] = L1[c] = 0.f;
-            const float *a = As + warp * D * CMAX;
-#pragma unroll 4
-            for (int i = 0; i < D; ++i) {
-                const float4 a0 = *reinterpret_cast<const float4 *>(a + i * CMAX);
-                const float4 a1 = *reinterpret_cast<const float4 *>(a + i * CMAX + 4);
-                const float2 b = *reinterpret_cast<const float2 *>(Bt + i * BS + 2 * lane);
-                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                for (int c = 0; c < CMAX; ++c) {
-                    L0[c] = fmaf(av[c], b.x, L0[c]);
-                    L1[c] = fmaf(av[c], b.y, L1[c]);
+    }
+    if (tid == 0) {
+        for (int s = 0; s < L::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 128);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, kScTmemCols);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int nch = (nkb + kScChunk - 1) / kScChunk;
+    const int njobs = nch == 1 ? 1 : 2 * nch;
+    auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, flag));
+    };
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (elect_one()) prefetch_tmap(&tmKB);
+        __syncwarp();
+        int pos = 0;
+        bool ok = true;
+        for (int j = 0; j < njobs && ok; ++j) {
+            const int ch = j < nch ? j : j - nch;
+            const int ns = (min(kScChunk, nkb - ch * kScChunk) + 63) >> 6;
+            for (int st = 0; st < ns; ++st) {
+                const int s = pos % L::kStages;
+                if (!wait(&empty[s], ((pos / L::kStages) & 1) ^ 1)) {
+                    ok = false;
+                    break;
                 }
-            }
-            const int ja = j0 + 2 * lane, jb = ja + 1;
-            if (pass == 0) {
+                if (elect_one()) {
+                    uint8_t *dst = smem + L::kB + s * L::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], L::kStageBytes);
 #pragma unroll
-                for (int c = 0; c < CMAX; ++c) {
-                    const float x0 = L0[c] * scale, x1 = L1[c] * scale;
-                    float mx = m[c];
-                    if (ja < nkb) mx = fmaxf(mx, x0);
-                    if (jb < nkb) mx = fmaxf(mx, x1);
-                    float zz = (m[c] == -INFINITY) ? 0.f : z[c] * expf(m[c] - mx);
-                    if (ja < nkb) zz += expf(x0 - mx);
-                    if (jb < nkb) zz += expf(x1 - mx);
-                    m[c] = mx;
-                    z[c] = zz;
+                    for (int t = 0; t < 3; ++t)
+#pragma unroll
+                        for (int h = 0; h < L::kPanels; ++h)
+                            tma_load_3d(dst + t * L::kBTerm + h * 8192, &tmKB, &full[s], h * 64,
+                                        ch * kScChunk + st * 64, t * BH + bh);
                 }
-            } else if (row_ok) {
-                float s0 = 0.f, s1 = 0.f;
+                __syncwarp();
+                ++pos;
+            }
+        }
+        if (!ok) {
+            // drain: the last loads issued may still be in flight
+            if (elect_one()) {
+                for (int k = pos - 1; k >= 0 && k >= pos - L::kStages; --k)
+                    drain_wait(&full[k % L::kStages], (k / L::kStages) & 1);
+            }
+            __syncwarp();
+        }
+    } else if (warp == 1) {
+        // ------------------------------- MMA issuer -------------------------------
+        const uint64_t a0 = smem_desc_sw128(smem_u32(smem + L::kA), 16, 1024);
+        const uint64_t b0 = smem_desc_sw128(smem_u32(smem + L::kB), 16, 1024);
+        constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
+        int pos = 0;
+        bool ok = true;
+        for (int j = 0; j < njobs && ok; ++j) {
+            const int buf = j & 1;
+            const int ch = j < nch ? j : j - nch;
+            const int ns = (min(kScChunk, nkb - ch * kScChunk) + 63) >> 6;
+            if (j >= 2 && !wait(&tempty[buf], ((j >> 1) - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            for (int st = 0; st < ns; ++st) {
+                const int s = pos % L::kStages;
+                if (!wait(&full[s], (pos / L::kStages) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + buf * kScChunk + st * 64;
+                const uint64_t bs = b0 + (uint64_t)((s * L::kStageBytes) >> 4);
+                if (elect_one()) {
 #pragma unroll
-                for (int c = 0; c < CMAX; ++c) {
-                    if (c < C) {
-                        s0 = fmaf(coef[c], expf(L0[c] * scale - m[c]), s0);
-                        s1 = fmaf(coef[c], expf(L1[c] * scale - m[c]), s1);
+                    for (int pr = 0; pr < 6; ++pr) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int ta = prod_term_a(pr), tb = prod_term_b(pr);
+                            mma_ss(d_tmem,
+                                   a0 + (uint64_t)((ta * L::kATerm + (kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                                   bs + (uint64_t)((tb * L::kBTerm + (kk >> 2) * 8192 + (kk & 3) * 32) >> 4),
+                                   idesc, (pr | kk) != 0 ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(&empty[s]);
+                }
+                __syncwarp();
+                ++pos;
+            }
+            if (!ok) break;
+            if (elect_one()) mma_commit(&tfull[buf]);
+            __syncwarp();
+        }
+        if (!ok) {
+            if (elect_one()) {
+                mma_commit(drain);
+                drain_wait(drain, 0);
+            }
+            __syncwarp();
+        }
+    } else {
+        // -------------------------------- epilogue --------------------------------
+        const int qd = warp & 3;
+        const int row = qd * 32 + lane;
+        const int qb = g * 16 + (row >> 3), c = row & 7;
+        const bool row_ok = qb < nqb;
+        const float wr = (row_ok && c < C) ? __ldg(cw + ((size_t)bh * nqb + qb) * C + c) : 0.f;
+        float *dst = scores + ((size_t)bh * nqb + (row_ok ? qb : 0)) * nkb;
+        const uint32_t t_lane = tmem + ((uint32_t)(qd * 32) << 16);
+        const int r8 = lane & 7;
+        const bool b4 = (r8 & 4) != 0, b2 = (r8 & 2) != 0, b1 = (r8 & 1) != 0;
+        float m = -INFINITY, z = 0.f, coef = 0.f;
+        for (int j = 0; j < njobs; ++j) {
+            const int buf = j & 1;
+            const int ch = j < nch ? j : j - nch;
+            if (!wait(&tfull[buf], (j >> 1) & 1)) break;
+            tc_fence_after();
+            const int c0 = ch * kScChunk;
+            const int ncols = min(kScChunk, nkb - c0);
+            const int nsl = (ncols + 31) >> 5;
+            const uint32_t tb = t_lane + buf * kScChunk;
+            if (j < nch) {
+                // row statistics in log2 units: max, then the sum of 2^(x - max)
+                float mx = m;
+                for (int sl = 0; sl < nsl; ++sl) {
+                    uint32_t v[32];
+                    tmem_ld32(tb + sl * 32, v);
+                    tmem_wait_ld();
+                    const int lim = ncols - sl * 32;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < lim) mx = fmaxf(mx, __uint_as_float(v[i]) * scale_log2);
+                }
+                float zz = m == -INFINITY ? 0.f : z * fast_exp2(m - mx);
+                for (int sl = 0; sl < nsl; ++sl) {
+                    uint32_t v[32];
+                    tmem_ld32(tb + sl * 32, v);
+                    tmem_wait_ld();
+                    const int lim = ncols - sl * 32;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < lim) zz += fast_exp2(fmaf(__uint_as_float(v[i]), scale_log2, -mx));
+                }
+                m = mx;
+                z = zz;
+                if (j == nch - 1) coef = z > 0.f ? wr / z : 0.f;
+            }
+            if (nch == 1 || j >= nch) {
+                for (int sl = 0; sl < nsl; ++sl) {
+                    uint32_t v[32];
+                    tmem_ld32(tb + sl * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        float e[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            e[i] = coef * fast_exp2(fmaf(__uint_as_float(v[q8 * 8 + i]), scale_log2, -m));
+                        // sum over the 8 rows (lanes) of this query block; lane r8 ends
+                        // with column q8 * 8 + r8
+                        float u[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float send = b4 ? e[i] : e[i + 4];
+                            const float keep = b4 ? e[i + 4] : e[i];
+                            u[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+                        }
+                        float w2[2];
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const float send = b2 ? u[i] : u[i + 2];
+                            const float keep = b2 ? u[i + 2] : u[i];
+                            w2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                        }
+                        const float send = b1 ? w2[0] : w2[1];
+                        const float keep = b1 ? w2[1] : w2[0];
+                        const float res = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                        const int col = c0 + sl * 32 + q8 * 8 + r8;
+                        if (row_ok && col < nkb) dst[col] = res;
                     }
                 }
-                float *dst = scores + ((size_t)bh * nqb + qb) * nkb;
-                if (jb < nkb) {
-                    if ((nkb & 1) == 0) {
-                        *reinterpret_cast<float2 *>(dst + ja) = make_float2(s0, s1);
-                    } else {
-                        dst[ja] = s0;
-                        dst[jb] = s1;
-                    }
-                } else if (ja < nkb) {
-                    dst[ja] = s0;
-                }
             }
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
         }
-        if (pass == 0) {
-            // merge (max, sum) across the 32 lanes of the warp
-#pragma unroll
-            for (int c = 0; c < CMAX; ++c) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float mo = __shfl_xor_sync(0xffffffffu, m[c], o);
-                    const float zo = __shfl_xor_sync(0xffffffffu, z[c], o);
-                    const float mx = fmaxf(m[c], mo);
-                    float zz = 0.f;
-                    if (m[c] != -INFINITY) zz += z[c] * expf(m[c] - mx);
-                    if (mo != -INFINITY) zz += zo * expf(mo - mx);
-                    m[c] = mx;
-                    z[c] = zz;
-                }
-            }
-        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kScTmemCols);
     }
 }
 
 // ---------------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------------
-cudaError_t launch_meankey(const void *k, float *kbar, int BH, int N, int N_pad, int d,
-                           cudaStream_t st)
+cudaError_t launch_meankey(const void *k, float *kbar, void *kbar_terms, int BH, int N, int N_pad,
+                           int d, cudaStream_t st)
 {
     const int nkb = N_pad / 128;
     const dim3 grid((unsigned)(BH * nkb));
+    __nv_bfloat16 *kbs = static_cast<__nv_bfloat16 *>(kbar_terms);
     if (d == 128)
-        meankey_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, N, N_pad, nkb);
+        meankey_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, N, N_pad, nkb);
     else
-        meankey_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, N, N_pad, nkb);
+        meankey_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, N, N_pad, nkb);
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_kmeans_t(const void *q, float *cent, float *cw, uint8_t *assign, int BH,
+                                   int N, int N_pad, int C, int T, int *flag, cudaStream_t st)
+{
+    CUtensorMap tm;
+    if (!make_tmap_bf16_3d(&tm, q, D, (uint64_t)N, (uint64_t)BH, (uint64_t)D * 2,
+                           (uint64_t)N_pad * D * 2, 64, 128))
+        return cudaErrorInvalidValue;
+    const int nqb = N_pad / 128;
+    const int smem = KmSmem<D>::kAlloc;
+    cudaError_t e =
+        cudaFuncSetAttribute(kmeans_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kmeans_kernel<D><<<(unsigned)(BH * nqb), 128, smem, st>>>(tm, N, N_pad, nqb, C, T, cent, cw,
+                                                                assign, flag);
     return cudaGetLastError();
 }
 
 cudaError_t launch_kmeans(const void *q, float *cent, float *cw, uint8_t *assign, int BH, int N,
-                          int N_pad, int d, int C, int T, cudaStream_t st)
+                          int N_pad, int d, int C, int T, int *flag, cudaStream_t st)
 {
-    const int nqb = N_pad / 128;
-    const dim3 grid((unsigned)(BH * nqb));
-    if (d == 128) {
-        const int smem = KmSmem<128>::kBytes;
-        cudaError_t e = cudaFuncSetAttribute(kmeans_kernel<128>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        kmeans_kernel<128><<<grid, 128, smem, st>>>((const __nv_bfloat16 *)q, N, N_pad, nqb, C, T,
-                                                    cent, cw, assign);
-    } else {
-        const int smem = KmSmem<64>::kBytes;
-        cudaError_t e = cudaFuncSetAttribute(kmeans_kernel<64>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        kmeans_kernel<64><<<grid, 128, smem, st>>>((const __nv_bfloat16 *)q, N, N_pad, nqb, C, T,
-                                                   cent, cw, assign);
-    }
+    return d == 128 ? launch_kmeans_t<128>(q, cent, cw, assign, BH, N, N_pad, C, T, flag, st)
+                    : launch_kmeans_t<64>(q, cent, cw, assign, BH, N, N_pad, C, T, flag, st);
+}
+
+template <int D>
+static cudaError_t launch_score_t(const float *cent, const float *cw, const void *kbar_terms,
+                                  float *scores, int BH, int nqb, int nkb, int C, int *flag,
+                                  cudaStream_t st)
+{
+    CUtensorMap tm;
+    if (!make_tmap_bf16_3d(&tm, kbar_terms, D, (uint64_t)nkb, (uint64_t)3 * BH, (uint64_t)D * 2,
+                           (uint64_t)nkb * D * 2, 64, 64))
+        return cudaErrorInvalidValue;
+    const int smem = ScSmem<D>::kAlloc;
+    cudaError_t e =
+        cudaFuncSetAttribute(score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    const dim3 grid((unsigned)((nqb + 15) / 16), (unsigned)BH);
+    score_kernel<D><<<grid, kScThreads, smem, st>>>(tm, cent, cw, BH, nqb, nkb, C, scale_log2,
+                                                    scores, flag);
     return cudaGetLastError();
 }
 
-cudaError_t launch_score(const float *cent, const float *cw, const float *kbar, float *scores,
-                         int BH, int nqb, int nkb, int d, int C, cudaStream_t st)
+cudaError_t launch_score(const float *cent, const float *cw, const void *kbar_terms, float *scores,
+                         int BH, int nqb, int nkb, int d, int C, int *flag, cudaStream_t st)
 {
-    const dim3 grid((unsigned)((nqb + 7) / 8), (unsigned)BH);
-    const float scale = (float)(1.0 / sqrt((double)d));
-    const size_t smem = sizeof(float) * (8 * d * 8 + d * 66);
-    if (d == 128) {
-        cudaError_t e = cudaFuncSetAttribute(score_kernel<128>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        score_kernel<128><<<grid, 256, smem, st>>>(cent, cw, kbar, nqb, nkb, C, scale, scores);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(score_kernel<64>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        score_kernel<64><<<grid, 256, smem, st>>>(cent, cw, kbar, nqb, nkb, C, scale, scores);
-    }
-    return cudaGetLastError();
+    return d == 128 ? launch_score_t<128>(cent, cw, kbar_terms, scores, BH, nqb, nkb, C, flag, st)
+                    : launch_score_t<64>(cent, cw, kbar_terms, scores, BH, nqb, nkb, C, flag, st);
 }
 
 }  // namespace ab

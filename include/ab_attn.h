@@ -74,8 +74,9 @@ typedef struct {
 
 /*
  * ab_score_workspace_size -- bytes of device scratch ab_score() needs for shape `s`
- * and `n_clusters`: the mean keys [B,H,n_kb,d] fp32, the centroids [B,H,n_qb,C,d] fp32
- * and the cluster weights [B,H,n_qb,C] fp32, each region 256-byte aligned.
+ * and `n_clusters`: the mean keys [B,H,n_kb,d] fp32, the centroids [B,H,n_qb,C,d] fp32,
+ * the cluster weights [B,H,n_qb,C] fp32 and the mean keys' exact three-term bf16 split
+ * [3,B,H,n_kb,d] (operands of the tensor-core block score), each region 256-byte aligned.
  * Returns AB_ERR_* for an invalid shape; *bytes is then 0.
  */
 ab_status ab_score_workspace_size(ab_shape s, int n_clusters, size_t *bytes);
@@ -117,13 +118,13 @@ ab_status ab_score(const void *q, const void *k, ab_shape s, int n_clusters, int
  * custom operator running inside a host framework that owns all device memory and
  * forbids allocation on its execution path, or code that has no allocator of its own.
  * This call computes exactly what ab_score computes (scores only; no optional
- * outputs), with its scratch (mean keys, centroids, cluster weights) in a fixed array
+ * outputs), with its scratch (the regions of ab_score_workspace_size) in a fixed array
  * of AB_NOALLOC_SCRATCH_BYTES bytes in the library's own device memory. That array
  * exists once on every GPU that loads the library and stays allocated until the
  * process exits. The call itself allocates nothing.
  *   - Scratch needed = ab_score_workspace_size(s, n_clusters); larger problems are
  *     rejected with AB_ERR_WORKSPACE (e.g. 12 heads x 32768 tokens, d = 128, C = 8
- *     needs 14.3 MB and fits; 24 heads x 118912 tokens does not).
+ *     needs 16.6 MB and fits; 24 heads x 118912 tokens does not).
  *   - The first call on each device looks up the array's device address (with that
  *     device current) and caches it; make that first call before any stream capture.
  *   - Every call uses the same array and leaves its contents behind; every region is
