@@ -28,6 +28,40 @@ __device__ __forceinline__ void split3(float x, __nv_bfloat16 &a, __nv_bfloat16 
     c = __float2bfloat16_rn(r - __bfloat162float(b));
 }
 
+// Round-to-nearest-even of a finite fp32 value to bf16 precision on its bit pattern:
+// add 0x7FFF plus the lowest kept bit, then clear the 16 dropped bits (integer pipe,
+// no conversion unit). The result is an fp32 bit pattern whose upper half is the bf16.
+__device__ __forceinline__ uint32_t rne_bf16_bits(float x)
+{
+    const uint32_t u = __float_as_uint(x);
+    return (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+}
+
+// split3 on the integer pipe: the three terms as fp32 bit patterns (bf16 in the upper half).
+__device__ __forceinline__ void split3_bits(float x, uint32_t &a, uint32_t &b, uint32_t &c)
+{
+    a = rne_bf16_bits(x);
+    const float r = x - __uint_as_float(a);
+    b = rne_bf16_bits(r);
+    c = rne_bf16_bits(r - __uint_as_float(b));
+}
+
+// x / n for a member count n >= 1: hardware reciprocal estimate, quotient, and one
+// Newton residual correction q + (x - q n) r (Markstein's method), within about one ulp
+// of the rounded quotient.
+__device__ __forceinline__ float div_by_count(float x, float n, float r)
+{
+    const float q = x * r;
+    return fmaf(fmaf(-q, n, x), r, q);
+}
+
+__device__ __forceinline__ float rcp_approx(float n)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(n));
+    return r;
+}
+
 // The same for 8 consecutive values, packed as three 16-byte rows (hi, mid, lo).
 __device__ __forceinline__ void split3x8(const float (&x)[8], uint4 (&t)[3])
 {
@@ -126,16 +160,18 @@ __global__ void __launch_bounds__(256) meankey_kernel(const __nv_bfloat16 *__res
 //           exact 0/1 and bf16 operands with fp32 accumulation, divided by the member
 //           counts; thread i reads TMEM lane i = feature i; an empty cluster keeps its
 //           centroid.
-// All 128 threads stage the operands; one elected thread of warp 0 issues the MMAs.
-// Every wait is bounded; a timed-out CTA drains its in-flight work and exits.
+// Thread i keeps feature i of the 8 centroids in registers: after each update it
+// writes column i of the next assignment's B operand and its share of the squared
+// norms (reduced across the warp, then across the 4 warps through shared memory).
+// One elected thread of warp 0 issues the MMAs. Every wait is bounded; a timed-out
+// CTA drains its in-flight work and exits.
 // ---------------------------------------------------------------------------------
 template <int D>
 struct KmSmem {
     static constexpr int kQ = 0;                        // queries: 2 panels [128][64] bf16
     static constexpr int kBA = kQ + 2 * 16384;          // centroid terms: (D/64) x [32][64]
     static constexpr int kBU = kBA + (D / 64) * 4096;   // one-hot: 2 panels [16][64]
-    static constexpr int kCS = kBU + 2 * 2048;          // fp32 centroids [8][D]
-    static constexpr int kBar = kCS + 8 * D * 4;        // q_full, mma_done, drain
+    static constexpr int kBar = kBU + 2 * 2048;         // q_full, mma_done, drain
     static constexpr int kMisc = kBar + 3 * 8;          // TMEM base, abort flag
     static constexpr int kBytes = kMisc + 8;
     static constexpr int kAlloc = kBytes + 1024;        // slack to align the base to 1024 B
@@ -143,8 +179,49 @@ struct KmSmem {
 
 constexpr int kKmTmemCols = 64;  // G in columns 0..31, S in columns 32..47
 
+// Write feature k of the 8 centroids as column k of the assignment GEMM's B operand
+// (three bf16 terms each) and the warp's partial squared norms to normw[c][warp].
 template <int D>
-__global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUtensorMap tmQ,
+__device__ __forceinline__ void km_publish(uint8_t *smem, const float (&cur)[8], int k,
+                                           bool has_k, int warp, int lane, float (*normw)[4])
+{
+    uint16_t *ba = reinterpret_cast<uint16_t *>(smem + KmSmem<D>::kBA);
+    float sq[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        sq[c] = cur[c] * cur[c];
+        if (has_k) {
+            uint32_t t0, t1, t2;
+            split3_bits(cur[c], t0, t1, t2);
+            // rows c, 8 + c, 16 + c share the swizzle phase (row mod 8 = c)
+            const int o = (sw128_chunk(c, k, 4096) >> 1) + (k & 7);
+            ba[o] = (uint16_t)(t0 >> 16);
+            ba[o + 8 * 64] = (uint16_t)(t1 >> 16);
+            ba[o + 16 * 64] = (uint16_t)(t2 >> 16);
+        }
+    }
+    // reduce-scatter across the warp: lane L ends with cluster (L >> 2) & 7
+    const bool b16 = (lane & 16) != 0, b8 = (lane & 8) != 0, b4 = (lane & 4) != 0;
+    float u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = b16 ? sq[i] : sq[i + 4], keep = b16 ? sq[i + 4] : sq[i];
+        u[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    float w2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = b8 ? u[i] : u[i + 2], keep = b8 ? u[i + 2] : u[i];
+        w2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    float v = (b4 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b4 ? w2[0] : w2[1], 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    if ((lane & 3) == 0) normw[(lane >> 2) & 7][warp] = v;
+}
+
+template <int D>
+__global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                      int N, int N_pad, int nqb, int C, int T,
                                                      float *__restrict__ cent_out,
                                                      float *__restrict__ w_out,
@@ -154,21 +231,21 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
     constexpr int CMAX = 8;
     extern __shared__ uint8_t km_raw[];
     uint8_t *smem = align_smem_1024(km_raw);
-    __shared__ float cn[CMAX];
-    __shared__ int wcount[4][CMAX];
+    __shared__ __align__(16) float normw[CMAX][4];  // squared-norm partials per warp
+    __shared__ __align__(16) int wcount[CMAX][4];   // member counts per warp
     __shared__ uint8_t lab[128];
     uint64_t *q_full = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint64_t *mma_done = q_full + 1;
     uint64_t *drain = q_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
-    float *cs = reinterpret_cast<float *>(smem + L::kCS);
 
     const int blk = blockIdx.x;
     const int bh = blk / nqb, qb = blk % nqb;
     const int t0 = qb * 128;
     const int nv = min(128, N - t0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool has_k = tid < D;  // this thread owns feature tid
 
     if (tid == 0) {
         mbar_init(q_full, 1);
@@ -185,9 +262,8 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
     for (int e = tid; e < (D / 64) * 64; e += 128)
         *reinterpret_cast<uint4 *>(smem + L::kBA + (e >> 6) * 4096 + (24 + ((e >> 3) & 7)) * 128 +
                                    (e & 7) * 16) = make_uint4(0, 0, 0, 0);
-    if (tid < 128)
-        *reinterpret_cast<uint4 *>(smem + L::kBU + (tid >> 6) * 2048 + (8 + ((tid >> 3) & 7)) * 128 +
-                                   (tid & 7) * 16) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4 *>(smem + L::kBU + (tid >> 6) * 2048 + (8 + ((tid >> 3) & 7)) * 128 +
+                               (tid & 7) * 16) = make_uint4(0, 0, 0, 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -203,23 +279,26 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
         }
         __syncwarp();
     }
-    bool ok = __syncthreads_and(mbar_wait(q_full, 0, abort_flag, flag));
+    bool ok = mbar_wait(q_full, 0, abort_flag, flag);
 
-    const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(smem + L::kQ);
-    if (ok) {
-        // initial centroid c: the query at block-local index c*floor(nv/C) (min(c, nv-1)
-        // when nv < C)
-        for (int e = tid; e < CMAX * D; e += 128) {
-            const int c = e / D, i = e % D;
-            float v = 0.f;
-            if (c < C) {
-                const int src = nv >= C ? c * (nv / C) : min(c, nv - 1);
-                v = __bfloat162float(qs[(sw128_chunk(src, i, 16384) >> 1) + (i & 7)]);
-            }
-            cs[c * D + i] = v;
+    // initial centroid c: the query at block-local index c*floor(nv/C) (min(c, nv-1)
+    // when nv < C); this thread holds feature tid of every centroid
+    float cur[CMAX];
+    {
+        const __nv_bfloat16 *qs = reinterpret_cast<const __nv_bfloat16 *>(smem + L::kQ);
+        const int stride = nv / C;
+#pragma unroll
+        for (int c = 0; c < CMAX; ++c) {
+            const int src = nv >= C ? c * stride : min(c, nv - 1);
+            cur[c] = (ok && has_k && c < C)
+                         ? __bfloat162float(qs[(sw128_chunk(src, tid, 16384) >> 1) + (tid & 7)])
+                         : 0.f;
         }
-        __syncthreads();
     }
+    km_publish<D>(smem, cur, tid, has_k, warp, lane, normw);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
 
     const uint32_t q_addr = smem_u32(smem + L::kQ);
     const uint64_t a_asg = smem_desc_sw128(q_addr, 16, 1024);
@@ -232,34 +311,8 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
     uint32_t phase = 0;
 
     for (int it = 0; it < T && ok; ++it) {
-        // (1) centroid terms (B of the assignment GEMM) and squared norms
-        {
-            constexpr int CH = D / 8;
-            if (tid < CMAX * CH) {
-                const int c = tid / CH, k0 = (tid % CH) * 8;
-                const float4 x0 = *reinterpret_cast<const float4 *>(cs + c * D + k0);
-                const float4 x1 = *reinterpret_cast<const float4 *>(cs + c * D + k0 + 4);
-                const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                uint4 t[3];
-                split3x8(xs, t);
-#pragma unroll
-                for (int s = 0; s < 3; ++s)
-                    *reinterpret_cast<uint4 *>(smem + L::kBA + sw128_chunk(8 * s + c, k0, 4096)) = t[s];
-            }
-            for (int c = warp; c < CMAX; c += 4) {
-                float sq = 0.f;
-                for (int i = lane; i < D; i += 32) sq = fmaf(cs[c * D + i], cs[c * D + i], sq);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-                if (lane == 0) cn[c] = sq;
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
         tc_fence_after();
-
-        // (2) assignment GEMM
+        // (1) assignment GEMM
         if (warp == 0) {
             if (elect_one()) {
 #pragma unroll
@@ -270,6 +323,12 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
                 mma_commit(mma_done);
             }
             __syncwarp();
+        }
+        float cn[CMAX];
+#pragma unroll
+        for (int c = 0; c < CMAX; ++c) {
+            const float4 p = *reinterpret_cast<const float4 *>(normw[c]);
+            cn[c] = (p.x + p.y) + (p.z + p.w);
         }
         bool good = __all_sync(0xffffffffu, mbar_wait(mma_done, phase, abort_flag, flag));
         phase ^= 1;
@@ -297,14 +356,14 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
             }
             const int a = tid < nv ? arg : 255;
             lab[tid] = (uint8_t)a;
-            // (3) one-hot column of this query (B of the update GEMM) and member counts
+            // (2) one-hot column of this query (B of the update GEMM) and member counts
             __nv_bfloat16 *oh = reinterpret_cast<__nv_bfloat16 *>(smem + L::kBU);
 #pragma unroll
             for (int c = 0; c < CMAX; ++c) {
                 oh[(sw128_chunk(c, tid, 2048) >> 1) + (tid & 7)] =
                     __ushort_as_bfloat16(a == c ? (unsigned short)0x3F80u : (unsigned short)0u);
                 const unsigned m = __ballot_sync(0xffffffffu, a == c);
-                if (lane == 0) wcount[warp][c] = __popc(m);
+                if (lane == 0) wcount[c][warp] = __popc(m);
             }
         }
         fence_proxy_async_smem();
@@ -313,7 +372,7 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
         if (!ok) break;
         tc_fence_after();
 
-        // (4) update GEMM
+        // (3) update GEMM
         if (warp == 0) {
             if (elect_one()) {
 #pragma unroll
@@ -325,6 +384,12 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
             }
             __syncwarp();
         }
+        int cnt[CMAX];
+#pragma unroll
+        for (int c = 0; c < CMAX; ++c) {
+            const int4 w4 = *reinterpret_cast<const int4 *>(wcount[c]);
+            cnt[c] = (w4.x + w4.y) + (w4.z + w4.w);
+        }
         good = __all_sync(0xffffffffu, mbar_wait(mma_done, phase, abort_flag, flag));
         phase ^= 1;
         tc_fence_after();
@@ -332,24 +397,33 @@ __global__ void __launch_bounds__(128) kmeans_kernel(const __grid_constant__ CUt
             uint32_t sv[16];
             tmem_ld16(t_lane + 32, sv);
             tmem_wait_ld();
-            if (tid < D) {
+            // lanes >= d (d = 64) hold rows of an unused panel: ignored
+            if (has_k) {
 #pragma unroll
                 for (int c = 0; c < CMAX; ++c) {
-                    const int n = wcount[0][c] + wcount[1][c] + wcount[2][c] + wcount[3][c];
-                    if (c < C && n > 0) cs[c * D + tid] = __uint_as_float(sv[c]) / (float)n;
+                    if (c < C && cnt[c] > 0) {
+                        const float n = (float)cnt[c];
+                        cur[c] = div_by_count(__uint_as_float(sv[c]), n, rcp_approx(n));
+                    }
                 }
             }
         }
+        // (4) next assignment's B operand and squared norms
+        km_publish<D>(smem, cur, tid, has_k, warp, lane, normw);
+        fence_proxy_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(good);
     }
 
     if (ok) {
-        const size_t rowc = (size_t)blk * C;
-        for (int e = tid; e < C * D; e += 128) cent_out[rowc * D + e] = cs[e];
+        if (has_k) {
+#pragma unroll
+            for (int c = 0; c < CMAX; ++c)
+                if (c < C) cent_out[((size_t)blk * C + c) * D + tid] = cur[c];
+        }
         if (tid < C) {
-            const int n = wcount[0][tid] + wcount[1][tid] + wcount[2][tid] + wcount[3][tid];
-            w_out[rowc + tid] = (float)n / (float)nv;
+            const int4 w4 = *reinterpret_cast<const int4 *>(wcount[tid]);
+            w_out[(size_t)blk * C + tid] = (float)((w4.x + w4.y) + (w4.z + w4.w)) / (float)nv;
         }
         if (assign_out) assign_out[(size_t)bh * N_pad + t0 + tid] = lab[tid];
     } else if (warp == 0) {
