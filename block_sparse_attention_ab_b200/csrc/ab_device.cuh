@@ -300,6 +300,14 @@ __device__ __forceinline__ float fast_log2(float x)
     return y;
 }
 
+// max of three (sm_100a three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ float fast_exp2(float x)
 {
     float y;

@@ -16,9 +16,11 @@
 //              fetched by block index with 3-D tensor maps whose row extent is N, so
 //              rows past the sequence end arrive as zeros;
 //   warp 9     TMEM owner and MMA issuer: S = Q K^T (both operands from shared
-//              memory) into one of two S buffers, O += P V (P from TMEM).
+//              memory) into S buffer g mod 3, O += P V (P from TMEM).
 // Issue order of the MMA warp over the CTA's whole block stream g = 0, 1, ...:
-//   S(0), S(1), PV(0), S(2), PV(1), ...  so S(g+1) runs while block g is in softmax.
+//   S(0), S(1), S(2), PV(0), S(3), PV(1), S(4), ...  S runs three blocks ahead, so the
+// softmax never waits for a QK^T product, and nothing in the softmax waits for a PV
+// product except an O rescale (PV(g-1)) and the end of an item (PV(g)).
 // Every wait is bounded (2 s); on a timeout the roles unwind, drain their own
 // asynchronous work and the CTA frees its TMEM before returning.
 #include <cmath>
@@ -36,7 +38,8 @@ namespace ab {
 constexpr int kAttnThreads = 320;  // 8 softmax warps, 1 TMA warp, 1 MMA warp
 constexpr int kWarpTma = 8, kWarpMma = 9;
 constexpr int kTmemCols = 512;
-constexpr int kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr int kSBufs = 3;  // S / P buffers in TMEM, columns 128 b .. 128 b + 127
+constexpr int kColO = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 256 without a rescale
 
 struct AttnParams {
@@ -59,9 +62,9 @@ struct AttnSmem {
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2],
-    // o_full, drain
-    static constexpr int kNumBars = 2 + 2 + kStages + kStages + 2 + 2 + 1 + 1;
+    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[3], p_full[3],
+    // o_full[3], drain
+    static constexpr int kNumBars = 2 + 2 + kStages + kStages + 3 * kSBufs + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kXchOff = kMiscOff + 16;  // softmax exchange: float [2][2][128] + [2][128]
     static constexpr int kBytes = kXchOff + (2 * 2 * 128 + 2 * 128) * 4;
@@ -133,9 +136,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint64_t *kv_full = bars + 4;
     uint64_t *kv_empty = kv_full + L::kStages;
     uint64_t *s_full = kv_empty + L::kStages;
-    uint64_t *p_full = s_full + 2;
-    uint64_t *o_full = p_full + 2;
-    uint64_t *drain = o_full + 1;
+    uint64_t *p_full = s_full + kSBufs;
+    uint64_t *o_full = p_full + kSBufs;
+    uint64_t *drain = o_full + kSBufs;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
 
@@ -145,14 +148,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&q_full[b], 1);
             mbar_init(&q_empty[b], 1);
+        }
+        for (int b = 0; b < kSBufs; ++b) {
             mbar_init(&s_full[b], 1);
             mbar_init(&p_full[b], 256);
+            mbar_init(&o_full[b], 1);
         }
         for (int s = 0; s < L::kStages; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
-        mbar_init(o_full, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -213,21 +218,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ++kv_pos;
             return true;
         };
-        Cursor cur = cursor_first(p);
-        if (cur.r < p.n_items) {
-            ok = load_q(cur) && load_kv(cur, &tmK);
-            while (ok) {
-                Cursor nxt = cur;
-                cursor_next(nxt, p);
-                const bool more = nxt.r < p.n_items;
-                if (more) {
-                    if (nxt.i == 0) ok = load_q(nxt);
-                    ok = ok && load_kv(nxt, &tmK);
-                }
-                ok = ok && load_kv(cur, &tmV);
-                if (!more) break;
-                cur = nxt;
-            }
+        // tile order = the MMA warp's consumption order: K of the first kSBufs blocks,
+        // then V(g), K(g + kSBufs), V(g + 1), ...; a Q tile precedes its item's first K
+        Cursor kc = cursor_first(p), vc = kc;
+        auto next_k = [&]() -> bool {
+            bool r = true;
+            if (kc.i == 0) r = load_q(kc);
+            r = r && load_kv(kc, &tmK);
+            cursor_next(kc, p);
+            return r;
+        };
+        for (int a = 0; a < kSBufs && ok && kc.r < p.n_items; ++a) ok = next_k();
+        while (ok && vc.r < p.n_items) {
+            ok = load_kv(vc, &tmV);
+            cursor_next(vc, p);
+            if (ok && kc.r < p.n_items) ok = next_k();
         }
         if (!ok) {
             // drain: the last loads issued may still be in flight
@@ -262,14 +267,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tc_fence_after();
             const uint64_t qd = q_desc0 + (uint64_t)qbuf * kTileDesc;
             const uint64_t kd = k_desc0 + (uint64_t)s * kTileDesc;
-            const uint32_t d_tmem = tmem + ((g & 1) ? kColS1 : kColS0);
+            const uint32_t d_tmem = tmem + (g % kSBufs) * 128;
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
                     mma_ss(d_tmem, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&s_full[g & 1]);
+                mma_commit(&s_full[g % kSBufs]);
                 mma_commit(&kv_empty[s]);
                 if (c.i == c.n - 1) mma_commit(&q_empty[qbuf]);
             }
@@ -277,45 +282,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ++kv_pos;
             return true;
         };
-        Cursor cur = cursor_first(p);
-        int g = 0;
-        if (cur.r < p.n_items) {
-            ok = issue_s(cur, 0);
-            while (ok) {
-                Cursor nxt = cur;
-                cursor_next(nxt, p);
-                const bool more = nxt.r < p.n_items;
-                if (more && !issue_s(nxt, g + 1)) {
-                    ok = false;
-                    break;
-                }
-                // O (+)= P(g) V(g)
-                if (!wait(&p_full[g & 1], (g >> 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                const int s = kv_pos % L::kStages;
-                if (!wait(&kv_full[s], (kv_pos / L::kStages) & 1)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint64_t vd = v_desc0 + (uint64_t)s * kTileDesc;
-                const uint32_t p_tmem = tmem + ((g & 1) ? kColS1 : kColS0);
-                const uint32_t acc0 = cur.i > 0 ? 1u : 0u;
-                if (elect_one()) {
+        Cursor sc = cursor_first(p), pc = sc;  // next S to issue, next PV to issue
+        int gs = 0;                              // index of the next S
+        for (int a = 0; a < kSBufs && ok && sc.r < p.n_items; ++a) {
+            ok = issue_s(sc, gs++);
+            cursor_next(sc, p);
+        }
+        for (int g = 0; ok && pc.r < p.n_items; ++g) {
+            // O (+)= P(g) V(g)
+            if (!wait(&p_full[g % kSBufs], (g / kSBufs) & 1)) {
+                ok = false;
+                break;
+            }
+            const int s = kv_pos % L::kStages;
+            if (!wait(&kv_full[s], (kv_pos / L::kStages) & 1)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint64_t vd = v_desc0 + (uint64_t)s * kTileDesc;
+            const uint32_t p_tmem = tmem + (g % kSBufs) * 128;
+            const uint32_t acc0 = pc.i > 0 ? 1u : 0u;
+            if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < 128 / 16; ++kk)
-                        mma_ts(tmem + kColO, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)),
-                               idesc_pv, kk > 0 ? 1u : acc0);
-                    mma_commit(&kv_empty[s]);
-                    mma_commit(o_full);
-                }
-                __syncwarp();
-                ++kv_pos;
-                if (!more) break;
-                cur = nxt;
-                ++g;
+                for (int kk = 0; kk < 128 / 16; ++kk)
+                    mma_ts(tmem + kColO, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)),
+                           idesc_pv, kk > 0 ? 1u : acc0);
+                mma_commit(&kv_empty[s]);
+                mma_commit(&o_full[g % kSBufs]);
+            }
+            __syncwarp();
+            ++kv_pos;
+            cursor_next(pc, p);
+            // S(g + kSBufs) reuses the buffer whose P(g) was just consumed (in order)
+            if (sc.r < p.n_items) {
+                ok = issue_s(sc, gs++);
+                cursor_next(sc, p);
             }
         }
         if (!ok) {
@@ -350,9 +352,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         auto wait_bar = [&](uint64_t *bar, uint32_t parity) {
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag));
         };
-        auto wait_o = [&](int k) {  // wait until PV(k) is complete
+        // wait until PV(k) is complete (k = g - 1 for a rescale, k = g at the end of an
+        // item). PV(k) completes phase k / 3 of o_full[k mod 3]. A parity wait is exact
+        // only within one phase of the barrier's state: PV(k - 3) is complete (S(g) was
+        // issued after PV(g - 3) and has completed) and PV(k + 3) cannot complete
+        // before P(k + 3) exists, so it is exact here.
+        auto wait_o = [&](int k) {
             if (o_seen > k) return;
-            wait_bar(o_full, k & 1);
+            wait_bar(&o_full[k % kSBufs], (k / kSBufs) & 1);
             o_seen = k + 1;
         };
         auto lw_of = [&](float wj) -> float {  // log2 of a block weight (0 for top-k)
@@ -386,21 +393,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             const int32_t *idx_row = p.idx + (size_t)r * p.nkb;
             const float *w_row = kWeighted ? p.w + (size_t)r * p.nkb : nullptr;
-            // the block's index and log2 weight are ready before the block starts: the
-            // next block's are loaded during this one and converted after its P is out
+            // block index and weight are loaded two blocks ahead; the next block's log2
+            // weight is taken right after this block's max exchange, while the MUFU unit
+            // is free of exp2 work
             int j = clamp_j(__ldg(idx_row));
             float lw = lw_of(kWeighted ? __ldg(w_row) : 1.f);
+            int j_n1 = 0;
+            float w_n1 = 1.f;
+            if (n > 1) {
+                j_n1 = __ldg(idx_row + 1);
+                if (kWeighted) w_n1 = __ldg(w_row + 1);
+            }
             float m_run = -INFINITY, l_run = 0.f;
             for (int i = 0; i < n; ++i, ++g) {
-                int j_next = 0;
-                float w_next = 1.f;
-                if (i + 1 < n) {
-                    j_next = __ldg(idx_row + i + 1);
-                    if (kWeighted) w_next = __ldg(w_row + i + 1);
+                int j_n2 = 0;
+                float w_n2 = 1.f;
+                if (i + 2 < n) {
+                    j_n2 = __ldg(idx_row + i + 2);
+                    if (kWeighted) w_n2 = __ldg(w_row + i + 2);
                 }
                 const int nvalid = min(128, p.N - j * 128) - half * 64;  // valid columns here
-                const uint32_t s_col = (g & 1) ? kColS1 : kColS0;
-                wait_bar(&s_full[g & 1], (g >> 1) & 1);
+                const uint32_t s_col = (g % kSBufs) * 128;
+                wait_bar(&s_full[g % kSBufs], (g / kSBufs) & 1);
                 tc_fence_after();
                 // the destination registers are only read after tcgen05.wait::ld
                 uint32_t su[64];
@@ -417,19 +431,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (int e = 0; e < 64; ++e)
                         if (e >= nvalid) sv[e] = -INFINITY;
                 }
-                // row max: 8 independent chains, then a tree; the two halves exchange theirs
+                // row max: 8 independent chains of three-input max, then a tree; the two
+                // halves exchange theirs
                 float mx[8];
 #pragma unroll
-                for (int t = 0; t < 8; ++t) mx[t] = sv[t];
-#pragma unroll
-                for (int e = 8; e < 64; e += 8)
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) mx[t] = fmaxf(mx[t], sv[e + t]);
-                mx[0] = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                for (int t = 0; t < 8; ++t) {
+                    mx[t] = fmax3(sv[t], sv[8 + t], sv[16 + t]);
+                    mx[t] = fmax3(mx[t], sv[24 + t], sv[32 + t]);
+                    mx[t] = fmax3(mx[t], sv[40 + t], sv[48 + t]);
+                    mx[t] = fmaxf(mx[t], sv[56 + t]);
+                }
+                mx[0] = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                              fmaxf(mx[6], mx[7]));
                 xmax_sh[((g & 1) * 2 + half) * 128 + row] = mx[0];
                 pair_sync();
                 const float smax = fmaxf(mx[0], xmax_sh[((g & 1) * 2 + (half ^ 1)) * 128 + row]);
+                const float lw_n1 = (kWeighted && i + 1 < n) ? lw_of(w_n1) : 0.f;
                 const float xmax = smax * p.scale_log2 + lw;
                 const float m_new = fmaxf(m_run, xmax);
                 bool rescale = false;
@@ -485,12 +502,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     l_run += a.x + a.y;
                 }
                 tmem_wait_st();
-                if (g > 0) wait_o(g - 1);
                 tc_fence_before();
-                mbar_arrive(&p_full[g & 1]);
+                mbar_arrive(&p_full[g % kSBufs]);
                 if (i + 1 < n) {
-                    j = clamp_j(j_next);
-                    lw = lw_of(w_next);
+                    j = clamp_j(j_n1);
+                    lw = lw_n1;
+                    j_n1 = j_n2;
+                    w_n1 = w_n2;
                 }
 
                 if (i == n - 1) {
