@@ -13,6 +13,11 @@ Metric: dense-equivalent TFLOPS = 4 B H N^2 d / step time (N valid tokens), plus
 sparse-attention kernel's ms/call and its tensor-pipe roofline on selected-block FLOPs
 (4 * 128 * 128 * d per kept (query block, key block) pair).
 
+Also reported, each in its own timed region after the main one: the amortised step
+with plan reuse (score + SIP select once every --reuse steps, attention every step: the
+pages' deployment schedule) and the same attention kernel run dense (every key block
+kept), the comparison the pages make against dense attention.
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 run under torchrun: every rank runs the same workload on its own data (weak
 scaling, no data-path collective); the step time is the max over ranks.
@@ -240,6 +245,47 @@ def run_ours(args, rank, world, local_rank):
     topk_total, topk_stage = timed("topk")
     topk_cnt = int(cnt.sum().item())
 
+    # plan reuse (the pages' deployment schedule): score + SIP select once every
+    # `reuse` steps, attention every step with the plan in force
+    def reuse_step(i):
+        if i % args.reuse == 0:
+            ab.score(qc, kc, w.N, w.n_clusters, w.iters, workspace=ws, out=scores)
+            ab.select(scores, K, "sip", w.sip_seed + i // args.reuse, dev_flag=flag, out=(idx, cnt, wt))
+        ab.attn_fwd(qc, kc, vc, w.N, idx, cnt, wt, dev_flag=flag, out=out)
+
+    for i in range(args.warmup * args.reuse):
+        reuse_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    a, b = ev(), ev()
+    a.record()
+    for i in range(args.steps):
+        reuse_step(i)
+    b.record()
+    torch.cuda.synchronize()
+    barrier()
+    reuse_ms = max_over_ranks(a.elapsed_time(b) / args.steps, world, dev)
+
+    # dense comparison: the same attention kernel with every key block kept (top-k at
+    # budget n_kb, all weights 1)
+    ab.select(scores, nb, "topk", out=(idx, cnt, wt))
+    dense_calls = max(3, args.steps // 30)
+    for _ in range(2):
+        ab.attn_topk_fwd(qc, kc, vc, w.N, idx, cnt, dev_flag=flag, out=out)
+    torch.cuda.synchronize()
+    barrier()
+    a, b = ev(), ev()
+    a.record()
+    for _ in range(dense_calls):
+        ab.attn_topk_fwd(qc, kc, vc, w.N, idx, cnt, dev_flag=flag, out=out)
+    b.record()
+    torch.cuda.synchronize()
+    barrier()
+    dense_ms = max_over_ranks(a.elapsed_time(b) / dense_calls, world, dev)
+    dense_pairs = int(cnt.sum().item())
+    if ab.check_flag(flag) != 0:
+        raise RuntimeError("device flag raised during the benchmark")
+
     ms_step = max_over_ranks(total_ms / args.steps, world, dev)
     attn_ms = float(np.mean(stage_ms[:, 2]))
     dense = dense_equiv_flops(w)
@@ -320,6 +366,16 @@ def run_ours(args, rank, world, local_rank):
                            "frac": round((2 * q.numel() * 2 + scores.numel() * 4) /
                                          (float(np.mean(stage_ms[:, 0])) * 1e-3) / 1e9 /
                                          peaks["hbm_gbs"], 4)},
+        "plan_reuse": {"every": args.reuse,
+                       "ms_per_step": round(reuse_ms, 4),
+                       "value": round(world * dense / (reuse_ms * 1e-3) / 1e12, 2),
+                       "unit": "TFLOPS (dense-equivalent)",
+                       "schedule": f"score + SIP select once per {args.reuse} steps, attention every step"},
+        "dense_attn": {"ms_per_call": round(dense_ms, 4), "sum_cnt": dense_pairs,
+                       "tflops": round(selected_flops(dense_pairs, d) / (dense_ms * 1e-3) / 1e12, 2),
+                       "frac": round(selected_flops(dense_pairs, d) / (dense_ms * 1e-3) / 1e12 /
+                                     peaks["bf16_tflops"], 4),
+                       "note": "same kernel, every key block kept (budget n_kb, weights 1)"},
         "e2e": {"value": round(world * dense / (e2e_ms * 1e-3) / 1e12, 2),
                 "unit": "TFLOPS (dense-equivalent, host buffers in and out)",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
@@ -414,6 +470,8 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="override head count (profiling)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reuse", type=int, default=4,
+                    help="plan reuse period for the amortised-step measurement")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per attention launch from an ncu capture of this kernel")
     args = ap.parse_args()
