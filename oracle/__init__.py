@@ -42,6 +42,10 @@ def lib():
         L.orc_philox4x32_10.argtypes = [P, P, P]
         L.orc_philox4x32_10.restype = None
         L.orc_mean_key.argtypes = [P, i32, i32, i32, i32, i32, P]
+        L.orc_mean_key_u.argtypes = [P, i32, i32, i32, i32, i32, i32, P]
+        L.orc_score_u.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, P]
+        L.orc_attn_rows_u.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P, P, P, i64, P, P,
+                                      P, P, P]
         L.orc_kmeans.argtypes = [P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P]
         L.orc_score.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P]
         L.orc_sip.argtypes = [P, i32, i32, i32, i32, i32, u64, P, P, P, P, P]
@@ -51,7 +55,8 @@ def lib():
         L.orc_dense_attn.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P]
         L.orc_num_threads.argtypes = []
         for name in ("orc_mean_key", "orc_kmeans", "orc_score", "orc_sip", "orc_topk",
-                     "orc_attn_rows", "orc_dense_attn", "orc_num_threads"):
+                     "orc_attn_rows", "orc_dense_attn", "orc_num_threads", "orc_mean_key_u",
+                     "orc_score_u", "orc_attn_rows_u"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -87,11 +92,13 @@ def philox4x32_10(ctr, key) -> np.ndarray:
     return out
 
 
-def mean_key(k, N: int) -> np.ndarray:
+def mean_key(k, N: int, unit: int = BLOCK) -> np.ndarray:
+    """Mean key per key unit of `unit` tokens [B, H, N_pad / unit, d] (units with no
+    valid token are 0)."""
     kb = _bits(k)
     B, H, N_pad, d = kb.shape
-    out = np.zeros((B, H, N_pad // BLOCK, d), dtype=np.float64)
-    rc = lib().orc_mean_key(_ptr(kb), B, H, N, N_pad, d, _ptr(out))
+    out = np.zeros((B, H, N_pad // unit, d), dtype=np.float64)
+    rc = lib().orc_mean_key_u(_ptr(kb), B, H, N, N_pad, d, unit, _ptr(out))
     if rc:
         raise ValueError(f"orc_mean_key rc={rc}")
     return out
@@ -115,7 +122,9 @@ def kmeans(q, N: int, C: int, T: int):
     return cent, wts, assign, gap, inert
 
 
-def score(cent, wts, kbar) -> np.ndarray:
+def score(cent, wts, kbar, n_valid: int = 0) -> np.ndarray:
+    """IBCS scores over the key units of `kbar`; only the first `n_valid` units exist
+    (0 = all), the rest score 0."""
     cent = np.ascontiguousarray(cent, dtype=np.float64)
     wts = np.ascontiguousarray(wts, dtype=np.float64)
     kbar = np.ascontiguousarray(kbar, dtype=np.float64)
@@ -123,16 +132,18 @@ def score(cent, wts, kbar) -> np.ndarray:
     nkb = kbar.shape[2]
     assert kbar.shape == (B, H, nkb, d) and wts.shape == (B, H, nqb, C)
     out = np.zeros((B, H, nqb, nkb), dtype=np.float64)
-    rc = lib().orc_score(_ptr(cent), _ptr(wts), _ptr(kbar), B, H, nqb, nkb, C, d, _ptr(out))
+    rc = lib().orc_score_u(_ptr(cent), _ptr(wts), _ptr(kbar), B, H, nqb, nkb, n_valid or nkb, C,
+                           d, _ptr(out))
     if rc:
         raise ValueError(f"orc_score rc={rc}")
     return out
 
 
-def ibcs_scores(q, k, N: int, C: int = 8, T: int = 5) -> np.ndarray:
-    """End-to-end oracle IBCS: mean keys, k-means, block scores."""
+def ibcs_scores(q, k, N: int, C: int = 8, T: int = 5, unit: int = BLOCK) -> np.ndarray:
+    """End-to-end oracle IBCS: mean keys per key unit, k-means of the 128-query
+    blocks, unit scores (units past the sequence end score 0)."""
     cent, wts, _, _, _ = kmeans(q, N, C, T)
-    return score(cent, wts, mean_key(k, N))
+    return score(cent, wts, mean_key(k, N, unit), n_valid=-(-N // unit))
 
 
 def sip(scores, budget: int, seed: int, with_p: bool = True):
@@ -163,9 +174,11 @@ def topk(scores, budget: int):
     return idx, cnt, w
 
 
-def attn_rows(q, k, v, N: int, idx, cnt, w=None, rows=None, want_num_den: bool = False):
-    """Block-sparse HT attention for the listed (b,h,qb) blocks (flat indices; None =
-    all). Returns (out [n,128,d], lse [n,128], num, den) in fp64."""
+def attn_rows(q, k, v, N: int, idx, cnt, w=None, rows=None, want_num_den: bool = False,
+              unit: int = BLOCK):
+    """Sparse HT attention over key units of `unit` tokens for the listed (b,h,qb)
+    query blocks (flat indices; None = all); idx / w rows have N_pad / unit entries.
+    Returns (out [n,128,d], lse [n,128], num, den) in fp64."""
     qb_, kb_, vb_ = _bits(q), _bits(k), _bits(v)
     B, H, N_pad, d = qb_.shape
     idx = np.ascontiguousarray(idx, dtype=np.int32)
@@ -182,9 +195,9 @@ def attn_rows(q, k, v, N: int, idx, cnt, w=None, rows=None, want_num_den: bool =
     lse = np.zeros((n, BLOCK), dtype=np.float64)
     num = np.zeros((n, BLOCK, d), dtype=np.float64) if want_num_den else None
     den = np.zeros((n, BLOCK), dtype=np.float64) if want_num_den else None
-    rc = lib().orc_attn_rows(_ptr(qb_), _ptr(kb_), _ptr(vb_), B, H, N, N_pad, d, _ptr(idx),
-                             _ptr(cnt), _ptr(wv), n, _ptr(rows_a), _ptr(out), _ptr(lse), _ptr(num),
-                             _ptr(den))
+    rc = lib().orc_attn_rows_u(_ptr(qb_), _ptr(kb_), _ptr(vb_), B, H, N, N_pad, d, unit,
+                               _ptr(idx), _ptr(cnt), _ptr(wv), n, _ptr(rows_a), _ptr(out),
+                               _ptr(lse), _ptr(num), _ptr(den))
     if rc:
         raise ValueError(f"orc_attn_rows rc={rc}")
     return out, lse, num, den

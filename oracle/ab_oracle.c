@@ -92,22 +92,25 @@ void orc_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint3
 }
 
 /* ------------------------------------------------------------------------------
- * Mean key of each 128-token key block (IBCS: "its averaged keys"), over the valid
- * tokens t < N only.  kbar: [B, H, n_kb, d].
+ * Mean key of each key unit of U tokens (IBCS: "its averaged keys"; U = 128 is the
+ * key block, U = 4 the page's fine-grained selection unit, third technique), over
+ * the valid tokens t < N only. A unit with no valid token does not exist: its row is
+ * 0 (the score gives it nothing). kbar: [B, H, N_pad / U, d].
  * ------------------------------------------------------------------------------ */
-int orc_mean_key(const uint16_t *K, int B, int H, int N, int N_pad, int d, double *kbar)
+int orc_mean_key_u(const uint16_t *K, int B, int H, int N, int N_pad, int d, int U, double *kbar)
 {
-    if (!K || !kbar || check_shape(B, H, N, N_pad, d)) return -1;
-    const int64_t nkb = n_blocks_of(N_pad);
-    const int64_t rows = (int64_t)B * H * nkb;
-#pragma omp parallel for schedule(dynamic, 4)
+    if (!K || !kbar || check_shape(B, H, N, N_pad, d) || U < 1 || N_pad % U != 0) return -1;
+    const int64_t nku = N_pad / U;
+    const int64_t rows = (int64_t)B * H * nku;
+#pragma omp parallel for schedule(dynamic, 64)
     for (int64_t r = 0; r < rows; ++r) {
-        const int64_t bh = r / nkb, j = r % nkb;
-        const int64_t t0 = j * ORC_BLOCK;
-        int64_t t1 = t0 + ORC_BLOCK;
+        const int64_t bh = r / nku, j = r % nku;
+        const int64_t t0 = j * U;
+        int64_t t1 = t0 + U;
         if (t1 > N) t1 = N;
         double *out = kbar + r * d;
         for (int i = 0; i < d; ++i) out[i] = 0.0;
+        if (t1 <= t0) continue;
         for (int64_t t = t0; t < t1; ++t) {
             const uint16_t *row = K + (bh * N_pad + t) * d;
             for (int i = 0; i < d; ++i) out[i] += bf16_val(row[i]);
@@ -115,6 +118,11 @@ int orc_mean_key(const uint16_t *K, int B, int H, int N, int N_pad, int d, doubl
         for (int i = 0; i < d; ++i) out[i] /= (double)(t1 - t0);
     }
     return 0;
+}
+
+int orc_mean_key(const uint16_t *K, int B, int H, int N, int N_pad, int d, double *kbar)
+{
+    return orc_mean_key_u(K, B, H, N, N_pad, d, ORC_BLOCK, kbar);
 }
 
 /* ------------------------------------------------------------------------------
@@ -220,14 +228,16 @@ int orc_kmeans(const uint16_t *Q, int B, int H, int N, int N_pad, int d, int C, 
 
 /* ------------------------------------------------------------------------------
  * IBCS block score: for each query block, L[c, j] = cent_c . kbar_j / sqrt(d); a
- * softmax over all key blocks j for each centroid c; s_j = sum_c w_c softmax_j(L[c,.]).
+ * softmax over the existing key units j < nkb_valid for each centroid c;
+ * s_j = sum_c w_c softmax_j(L[c,.]), and s_j = 0 for j >= nkb_valid (units past the
+ * sequence end).
  * cent [B,H,nqb,C,d], wts [B,H,nqb,C], kbar [B,H,nkb,d] -> scores [B,H,nqb,nkb].
  * ------------------------------------------------------------------------------ */
-int orc_score(const double *cent, const double *wts, const double *kbar, int B, int H,
-              int nqb, int nkb, int C, int d, double *scores)
+int orc_score_u(const double *cent, const double *wts, const double *kbar, int B, int H,
+                int nqb, int nkb, int nkb_valid, int C, int d, double *scores)
 {
     if (!cent || !wts || !kbar || !scores || B <= 0 || H <= 0 || nqb <= 0 || nkb <= 0 ||
-        C < 1 || d <= 0)
+        nkb_valid < 1 || nkb_valid > nkb || C < 1 || d <= 0)
         return -1;
     const int64_t rows = (int64_t)B * H * nqb;
     const double scale = 1.0 / sqrt((double)d);
@@ -249,21 +259,27 @@ int orc_score(const double *cent, const double *wts, const double *kbar, int B, 
             for (int c = 0; c < C; ++c) {
                 const double *cv = cent + (r * C + c) * (int64_t)d;
                 double m = -INFINITY;
-                for (int j = 0; j < nkb; ++j) {
+                for (int j = 0; j < nkb_valid; ++j) {
                     double acc = 0.0;
                     for (int i = 0; i < d; ++i) acc += cv[i] * kb[(int64_t)j * d + i];
                     logit[j] = acc * scale;
                     if (logit[j] > m) m = logit[j];
                 }
                 double z = 0.0;
-                for (int j = 0; j < nkb; ++j) z += exp(logit[j] - m);
+                for (int j = 0; j < nkb_valid; ++j) z += exp(logit[j] - m);
                 const double wc = wts[r * C + c];
-                for (int j = 0; j < nkb; ++j) s[j] += wc * exp(logit[j] - m) / z;
+                for (int j = 0; j < nkb_valid; ++j) s[j] += wc * exp(logit[j] - m) / z;
             }
         }
         free(logit);
     }
     return rc;
+}
+
+int orc_score(const double *cent, const double *wts, const double *kbar, int B, int H,
+              int nqb, int nkb, int C, int d, double *scores)
+{
+    return orc_score_u(cent, wts, kbar, B, H, nqb, nkb, nkb, C, d, scores);
 }
 
 /* ------------------------------------------------------------------------------
@@ -458,24 +474,29 @@ int orc_topk(const float *scores, int B, int H, int nqb, int nkb, int budget, in
 }
 
 /* ------------------------------------------------------------------------------
- * Block-sparse attention with Horvitz-Thompson weights, per query row i of query
- * block qb:
+ * Block-sparse attention with Horvitz-Thompson weights over key units of U tokens
+ * (U = 128: key blocks; U = 4: the page's fine-grained units), per query row i of
+ * query block qb (128 queries):
  *   O_i = sum_{j in sel} w_j sum_{t in j, t<N} e^{q_i.k_t/sqrt(d)} v_t
  *         / sum_{j in sel} w_j sum_{t in j, t<N} e^{q_i.k_t/sqrt(d)}
- * (w = NULL means all weights 1, the top-k mode). Rows i >= N are 0 (lse 0); a row
- * with an empty selection is 0 with lse = -inf.
+ * (w = NULL means all weights 1, the top-k mode); unit j holds tokens
+ * [j U, j U + U). Rows i >= N are 0 (lse 0); a row with an empty selection (or only
+ * units past the sequence end) is 0 with lse = -inf. idx / w rows have N_pad / U
+ * entries.
  * The `rows` list picks which (b, h, qb) blocks to compute: flat index
  * (b*H + h)*nqb + qb; NULL means all, in order. Outputs are per listed block:
  * out [n_rows, 128, d], lse [n_rows, 128] (ln of the denominator), and optionally
  * the unshifted numerator num [n_rows, 128, d] and denominator den [n_rows, 128].
  * ------------------------------------------------------------------------------ */
-int orc_attn_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B, int H, int N,
-                  int N_pad, int d, const int32_t *idx, const int32_t *cnt, const float *w,
-                  int64_t n_rows, const int64_t *rows, double *out, double *lse, double *num,
-                  double *den)
+int orc_attn_rows_u(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B, int H,
+                    int N, int N_pad, int d, int U, const int32_t *idx, const int32_t *cnt,
+                    const float *w, int64_t n_rows, const int64_t *rows, double *out,
+                    double *lse, double *num, double *den)
 {
-    if (!Q || !K || !V || !idx || !cnt || !out || check_shape(B, H, N, N_pad, d)) return -1;
-    const int64_t nqb = n_blocks_of(N_pad), nkb = nqb;
+    if (!Q || !K || !V || !idx || !cnt || !out || check_shape(B, H, N, N_pad, d) || U < 1 ||
+        N_pad % U != 0)
+        return -1;
+    const int64_t nqb = n_blocks_of(N_pad), nkb = N_pad / U;
     const int64_t total = (int64_t)B * H * nqb;
     if (!rows) n_rows = total;
     for (int64_t n = 0; n < n_rows; ++n)
@@ -490,7 +511,7 @@ int orc_attn_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B
     int rc = 0;
 #pragma omp parallel
     {
-        double *logit = (double *)malloc(sizeof(double) * nkb * ORC_BLOCK);
+        double *logit = (double *)malloc(sizeof(double) * nkb * U);
         double *qv = (double *)malloc(sizeof(double) * d);
         double *acc = (double *)malloc(sizeof(double) * d);
         if (!logit || !qv || !acc) {
@@ -523,8 +544,8 @@ int orc_attn_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B
                 for (int32_t c = 0; c < nsel; ++c) {
                     const int64_t j = sel[c];
                     const double lw = w ? log((double)w[r * nkb + c]) : 0.0;
-                    for (int t = 0; t < ORC_BLOCK; ++t) {
-                        const int64_t tk = j * ORC_BLOCK + t;
+                    for (int t = 0; t < U; ++t) {
+                        const int64_t tk = j * U + t;
                         if (tk >= N) break;
                         double dot = 0.0;
                         for (int e = 0; e < d; ++e)
@@ -547,8 +568,8 @@ int orc_attn_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B
                 nl = 0;
                 for (int32_t c = 0; c < nsel; ++c) {
                     const int64_t j = sel[c];
-                    for (int t = 0; t < ORC_BLOCK; ++t) {
-                        const int64_t tk = j * ORC_BLOCK + t;
+                    for (int t = 0; t < U; ++t) {
+                        const int64_t tk = j * U + t;
                         if (tk >= N) break;
                         const double pexp = exp(logit[nl++] - m);
                         z += pexp;
@@ -570,6 +591,15 @@ int orc_attn_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B
         free(acc);
     }
     return rc;
+}
+
+int orc_attn_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B, int H, int N,
+                  int N_pad, int d, const int32_t *idx, const int32_t *cnt, const float *w,
+                  int64_t n_rows, const int64_t *rows, double *out, double *lse, double *num,
+                  double *den)
+{
+    return orc_attn_rows_u(Q, K, V, B, H, N, N_pad, d, ORC_BLOCK, idx, cnt, w, n_rows, rows, out,
+                           lse, num, den);
 }
 
 /* ------------------------------------------------------------------------------
