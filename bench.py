@@ -15,8 +15,9 @@ sparse-attention kernel's ms/call and its tensor-pipe roofline on selected-block
 
 Also reported, each in its own timed region after the main one: the amortised step
 with plan reuse (score + SIP select once every --reuse steps, attention every step: the
-pages' deployment schedule) and the same attention kernel run dense (every key block
-kept), the comparison the pages make against dense attention.
+pages' deployment schedule), the same path with the pages' 4-token key units at the same
+tile budget (units gathered 32 per 128-key tile), and the same attention kernel run dense
+(every key block kept), the comparison the pages make against dense attention.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 For N > 1 run under torchrun: every rank runs the same workload on its own data (weak
@@ -286,6 +287,56 @@ def run_ours(args, rank, world, local_rank):
     if ab.check_flag(flag) != 0:
         raise RuntimeError("device flag raised during the benchmark")
 
+    # the page's 4-token key units at the same tile budget (32 units per 128-key tile):
+    # unit scores -> SIP over units -> attention over the gathered units
+    units = None
+    if N_pad // 4 <= 8192:
+        K4 = 32 * K
+        nku = N_pad // 4
+        ws4 = torch.empty(ab.score_workspace_bytes(shape, w.n_clusters, 4), device=dev, dtype=torch.uint8)
+        scores4 = torch.empty(B, H, nb, nku, device=dev, dtype=torch.float32)
+        idx4 = torch.empty(B, H, nb, nku, device=dev, dtype=torch.int32)
+        cnt4 = torch.empty(B, H, nb, device=dev, dtype=torch.int32)
+        wt4 = torch.empty(B, H, nb, nku, device=dev, dtype=torch.float32)
+
+        def unit_step(e=None):
+            if e:
+                e[0].record()
+            ab.score(qc, kc, w.N, w.n_clusters, w.iters, workspace=ws4, out=scores4, unit=4)
+            if e:
+                e[1].record()
+            ab.select(scores4, K4, "sip", w.sip_seed, dev_flag=flag, out=(idx4, cnt4, wt4))
+            if e:
+                e[2].record()
+            ab.attn_fwd(qc, kc, vc, w.N, idx4, cnt4, wt4, dev_flag=flag, out=out, unit=4)
+            if e:
+                e[3].record()
+
+        unit_iters = max(3, args.steps // 30)
+        for _ in range(2):
+            unit_step()
+        torch.cuda.synchronize()
+        barrier()
+        per4 = [[ev() for _ in range(4)] for _ in range(unit_iters)]
+        for i in range(unit_iters):
+            unit_step(per4[i])
+        torch.cuda.synchronize()
+        barrier()
+        st4 = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
+                        for e in per4])
+        tiles4 = int(((cnt4 + 31) // 32).sum().item())
+        attn4 = max_over_ranks(float(np.mean(st4[:, 2])), world, dev)
+        if ab.check_flag(flag) != 0:
+            raise RuntimeError("device flag raised during the unit benchmark")
+        units = {"unit_tokens": 4, "budget_units": K4, "tiles": tiles4,
+                 "kept_units": int(cnt4.sum().item()),
+                 "score_ms": round(float(np.mean(st4[:, 0])), 4),
+                 "select_ms": round(float(np.mean(st4[:, 1])), 4),
+                 "attn_ms": round(attn4, 4),
+                 "ms_per_step": round(max_over_ranks(float(np.mean(st4.sum(1))), world, dev), 4),
+                 "attn_tile_tflops": round(selected_flops(tiles4, d) / (attn4 * 1e-3) / 1e12, 2),
+                 "note": "SIP over 4-token key units, gathered 32 per 128-key tile"}
+
     ms_step = max_over_ranks(total_ms / args.steps, world, dev)
     attn_ms = float(np.mean(stage_ms[:, 2]))
     dense = dense_equiv_flops(w)
@@ -371,6 +422,7 @@ def run_ours(args, rank, world, local_rank):
                        "value": round(world * dense / (reuse_ms * 1e-3) / 1e12, 2),
                        "unit": "TFLOPS (dense-equivalent)",
                        "schedule": f"score + SIP select once per {args.reuse} steps, attention every step"},
+        "units4": units,
         "dense_attn": {"ms_per_call": round(dense_ms, 4), "sum_cnt": dense_pairs,
                        "tflops": round(selected_flops(dense_pairs, d) / (dense_ms * 1e-3) / 1e12, 2),
                        "frac": round(selected_flops(dense_pairs, d) / (dense_ms * 1e-3) / 1e12 /

@@ -73,6 +73,10 @@ def lib():
         L.ab_select.argtypes = [P, I, I, I, I, I, I, ctypes.c_uint64, P, P, P, P, P, P]
         L.ab_attn_fwd.argtypes = [P, P, P, S, P, P, P, P, I, P, P, P]
         L.ab_attn_topk_fwd.argtypes = [P, P, P, S, P, P, P, I, P, P, P]
+        L.ab_score_units_workspace_size.argtypes = [S, I, I, ctypes.POINTER(ctypes.c_size_t)]
+        L.ab_score_units.argtypes = [P, P, S, I, I, I, P, P, P, P, P, P, ctypes.c_size_t, P, P]
+        L.ab_attn_units_fwd.argtypes = [P, P, P, S, I, P, P, P, P, I, P, P, P]
+        L.ab_attn_units_topk_fwd.argtypes = [P, P, P, S, I, P, P, P, I, P, P, P]
         L.ab_check_flag.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
         L.ab_status_str.argtypes = [I]
         L.ab_status_str.restype = ctypes.c_char_p
@@ -80,7 +84,8 @@ def lib():
         L.ab_last_cuda_error.argtypes = []
         L.ab_last_cuda_error.restype = ctypes.c_char_p
         for name in ("ab_score_workspace_size", "ab_score", "ab_score_noalloc", "ab_select", "ab_attn_fwd",
-                     "ab_attn_topk_fwd", "ab_check_flag", "ab_version"):
+                     "ab_attn_topk_fwd", "ab_check_flag", "ab_version", "ab_score_units_workspace_size",
+                     "ab_score_units", "ab_attn_units_fwd", "ab_attn_units_topk_fwd"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -113,35 +118,48 @@ def make_shape(q: torch.Tensor, N: int) -> Shape:
     return Shape(B, H, int(N), N_pad, d, AB_BF16)
 
 
-def score_workspace_bytes(shape: Shape, n_clusters: int = 8) -> int:
+def score_workspace_bytes(shape: Shape, n_clusters: int = 8, unit: int = BLOCK) -> int:
     n = ctypes.c_size_t(0)
-    _check(lib().ab_score_workspace_size(shape, n_clusters, ctypes.byref(n)), "ab_score_workspace_size")
+    if unit == BLOCK:
+        _check(lib().ab_score_workspace_size(shape, n_clusters, ctypes.byref(n)), "ab_score_workspace_size")
+    else:
+        _check(lib().ab_score_units_workspace_size(shape, n_clusters, unit, ctypes.byref(n)),
+               "ab_score_units_workspace_size")
     return int(n.value)
 
 
 def score(q: torch.Tensor, k: torch.Tensor, N: int, n_clusters: int = 8, iters: int = 5,
           intermediates: bool = False, workspace: Optional[torch.Tensor] = None,
-          out: Optional[torch.Tensor] = None):
-    """IBCS block scores [B,H,nqb,nkb] fp32. With intermediates=True also returns
-    (kbar, centroids, cluster weights, assignment)."""
+          out: Optional[torch.Tensor] = None, unit: int = BLOCK):
+    """IBCS scores [B,H,nqb,N_pad/unit] fp32 over key blocks (unit=128) or 4-token key
+    units (unit=4). With intermediates=True also returns (kbar, centroids, cluster
+    weights, assignment)."""
     _need(q, torch.bfloat16, "q")
     _need(k, torch.bfloat16, "k")
     B, H, N_pad, d = q.shape
     nb = N_pad // BLOCK
+    nku = N_pad // unit
     shape = make_shape(q, N)
     dev = q.device
-    scores = out if out is not None else torch.empty(B, H, nb, nb, device=dev, dtype=torch.float32)
+    scores = out if out is not None else torch.empty(B, H, nb, nku, device=dev, dtype=torch.float32)
     kbar = cent = cw = assign = None
     if intermediates:
-        kbar = torch.empty(B, H, nb, d, device=dev, dtype=torch.float32)
+        kbar = torch.empty(B, H, nku, d, device=dev, dtype=torch.float32)
         cent = torch.empty(B, H, nb, n_clusters, d, device=dev, dtype=torch.float32)
         cw = torch.empty(B, H, nb, n_clusters, device=dev, dtype=torch.float32)
         assign = torch.empty(B, H, N_pad, device=dev, dtype=torch.uint8)
     if workspace is None:
-        workspace = torch.empty(score_workspace_bytes(shape, n_clusters), device=dev, dtype=torch.uint8)
-    _check(lib().ab_score(_ptr(q), _ptr(k), shape, n_clusters, iters, _ptr(scores), _ptr(kbar),
-                          _ptr(cent), _ptr(cw), _ptr(assign), _ptr(workspace),
-                          workspace.numel(), None, _stream()), "ab_score")
+        workspace = torch.empty(score_workspace_bytes(shape, n_clusters, unit), device=dev,
+                                dtype=torch.uint8)
+    if unit == BLOCK:
+        _check(lib().ab_score(_ptr(q), _ptr(k), shape, n_clusters, iters, _ptr(scores), _ptr(kbar),
+                              _ptr(cent), _ptr(cw), _ptr(assign), _ptr(workspace),
+                              workspace.numel(), None, _stream()), "ab_score")
+    else:
+        _check(lib().ab_score_units(_ptr(q), _ptr(k), shape, n_clusters, iters, unit, _ptr(scores),
+                                    _ptr(kbar), _ptr(cent), _ptr(cw), _ptr(assign),
+                                    _ptr(workspace), workspace.numel(), None, _stream()),
+               "ab_score_units")
     if intermediates:
         return scores, kbar, cent, cw, assign
     return scores
@@ -194,8 +212,9 @@ def _out_code(out_dtype):
 
 def attn_fwd(q, k, v, N: int, idx, cnt, w, want_lse: bool = False,
              dev_flag: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-             out_dtype=torch.bfloat16):
-    """Block-sparse HT-weighted attention; returns out (bf16 or fp32) [and lse fp32]."""
+             out_dtype=torch.bfloat16, unit: int = BLOCK):
+    """Sparse HT-weighted attention over the kept key blocks (unit=128) or 4-token key
+    units (unit=4); returns out (bf16 or fp32) [and lse fp32]."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, n)
     _need(idx, torch.int32, "idx")
@@ -203,24 +222,35 @@ def attn_fwd(q, k, v, N: int, idx, cnt, w, want_lse: bool = False,
     _need(w, torch.float32, "w")
     o = _out_buffer(q, out, out_dtype)
     lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32) if want_lse else None
-    _check(lib().ab_attn_fwd(_ptr(q), _ptr(k), _ptr(v), make_shape(q, N), _ptr(idx), _ptr(cnt),
-                             _ptr(w), _ptr(o), _out_code(out_dtype), _ptr(lse), _ptr(dev_flag),
-                             _stream()), "ab_attn_fwd")
+    if unit == BLOCK:
+        _check(lib().ab_attn_fwd(_ptr(q), _ptr(k), _ptr(v), make_shape(q, N), _ptr(idx), _ptr(cnt),
+                                 _ptr(w), _ptr(o), _out_code(out_dtype), _ptr(lse), _ptr(dev_flag),
+                                 _stream()), "ab_attn_fwd")
+    else:
+        _check(lib().ab_attn_units_fwd(_ptr(q), _ptr(k), _ptr(v), make_shape(q, N), unit, _ptr(idx),
+                                       _ptr(cnt), _ptr(w), _ptr(o), _out_code(out_dtype), _ptr(lse),
+                                       _ptr(dev_flag), _stream()), "ab_attn_units_fwd")
     return (o, lse) if want_lse else o
 
 
 def attn_topk_fwd(q, k, v, N: int, idx, cnt, want_lse: bool = False,
                   dev_flag: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                  out_dtype=torch.bfloat16):
+                  out_dtype=torch.bfloat16, unit: int = BLOCK):
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, n)
     _need(idx, torch.int32, "idx")
     _need(cnt, torch.int32, "cnt")
     o = _out_buffer(q, out, out_dtype)
     lse = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32) if want_lse else None
-    _check(lib().ab_attn_topk_fwd(_ptr(q), _ptr(k), _ptr(v), make_shape(q, N), _ptr(idx),
-                                  _ptr(cnt), _ptr(o), _out_code(out_dtype), _ptr(lse),
-                                  _ptr(dev_flag), _stream()), "ab_attn_topk_fwd")
+    if unit == BLOCK:
+        _check(lib().ab_attn_topk_fwd(_ptr(q), _ptr(k), _ptr(v), make_shape(q, N), _ptr(idx),
+                                      _ptr(cnt), _ptr(o), _out_code(out_dtype), _ptr(lse),
+                                      _ptr(dev_flag), _stream()), "ab_attn_topk_fwd")
+    else:
+        _check(lib().ab_attn_units_topk_fwd(_ptr(q), _ptr(k), _ptr(v), make_shape(q, N), unit,
+                                            _ptr(idx), _ptr(cnt), _ptr(o), _out_code(out_dtype),
+                                            _ptr(lse), _ptr(dev_flag), _stream()),
+               "ab_attn_units_topk_fwd")
     return (o, lse) if want_lse else o
 
 
@@ -234,10 +264,11 @@ def check_flag(dev_flag: torch.Tensor) -> int:
 
 
 def ab_attention(q, k, v, N: int, budget: int, mode: str = "sip", seed: int = 0,
-                 n_clusters: int = 8, iters: int = 5):
-    """One pass of the whole path: score -> select -> sparse attention (device tensors)."""
-    s = score(q, k, N, n_clusters, iters)
+                 n_clusters: int = 8, iters: int = 5, unit: int = BLOCK):
+    """One pass of the whole path: score -> select -> sparse attention (device tensors).
+    `budget` counts selection units (key blocks, or 4-token units when unit=4)."""
+    s = score(q, k, N, n_clusters, iters, unit=unit)
     idx, cnt, w = select(s, budget, mode, seed)
     if mode == "sip":
-        return attn_fwd(q, k, v, N, idx, cnt, w)
-    return attn_topk_fwd(q, k, v, N, idx, cnt)
+        return attn_fwd(q, k, v, N, idx, cnt, w, unit=unit)
+    return attn_topk_fwd(q, k, v, N, idx, cnt, unit=unit)

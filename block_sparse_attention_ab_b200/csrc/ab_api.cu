@@ -24,9 +24,19 @@ ab_status check_shape(const ab_shape &s)
     return AB_OK;
 }
 
-ab::ScoreLayout score_layout(const ab_shape &s, int C)
+ab::ScoreLayout score_layout(const ab_shape &s, int C, int unit = AB_BLOCK)
 {
-    return ab::score_layout((size_t)s.B * s.H, (size_t)s.N_pad / AB_BLOCK, (size_t)s.d, (size_t)C);
+    return ab::score_layout((size_t)s.B * s.H, (size_t)s.N_pad / AB_BLOCK, (size_t)s.N_pad / unit,
+                            (size_t)s.d, (size_t)C);
+}
+
+// key units accepted by the unit entry points: 128-token blocks or 4-token units, with at
+// most AB_MAX_BLOCKS units per head
+ab_status check_unit(const ab_shape &s, int unit)
+{
+    if (unit != AB_BLOCK && unit != AB_UNIT4) return AB_ERR_UNSUPPORTED;
+    if (s.N_pad / unit > AB_MAX_BLOCKS) return AB_ERR_RANGE;
+    return AB_OK;
 }
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
@@ -38,12 +48,14 @@ ab_status cuda_status(cudaError_t e)
     return AB_ERR_CUDA;
 }
 
-ab_status attn_common(const void *q, const void *k, const void *v, ab_shape s, const int32_t *idx,
-                      const int32_t *cnt, const float *w, void *out, ab_dtype out_dtype,
-                      float *lse, int *dev_flag, void *stream)
+ab_status attn_common(const void *q, const void *k, const void *v, ab_shape s, int unit,
+                      const int32_t *idx, const int32_t *cnt, const float *w, void *out,
+                      ab_dtype out_dtype, float *lse, int *dev_flag, void *stream)
 {
     if (!q || !k || !v || !idx || !cnt || !out) return AB_ERR_NULL;
     ab_status st = check_shape(s);
+    if (st != AB_OK) return st;
+    st = check_unit(s, unit);
     if (st != AB_OK) return st;
     if (out_dtype != AB_BF16 && out_dtype != AB_F32) return AB_ERR_DTYPE;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(idx) ||
@@ -65,6 +77,7 @@ ab_status attn_common(const void *q, const void *k, const void *v, ab_shape s, c
     a.N = s.N;
     a.N_pad = s.N_pad;
     a.d = s.d;
+    a.unit = unit;
     a.grid_override = 0;
     return cuda_status(ab::launch_attn(a, (cudaStream_t)stream));
 }
@@ -84,13 +97,37 @@ ab_status ab_score_workspace_size(ab_shape s, int n_clusters, size_t *bytes)
     return AB_OK;
 }
 
+ab_status ab_score_units_workspace_size(ab_shape s, int n_clusters, int key_unit, size_t *bytes)
+{
+    if (!bytes) return AB_ERR_NULL;
+    *bytes = 0;
+    ab_status st = check_shape(s);
+    if (st != AB_OK) return st;
+    st = check_unit(s, key_unit);
+    if (st != AB_OK) return st;
+    if (n_clusters < 1 || n_clusters > 8) return AB_ERR_UNSUPPORTED;
+    *bytes = score_layout(s, n_clusters, key_unit).total;
+    return AB_OK;
+}
+
 ab_status ab_score(const void *q, const void *k, ab_shape s, int n_clusters, int iters,
                    float *scores, float *kbar, float *centroids, float *cweights,
                    uint8_t *assign, void *workspace, size_t workspace_bytes, int *dev_flag,
                    void *stream)
 {
+    return ab_score_units(q, k, s, n_clusters, iters, AB_BLOCK, scores, kbar, centroids, cweights,
+                          assign, workspace, workspace_bytes, dev_flag, stream);
+}
+
+ab_status ab_score_units(const void *q, const void *k, ab_shape s, int n_clusters, int iters,
+                         int key_unit, float *scores, float *kbar, float *centroids,
+                         float *cweights, uint8_t *assign, void *workspace,
+                         size_t workspace_bytes, int *dev_flag, void *stream)
+{
     if (!q || !k || !scores) return AB_ERR_NULL;
     ab_status st = check_shape(s);
+    if (st != AB_OK) return st;
+    st = check_unit(s, key_unit);
     if (st != AB_OK) return st;
     if (n_clusters < 1 || n_clusters > 8) return AB_ERR_UNSUPPORTED;
     if (iters < 1 || iters > 1000) return AB_ERR_RANGE;
@@ -98,21 +135,23 @@ ab_status ab_score(const void *q, const void *k, ab_shape s, int n_clusters, int
         (centroids && !aligned16(centroids)) || (cweights && !aligned16(cweights)) ||
         !aligned16(workspace))
         return AB_ERR_ALIGN;
-    const ab::ScoreLayout L = score_layout(s, n_clusters);
+    const ab::ScoreLayout L = score_layout(s, n_clusters, key_unit);
     if (!workspace || workspace_bytes < L.total) return AB_ERR_WORKSPACE;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     float *kb = kbar ? kbar : reinterpret_cast<float *>(ws + L.kbar);
     float *ce = centroids ? centroids : reinterpret_cast<float *>(ws + L.cent);
     float *cw = cweights ? cweights : reinterpret_cast<float *>(ws + L.cw);
-    const int BH = s.B * s.H, nb = s.N_pad / AB_BLOCK;
+    const int BH = s.B * s.H, nqb = s.N_pad / AB_BLOCK, nku = s.N_pad / key_unit;
+    const int nku_valid = (s.N + key_unit - 1) / key_unit;  // units holding a valid token
     cudaStream_t cs = (cudaStream_t)stream;
     void *kt = ws + L.kbar_terms;
-    cudaError_t e = ab::launch_meankey(k, kb, kt, BH, s.N, s.N_pad, s.d, cs);
+    cudaError_t e = ab::launch_meankey_units(k, kb, kt, BH, s.N, s.N_pad, s.d, key_unit, cs);
     if (e == cudaSuccess)
         e = ab::launch_kmeans(q, ce, cw, assign, BH, s.N, s.N_pad, s.d, n_clusters, iters,
                               dev_flag, cs);
     if (e == cudaSuccess)
-        e = ab::launch_score(ce, cw, kt, scores, BH, nb, nb, s.d, n_clusters, dev_flag, cs);
+        e = ab::launch_score(ce, cw, kt, scores, BH, nqb, nku, nku_valid, s.d, n_clusters,
+                             dev_flag, cs);
     return cuda_status(e);
 }
 
@@ -144,14 +183,31 @@ ab_status ab_attn_fwd(const void *q, const void *k, const void *v, ab_shape s, c
                       float *lse, int *dev_flag, void *stream)
 {
     if (!w) return AB_ERR_NULL;
-    return attn_common(q, k, v, s, idx, cnt, w, out, out_dtype, lse, dev_flag, stream);
+    return attn_common(q, k, v, s, AB_BLOCK, idx, cnt, w, out, out_dtype, lse, dev_flag, stream);
+}
+
+ab_status ab_attn_units_fwd(const void *q, const void *k, const void *v, ab_shape s, int key_unit,
+                            const int32_t *idx, const int32_t *cnt, const float *w, void *out,
+                            ab_dtype out_dtype, float *lse, int *dev_flag, void *stream)
+{
+    if (!w) return AB_ERR_NULL;
+    return attn_common(q, k, v, s, key_unit, idx, cnt, w, out, out_dtype, lse, dev_flag, stream);
+}
+
+ab_status ab_attn_units_topk_fwd(const void *q, const void *k, const void *v, ab_shape s,
+                                 int key_unit, const int32_t *idx, const int32_t *cnt, void *out,
+                                 ab_dtype out_dtype, float *lse, int *dev_flag, void *stream)
+{
+    return attn_common(q, k, v, s, key_unit, idx, cnt, nullptr, out, out_dtype, lse, dev_flag,
+                       stream);
 }
 
 ab_status ab_attn_topk_fwd(const void *q, const void *k, const void *v, ab_shape s,
                            const int32_t *idx, const int32_t *cnt, void *out, ab_dtype out_dtype,
                            float *lse, int *dev_flag, void *stream)
 {
-    return attn_common(q, k, v, s, idx, cnt, nullptr, out, out_dtype, lse, dev_flag, stream);
+    return attn_common(q, k, v, s, AB_BLOCK, idx, cnt, nullptr, out, out_dtype, lse, dev_flag,
+                       stream);
 }
 
 ab_status ab_check_flag(const int *dev_flag, int *host_flag, void *stream)

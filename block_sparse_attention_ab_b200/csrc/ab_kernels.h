@@ -8,30 +8,34 @@ namespace ab {
 
 // IBCS scoring (score_kernels.cu)
 // Device scratch of the scoring pass, each region 256-byte aligned: mean keys fp32
-// [BH][n_kb][d], centroids fp32 [BH][n_qb][C][d], cluster weights fp32 [BH][n_qb][C],
-// and the three bf16 terms of the mean keys [3][BH][n_kb][d].
+// [BH][n_ku][d], centroids fp32 [BH][n_qb][C][d], cluster weights fp32 [BH][n_qb][C],
+// and the three bf16 terms of the mean keys [3][BH][n_ku][d]; n_ku = key units per head
+// (n_qb for 128-token key blocks).
 struct ScoreLayout {
     size_t kbar, cent, cw, kbar_terms, total;
 };
 
-inline ScoreLayout score_layout(size_t BH, size_t nb, size_t d, size_t C)
+inline ScoreLayout score_layout(size_t BH, size_t nqb, size_t nku, size_t d, size_t C)
 {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     ScoreLayout L;
     L.kbar = 0;
-    L.cent = up(L.kbar + BH * nb * d * sizeof(float));
-    L.cw = up(L.cent + BH * nb * C * d * sizeof(float));
-    L.kbar_terms = up(L.cw + BH * nb * C * sizeof(float));
-    L.total = up(L.kbar_terms + 3 * BH * nb * d * 2);
+    L.cent = up(L.kbar + BH * nku * d * sizeof(float));
+    L.cw = up(L.cent + BH * nqb * C * d * sizeof(float));
+    L.kbar_terms = up(L.cw + BH * nqb * C * sizeof(float));
+    L.total = up(L.kbar_terms + 3 * BH * nku * d * 2);
     return L;
 }
 
 cudaError_t launch_meankey(const void *k, float *kbar, void *kbar_terms, int BH, int N, int N_pad,
                            int d, cudaStream_t st);
+cudaError_t launch_meankey_units(const void *k, float *kbar, void *kbar_terms, int BH, int N,
+                                 int N_pad, int d, int unit, cudaStream_t st);
 cudaError_t launch_kmeans(const void *q, float *cent, float *cw, uint8_t *assign, int BH, int N,
                           int N_pad, int d, int C, int T, int *flag, cudaStream_t st);
 cudaError_t launch_score(const float *cent, const float *cw, const void *kbar_terms, float *scores,
-                         int BH, int nqb, int nkb, int d, int C, int *flag, cudaStream_t st);
+                         int BH, int nqb, int nkb, int nkb_valid, int d, int C, int *flag,
+                         cudaStream_t st);
 
 // SIP / top-k selection (select_kernels.cu)
 cudaError_t launch_sip(const float *scores, int B, int H, int nqb, int nkb, int K, uint64_t seed,
@@ -50,6 +54,7 @@ struct AttnLaunch {
     float *lse;
     int *flag;
     int B, H, N, N_pad, d;
+    int unit;           // key unit of idx entries: 128 (key blocks) or 4 (gathered 4-token units)
     int grid_override;  // > 0: number of CTAs (tests); 0: one per SM
 };
 cudaError_t launch_attn(const AttnLaunch &a, cudaStream_t st);

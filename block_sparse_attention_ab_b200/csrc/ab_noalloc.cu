@@ -55,7 +55,8 @@ extern "C" ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, 
     if (!aligned16(q) || !aligned16(k) || !aligned16(scores)) return AB_ERR_ALIGN;
 
     const ab::ScoreLayout L = ab::score_layout((size_t)s.B * s.H, (size_t)s.N_pad / AB_BLOCK,
-                                               (size_t)s.d, (size_t)n_clusters);
+                                               (size_t)s.N_pad / AB_BLOCK, (size_t)s.d,
+                                               (size_t)n_clusters);
     if (L.total > kScratchBytes) return AB_ERR_WORKSPACE;
 
     void *base = nullptr;
@@ -75,6 +76,6 @@ extern "C" ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, 
         e = ab::launch_kmeans(q, ce, cw, nullptr, BH, s.N, s.N_pad, s.d, n_clusters, iters,
                               dev_flag, cs);
     if (e == cudaSuccess)
-        e = ab::launch_score(ce, cw, kt, scores, BH, nb, nb, s.d, n_clusters, dev_flag, cs);
+        e = ab::launch_score(ce, cw, kt, scores, BH, nb, nb, nb, s.d, n_clusters, dev_flag, cs);
     return e == cudaSuccess ? AB_OK : AB_ERR_CUDA;
 }

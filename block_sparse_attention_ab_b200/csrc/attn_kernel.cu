@@ -49,10 +49,28 @@ struct AttnParams {
     void *out;       // bf16 or fp32 [B*H, N_pad, D]
     float *lse;
     int *flag;
-    int H, N, N_pad, nqb, nkb;
+    const __nv_bfloat16 *kg, *vg;  // K, V in global memory (4-token units: gathered per unit)
+    int H, N, N_pad, nqb;
+    int nkb;       // entries per idx / w row: key blocks (N_pad / 128) or key units (N_pad / 4)
+    int per_tile;  // selected entries per 128-key tile: 1 (blocks) or 32 (units)
     int n_items;
     float scale_log2;  // log2(e) / sqrt(d)
 };
+
+// 4-token key units: one 16-byte cp.async per lane (zero fill when src_bytes == 0) and
+// an arrive on an mbarrier when this thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
 
 template <int D>
 struct AttnSmem {
@@ -74,8 +92,8 @@ struct AttnSmem {
 // The per-CTA stream of (item, block) pairs shared by the three roles.
 struct Cursor {
     int r;    // work item (flat (b*H + h)*nqb + qb); >= n_items when done
-    int i;    // block position within the item
-    int n;    // selected-block count of the item (clamped to [0, nkb])
+    int i;    // tile position within the item
+    int n;    // tiles of the item: selected entries (clamped to [0, nkb]) / per_tile, rounded up
     int seq;  // index of the item among this CTA's non-empty items
 };
 
@@ -85,13 +103,18 @@ __device__ __forceinline__ int load_cnt(const AttnParams &p, int r)
     return c < 0 ? 0 : (c > p.nkb ? p.nkb : c);
 }
 
+__device__ __forceinline__ int load_tiles(const AttnParams &p, int r)
+{
+    return (load_cnt(p, r) + p.per_tile - 1) / p.per_tile;
+}
+
 __device__ __forceinline__ void cursor_seek(Cursor &c, const AttnParams &p)
 {
     while (c.r < p.n_items && c.i >= c.n) {
         if (c.n > 0) ++c.seq;
         c.r += gridDim.x;
         c.i = 0;
-        c.n = c.r < p.n_items ? load_cnt(p, c.r) : 0;
+        c.n = c.r < p.n_items ? load_tiles(p, c.r) : 0;
     }
 }
 
@@ -101,7 +124,7 @@ __device__ __forceinline__ Cursor cursor_first(const AttnParams &p)
     c.r = blockIdx.x;
     c.i = 0;
     c.seq = 0;
-    c.n = c.r < p.n_items ? load_cnt(p, c.r) : 0;
+    c.n = c.r < p.n_items ? load_tiles(p, c.r) : 0;
     cursor_seek(c, p);
     return c;
 }
@@ -122,7 +145,7 @@ __device__ __forceinline__ int block_index(const AttnParams &p, int r, int i, bo
     return j;
 }
 
-template <int D, bool kWeighted, bool kOutF32>
+template <int D, bool kWeighted, bool kOutF32, bool kUnits>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p)
@@ -155,7 +178,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&o_full[b], 1);
         }
         for (int s = 0; s < L::kStages; ++s) {
-            mbar_init(&kv_full[s], 1);
+            // TMA: one arrive with the tile's byte count; units: one cp.async arrive per lane
+            mbar_init(&kv_full[s], kUnits ? 32 : 1);
             mbar_init(&kv_empty[s], 1);
         }
         mbar_init(drain, 1);
@@ -205,6 +229,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         auto load_kv = [&](const Cursor &c, const CUtensorMap *tm) -> bool {
             const int s = kv_pos % L::kStages;
             if (!wait(&kv_empty[s], ((kv_pos / L::kStages) & 1) ^ 1)) return false;
+            if constexpr (kUnits) {
+                // gather 32 units of 4 key rows into tile rows 4 s' .. 4 s' + 3, in the
+                // 128-byte-swizzled layout the MMA descriptors read; one warp
+                // instruction copies one unit's 4 rows x 64 columns (lane = row, chunk)
+                const int cnt = load_cnt(p, c.r);
+                const int slot = c.i * 32 + lane;
+                int u = -1;
+                if (slot < cnt) {
+                    u = __ldg(p.idx + (size_t)c.r * p.nkb + slot);
+                    if (u < 0 || u >= p.nkb) {
+                        if (tm == &tmK) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
+                        u = -1;
+                    }
+                }
+                const __nv_bfloat16 *src = (tm == &tmK ? p.kg : p.vg) + (size_t)(c.r / p.nqb) * p.N_pad * D;
+                const uint32_t dst = smem_u32(smem + L::kKVOff + s * L::kTileBytes);
+                const int rr = lane >> 3, c8 = lane & 7;
+#pragma unroll 4
+                for (int su = 0; su < 32; ++su) {
+                    const int us = __shfl_sync(0xffffffffu, u, su);
+                    const int tok = us * 4 + rr;
+                    const bool valid = us >= 0 && tok < p.N;
+                    const int row = su * 4 + rr;
+                    const __nv_bfloat16 *g = src + (size_t)(valid ? tok : 0) * D + c8 * 8;
+#pragma unroll
+                    for (int h = 0; h < L::kBoxes; ++h)
+                        cp_async_16(dst + h * 16384 + row * 128 + ((c8 ^ (row & 7)) << 4), g + h * 64,
+                                    valid ? 16u : 0u);
+                }
+                cp_async_arrive_noinc(&kv_full[s]);
+                ++kv_pos;
+                return true;
+            }
             const int j = block_index(p, c.r, c.i, tm == &tmK && lane == 0);
             uint8_t *dst = smem + L::kKVOff + s * L::kTileBytes;
             const int bh = c.r / p.nqb;
@@ -264,6 +321,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (c.i == 0 && !wait(&q_full[qbuf], (c.seq >> 1) & 1)) return false;
             const int s = kv_pos % L::kStages;
             if (!wait(&kv_full[s], (kv_pos / L::kStages) & 1)) return false;
+            if constexpr (kUnits) fence_proxy_async_smem();  // tile written by cp.async
             tc_fence_after();
             const uint64_t qd = q_desc0 + (uint64_t)qbuf * kTileDesc;
             const uint64_t kd = k_desc0 + (uint64_t)s * kTileDesc;
@@ -299,6 +357,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 ok = false;
                 break;
             }
+            if constexpr (kUnits) fence_proxy_async_smem();  // tile written by cp.async
             tc_fence_after();
             const uint64_t vd = v_desc0 + (uint64_t)s * kTileDesc;
             const uint32_t p_tmem = tmem + (g % kSBufs) * 128;
@@ -373,7 +432,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         constexpr int kSoftPairs = 6;  // of 32 pairs per block: exp2 on the FMA pipe
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         for (int r = blockIdx.x; r < p.n_items; r += gridDim.x) {
-            const int n = load_cnt(p, r);
+            const int cnt_r = load_cnt(p, r);
+            const int n = kUnits ? (cnt_r + 31) / 32 : cnt_r;  // 128-key tiles of this item
             const int bh = r / p.nqb, qb = r % p.nqb;
             const int tok = qb * 128 + row;
             const size_t orow_off = ((size_t)bh * p.N_pad + tok) * D + half * kHalfD;
@@ -393,26 +453,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             const int32_t *idx_row = p.idx + (size_t)r * p.nkb;
             const float *w_row = kWeighted ? p.w + (size_t)r * p.nkb : nullptr;
-            // block index and weight are loaded two blocks ahead; the next block's log2
+            // blocks: index and weight are loaded two blocks ahead; the next block's log2
             // weight is taken right after this block's max exchange, while the MUFU unit
-            // is free of exp2 work
-            int j = clamp_j(__ldg(idx_row));
-            float lw = lw_of(kWeighted ? __ldg(w_row) : 1.f);
+            // is free of exp2 work.
+            // units: lane l < 16 of each warp holds unit slot 32 i + 16 half + l of tile i
+            // (this warp's 64 columns = 16 units); its log2 weight (-inf for an empty
+            // slot) and valid-token count reach the other lanes by shuffles.
+            int j = 0;
+            float lw = 0.f;
             int j_n1 = 0;
             float w_n1 = 1.f;
-            if (n > 1) {
-                j_n1 = __ldg(idx_row + 1);
-                if (kWeighted) w_n1 = __ldg(w_row + 1);
+            auto unit_of = [&](int t, int &u, float &wv) {
+                const int slot = t * 32 + half * 16 + (lane & 15);
+                u = -1;
+                wv = 1.f;
+                if (lane < 16 && slot < cnt_r) {
+                    const int x = __ldg(idx_row + slot);
+                    if (x >= 0 && x < p.nkb) {
+                        u = x;
+                        if (kWeighted) wv = __ldg(w_row + slot);
+                    }
+                }
+            };
+            auto unit_lw = [&](int u, float wv, int &nv) -> float {
+                nv = u >= 0 ? max(0, min(4, p.N - 4 * u)) : 0;
+                if (nv == 0) return -INFINITY;
+                if (!kWeighted) return 0.f;
+                if (wv > 0.f && wv < INFINITY) return fast_log2(wv);
+                raise_flag(p.flag, AB_FLAG_BAD_WEIGHT);
+                return 0.f;
+            };
+            int nv_l = 0, nv_n = 0;  // units: valid tokens of this lane's slot (tile i, i + 1)
+            if constexpr (kUnits) {
+                int u;
+                float wv;
+                unit_of(0, u, wv);
+                lw = unit_lw(u, wv, nv_l);
+                if (n > 1) unit_of(1, j_n1, w_n1);
+            } else {
+                j = clamp_j(__ldg(idx_row));
+                lw = lw_of(kWeighted ? __ldg(w_row) : 1.f);
+                if (n > 1) {
+                    j_n1 = __ldg(idx_row + 1);
+                    if (kWeighted) w_n1 = __ldg(w_row + 1);
+                }
             }
             float m_run = -INFINITY, l_run = 0.f;
             for (int i = 0; i < n; ++i, ++g) {
                 int j_n2 = 0;
                 float w_n2 = 1.f;
                 if (i + 2 < n) {
-                    j_n2 = __ldg(idx_row + i + 2);
-                    if (kWeighted) w_n2 = __ldg(w_row + i + 2);
+                    if constexpr (kUnits) {
+                        unit_of(i + 2, j_n2, w_n2);
+                    } else {
+                        j_n2 = __ldg(idx_row + i + 2);
+                        if (kWeighted) w_n2 = __ldg(w_row + i + 2);
+                    }
                 }
-                const int nvalid = min(128, p.N - j * 128) - half * 64;  // valid columns here
+                const int nvalid = min(128, p.N - j * 128) - half * 64;  // blocks: valid columns here
                 const uint32_t s_col = (g % kSBufs) * 128;
                 wait_bar(&s_full[g % kSBufs], (g / kSBufs) & 1);
                 tc_fence_after();
@@ -426,7 +524,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 float sv[64];
 #pragma unroll
                 for (int e = 0; e < 64; ++e) sv[e] = __uint_as_float(su[e]);
-                if (nvalid < 64) {
+                if constexpr (kUnits) {
+                    // x = s * scale_log2 + log2 w of the column's unit (-inf: empty slot
+                    // or a token past the sequence end)
+                    float lwu[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) lwu[k] = __shfl_sync(0xffffffffu, lw, k);
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) sv[e] = fmaf(sv[e], p.scale_log2, lwu[e >> 2]);
+                    if (__any_sync(0xffffffffu, nv_l > 0 && nv_l < 4)) {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const int nvk = __shfl_sync(0xffffffffu, nv_l, k);
+#pragma unroll
+                            for (int t = 0; t < 4; ++t)
+                                if (t >= nvk) sv[4 * k + t] = -INFINITY;
+                        }
+                    }
+                } else if (nvalid < 64) {
 #pragma unroll
                     for (int e = 0; e < 64; ++e)
                         if (e >= nvalid) sv[e] = -INFINITY;
@@ -446,8 +561,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 xmax_sh[((g & 1) * 2 + half) * 128 + row] = mx[0];
                 pair_sync();
                 const float smax = fmaxf(mx[0], xmax_sh[((g & 1) * 2 + (half ^ 1)) * 128 + row]);
-                const float lw_n1 = (kWeighted && i + 1 < n) ? lw_of(w_n1) : 0.f;
-                const float xmax = smax * p.scale_log2 + lw;
+                float lw_n1 = 0.f;
+                if constexpr (kUnits) {
+                    if (i + 1 < n) lw_n1 = unit_lw(j_n1, w_n1, nv_n);
+                } else if (kWeighted && i + 1 < n) {
+                    lw_n1 = lw_of(w_n1);
+                }
+                // units: the maxima were taken over scaled, weight-shifted logits
+                const float xmax = kUnits ? smax : smax * p.scale_log2 + lw;
                 const float m_new = fmaxf(m_run, xmax);
                 bool rescale = false;
                 if (i == 0) {
@@ -478,13 +599,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 // P = 2^(s * scale_log2 + lw - m_run) in fp32 pairs, packed to bf16 over
                 // the S columns; the first kSoftPairs pairs use the FMA-pipe exp2
-                const float bias = lw - m_run;
+                // units: a row may have seen no valid key yet (every kept unit past the
+                // sequence end); its P is then 0, not NaN
+                const float m_ref = (kUnits && m_run == -INFINITY) ? 0.f : m_run;
+                const float bias = kUnits ? -m_ref : lw - m_ref;
                 const uint64_t bias2 = f2_pack(bias, bias);
                 uint64_t ls2[4] = {0, 0, 0, 0};
                 uint32_t pk[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const uint64_t x2 = f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), scale2, bias2);
+                    const uint64_t x2 = kUnits ? f2_add(f2_pack(sv[2 * e], sv[2 * e + 1]), bias2)
+                                               : f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), scale2, bias2);
                     float2 pr;
                     if (e < kSoftPairs) {
                         pr = soft_exp2_pair(x2);
@@ -505,8 +630,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&p_full[g % kSBufs]);
                 if (i + 1 < n) {
-                    j = clamp_j(j_n1);
+                    j = kUnits ? 0 : clamp_j(j_n1);
                     lw = lw_n1;
+                    nv_l = nv_n;
                     j_n1 = j_n2;
                     w_n1 = w_n2;
                 }
@@ -517,7 +643,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     xl_sh[half * 128 + row] = l_run;
                     pair_sync();
                     const float l_tot = l_run + xl_sh[(half ^ 1) * 128 + row];
-                    const float inv = tok < p.N ? 1.0f / l_tot : 0.f;
+                    const float inv = (tok < p.N && l_tot > 0.f) ? 1.0f / l_tot : 0.f;
 #pragma unroll 1
                     for (int ch = 0; ch < kHalfD / 32; ++ch) {
                         uint32_t r32[32];
@@ -551,7 +677,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                     if (p.lse && half == 0)
                         p.lse[(size_t)bh * p.N_pad + tok] =
-                            tok < p.N ? (m_run + log2f(l_tot)) * 0.69314718055994531f : 0.f;
+                            tok < p.N ? (l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f
+                                                     : -INFINITY)
+                                      : 0.f;
                 }
             }
         }
@@ -577,7 +705,7 @@ static bool make_tmap(CUtensorMap *tm, const void *base, int BH, int N, int N_pa
                              (uint64_t)N_pad * d * 2, 64, 128);
 }
 
-template <int D, bool W, bool F32>
+template <int D, bool W, bool F32, bool U4>
 static cudaError_t launch_attn_t(const AttnLaunch &a, cudaStream_t st)
 {
     CUtensorMap tq, tk, tv;
@@ -592,29 +720,38 @@ static cudaError_t launch_attn_t(const AttnLaunch &a, cudaStream_t st)
     p.out = a.out;
     p.lse = a.lse;
     p.flag = a.flag;
+    p.kg = static_cast<const __nv_bfloat16 *>(a.k);
+    p.vg = static_cast<const __nv_bfloat16 *>(a.v);
     p.H = a.H;
     p.N = a.N;
     p.N_pad = a.N_pad;
     p.nqb = a.N_pad / 128;
-    p.nkb = a.N_pad / 128;
+    p.nkb = a.N_pad / (U4 ? 4 : 128);
+    p.per_tile = U4 ? 32 : 1;
     p.n_items = a.B * a.H * p.nqb;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     const int smem = AttnSmem<D>::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, W, F32>,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, W, F32, U4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = a.grid_override > 0 ? a.grid_override : (p.n_items < sms ? p.n_items : sms);
-    attn_fwd_kernel<D, W, F32><<<grid, kAttnThreads, smem, st>>>(tq, tk, tv, p);
+    attn_fwd_kernel<D, W, F32, U4><<<grid, kAttnThreads, smem, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
+}
+
+template <int D, bool W, bool F32>
+static cudaError_t launch_attn_u(const AttnLaunch &a, cudaStream_t st)
+{
+    return a.unit == 4 ? launch_attn_t<D, W, F32, true>(a, st) : launch_attn_t<D, W, F32, false>(a, st);
 }
 
 template <int D, bool W>
 static cudaError_t launch_attn_o(const AttnLaunch &a, cudaStream_t st)
 {
-    return a.out_f32 ? launch_attn_t<D, W, true>(a, st) : launch_attn_t<D, W, false>(a, st);
+    return a.out_f32 ? launch_attn_u<D, W, true>(a, st) : launch_attn_u<D, W, false>(a, st);
 }
 
 cudaError_t launch_attn(const AttnLaunch &a, cudaStream_t st)

@@ -146,6 +146,57 @@ __global__ void __launch_bounds__(256) meankey_kernel(const __nv_bfloat16 *__res
 }
 
 // ---------------------------------------------------------------------------------
+// Mean key of 4-token key units (the page's fine-grained selection unit): one CTA of
+// 256 threads per (b, h, 128-token span) = 32 units; thread (unit pair, 16-byte column
+// chunk) sums the unit's valid rows (fixed order) and writes the fp32 mean and its
+// three bf16 terms. A unit with no valid token gets 0.
+// ---------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) meankey4_kernel(const __nv_bfloat16 *__restrict__ k,
+                                                       float *__restrict__ kbar,
+                                                       __nv_bfloat16 *__restrict__ kbs, int N,
+                                                       int N_pad, int nspan)
+{
+    constexpr int CH = D / 8;                // 16-byte chunks per row
+    constexpr int PER = 32 * CH / 256;       // (unit, chunk) pairs per thread
+    const int span = blockIdx.x;
+    const int bh = span / nspan, sp = span % nspan;
+    const int nku = N_pad / 4;
+    const size_t term = (size_t)gridDim.x * 32 * D;  // one term of all units
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+        const int e = threadIdx.x + it * 256;
+        const int ul = e / CH, ch = e % CH;        // unit within the span, chunk
+        const int u = sp * 32 + ul;                // unit within the head
+        const int t0 = u * 4;
+        const int nv = max(0, min(4, N - t0));
+        float acc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+        const uint4 *base = reinterpret_cast<const uint4 *>(k + ((size_t)bh * N_pad + t0) * D) + ch;
+        for (int r = 0; r < nv; ++r) {
+            const uint4 v = __ldg(base + (size_t)r * CH);
+            acc[0] += bf16_lo(v.x); acc[1] += bf16_hi(v.x);
+            acc[2] += bf16_lo(v.y); acc[3] += bf16_hi(v.y);
+            acc[4] += bf16_lo(v.z); acc[5] += bf16_hi(v.z);
+            acc[6] += bf16_lo(v.w); acc[7] += bf16_hi(v.w);
+        }
+        const float inv = nv > 0 ? 1.0f / (float)nv : 0.f;
+        float m[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) m[c] = acc[c] * inv;
+        const size_t o = ((size_t)bh * nku + u) * D + ch * 8;
+        float4 *dst = reinterpret_cast<float4 *>(kbar + o);
+        dst[0] = make_float4(m[0], m[1], m[2], m[3]);
+        dst[1] = make_float4(m[4], m[5], m[6], m[7]);
+        uint4 t[3];
+        split3x8(m, t);
+#pragma unroll
+        for (int s3 = 0; s3 < 3; ++s3) *reinterpret_cast<uint4 *>(kbs + s3 * term + o) = t[s3];
+    }
+}
+
+// ---------------------------------------------------------------------------------
 // Per-block k-means on the 5th-generation tensor cores. One CTA of 128 threads per
 // (b, h, query block). The block's queries arrive by TMA (128-byte swizzle; rows past
 // N read as zero) and stay in shared memory for all T iterations. Each iteration runs
@@ -491,8 +542,8 @@ __host__ __device__ constexpr int prod_term_b(int pr) { return pr == 1 || pr == 
 template <int D>
 __global__ void __launch_bounds__(kScThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tmKB, const float *__restrict__ cent,
-                 const float *__restrict__ cw, int BH, int nqb, int nkb, int C, float scale_log2,
-                 float *__restrict__ scores, int *flag)
+                 const float *__restrict__ cw, int BH, int nqb, int nkb, int nkb_valid, int C,
+                 float scale_log2, float *__restrict__ scores, int *flag)
 {
     using L = ScSmem<D>;
     extern __shared__ uint8_t sc_raw[];
@@ -671,25 +722,28 @@ __global__ void __launch_bounds__(kScThreads, 1)
             const int c0 = ch * kScChunk;
             const int ncols = min(kScChunk, nkb - c0);
             const int nsl = (ncols + 31) >> 5;
+            // key units past the sequence end (j >= nkb_valid) take no part and score 0
+            const int nvcols = max(0, min(ncols, nkb_valid - c0));
+            const int nvsl = (nvcols + 31) >> 5;
             const uint32_t tb = t_lane + buf * kScChunk;
             if (j < nch) {
                 // row statistics in log2 units: max, then the sum of 2^(x - max)
                 float mx = m;
-                for (int sl = 0; sl < nsl; ++sl) {
+                for (int sl = 0; sl < nvsl; ++sl) {
                     uint32_t v[32];
                     tmem_ld32(tb + sl * 32, v);
                     tmem_wait_ld();
-                    const int lim = ncols - sl * 32;
+                    const int lim = nvcols - sl * 32;
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (i < lim) mx = fmaxf(mx, __uint_as_float(v[i]) * scale_log2);
                 }
                 float zz = m == -INFINITY ? 0.f : z * fast_exp2(m - mx);
-                for (int sl = 0; sl < nsl; ++sl) {
+                for (int sl = 0; sl < nvsl; ++sl) {
                     uint32_t v[32];
                     tmem_ld32(tb + sl * 32, v);
                     tmem_wait_ld();
-                    const int lim = ncols - sl * 32;
+                    const int lim = nvcols - sl * 32;
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (i < lim) zz += fast_exp2(fmaf(__uint_as_float(v[i]), scale_log2, -mx));
@@ -708,7 +762,9 @@ __global__ void __launch_bounds__(kScThreads, 1)
                         float e[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            e[i] = coef * fast_exp2(fmaf(__uint_as_float(v[q8 * 8 + i]), scale_log2, -m));
+                            e[i] = c0 + sl * 32 + q8 * 8 + i < nkb_valid
+                                       ? coef * fast_exp2(fmaf(__uint_as_float(v[q8 * 8 + i]), scale_log2, -m))
+                                       : 0.f;
                         // sum over the 8 rows (lanes) of this query block; lane r8 ends
                         // with column q8 * 8 + r8
                         float u[4];
@@ -749,6 +805,20 @@ __global__ void __launch_bounds__(kScThreads, 1)
 // ---------------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------------
+cudaError_t launch_meankey_units(const void *k, float *kbar, void *kbar_terms, int BH, int N,
+                                 int N_pad, int d, int unit, cudaStream_t st)
+{
+    if (unit != 4) return launch_meankey(k, kbar, kbar_terms, BH, N, N_pad, d, st);
+    const int nspan = N_pad / 128;
+    const dim3 grid((unsigned)(BH * nspan));
+    __nv_bfloat16 *kbs = static_cast<__nv_bfloat16 *>(kbar_terms);
+    if (d == 128)
+        meankey4_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, N, N_pad, nspan);
+    else
+        meankey4_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, N, N_pad, nspan);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_meankey(const void *k, float *kbar, void *kbar_terms, int BH, int N, int N_pad,
                            int d, cudaStream_t st)
 {
@@ -789,8 +859,8 @@ cudaError_t launch_kmeans(const void *q, float *cent, float *cw, uint8_t *assign
 
 template <int D>
 static cudaError_t launch_score_t(const float *cent, const float *cw, const void *kbar_terms,
-                                  float *scores, int BH, int nqb, int nkb, int C, int *flag,
-                                  cudaStream_t st)
+                                  float *scores, int BH, int nqb, int nkb, int nkb_valid, int C,
+                                  int *flag, cudaStream_t st)
 {
     CUtensorMap tm;
     if (!make_tmap_bf16_3d(&tm, kbar_terms, D, (uint64_t)nkb, (uint64_t)3 * BH, (uint64_t)D * 2,
@@ -802,16 +872,19 @@ static cudaError_t launch_score_t(const float *cent, const float *cw, const void
     if (e != cudaSuccess) return e;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     const dim3 grid((unsigned)((nqb + 15) / 16), (unsigned)BH);
-    score_kernel<D><<<grid, kScThreads, smem, st>>>(tm, cent, cw, BH, nqb, nkb, C, scale_log2,
-                                                    scores, flag);
+    score_kernel<D><<<grid, kScThreads, smem, st>>>(tm, cent, cw, BH, nqb, nkb, nkb_valid, C,
+                                                    scale_log2, scores, flag);
     return cudaGetLastError();
 }
 
 cudaError_t launch_score(const float *cent, const float *cw, const void *kbar_terms, float *scores,
-                         int BH, int nqb, int nkb, int d, int C, int *flag, cudaStream_t st)
+                         int BH, int nqb, int nkb, int nkb_valid, int d, int C, int *flag,
+                         cudaStream_t st)
 {
-    return d == 128 ? launch_score_t<128>(cent, cw, kbar_terms, scores, BH, nqb, nkb, C, flag, st)
-                    : launch_score_t<64>(cent, cw, kbar_terms, scores, BH, nqb, nkb, C, flag, st);
+    return d == 128 ? launch_score_t<128>(cent, cw, kbar_terms, scores, BH, nqb, nkb, nkb_valid, C,
+                                          flag, st)
+                    : launch_score_t<64>(cent, cw, kbar_terms, scores, BH, nqb, nkb, nkb_valid, C,
+                                         flag, st);
 }
 
 }  // namespace ab

@@ -71,6 +71,10 @@ typedef struct {
 /* Limits: head dim d in {64, 128}; 1 <= n_kb <= 8192 (N_pad <= 1,048,576). */
 #define AB_BLOCK 128
 #define AB_MAX_BLOCKS 8192
+/* The page's fine-grained key/value selection unit (section «Три приёма AB-Attention»,
+ * third technique): 4 tokens. With it at most AB_MAX_BLOCKS units per head
+ * (N_pad <= 32768). */
+#define AB_UNIT4 4
 
 /*
  * ab_score_workspace_size -- bytes of device scratch ab_score() needs for shape `s`
@@ -138,6 +142,27 @@ ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, int n_clust
                            float *scores, int *dev_flag, void *stream);
 
 /*
+ * ab_score_units, ab_score_units_workspace_size -- IBCS scores at key-unit granularity
+ * (page section «Три приёма AB-Attention», third technique: key/value selection units
+ * of 4 tokens instead of 128, at the same tile budget). Queries stay in 128-token
+ * blocks with their k-means clusters; keys are grouped into units of key_unit tokens
+ * (AB_BLOCK or AB_UNIT4): kbar_u = mean of the valid keys of unit u, and
+ * scores[qb][u] = sum_c w_c softmax_u(cent_c . kbar_u / sqrt(d)) over the units that
+ * hold at least one valid token (u < ceil(N / key_unit)); the other units score 0.
+ * With key_unit = AB_BLOCK this is ab_score.
+ * scores : out, fp32 [B,H,n_qb,n_ku], n_ku = N_pad / key_unit (<= AB_MAX_BLOCKS).
+ * kbar   : optional out, fp32 [B,H,n_ku,d]. Other arguments as ab_score; the workspace
+ *          needs ab_score_units_workspace_size() bytes.
+ * Errors: as ab_score; AB_ERR_UNSUPPORTED for another key_unit, AB_ERR_RANGE when
+ * n_ku > AB_MAX_BLOCKS.
+ */
+ab_status ab_score_units_workspace_size(ab_shape s, int n_clusters, int key_unit, size_t *bytes);
+ab_status ab_score_units(const void *q, const void *k, ab_shape s, int n_clusters, int iters,
+                         int key_unit, float *scores, float *kbar, float *centroids,
+                         float *cweights, uint8_t *assign, void *workspace,
+                         size_t workspace_bytes, int *dev_flag, void *stream);
+
+/*
  * ab_select -- choose key blocks per query block (page section «Три приёма
  * AB-Attention», second technique SIP; section «Где ломаются прежние разреженные
  * схемы» for top-k).
@@ -199,6 +224,28 @@ ab_status ab_attn_fwd(const void *q, const void *k, const void *v, ab_shape s,
 ab_status ab_attn_topk_fwd(const void *q, const void *k, const void *v, ab_shape s,
                            const int32_t *idx, const int32_t *cnt, void *out, ab_dtype out_dtype,
                            float *lse, int *dev_flag, void *stream);
+
+/*
+ * ab_attn_units_fwd, ab_attn_units_topk_fwd -- the attention of ab_attn_fwd /
+ * ab_attn_topk_fwd over selected key units of key_unit tokens (AB_BLOCK, or AB_UNIT4:
+ * the page's 4-token units, third technique). idx / cnt / w come from ab_select run on
+ * ab_score_units' scores (rows of n_ku = N_pad / key_unit entries, kept unit indices
+ * ascending). For AB_UNIT4 the kernel gathers the kept units 32 at a time into
+ * 128-key tiles (unit s of a tile -> tile rows 4s..4s+3), so a query block costs
+ * ceil(cnt / 32) tensor-core tiles; tokens t >= N and empty tile slots take no part.
+ * Unit u counts with weight w (HT: logit + ln w), 1 in the top-k call.
+ *   O_i = sum_{u in sel} w_u sum_{t in u, t<N} e^{q_i.k_t/sqrt(d)} v_t
+ *         / sum_{u in sel} w_u sum_{t in u, t<N} e^{q_i.k_t/sqrt(d)}
+ * With key_unit = AB_BLOCK these are ab_attn_fwd / ab_attn_topk_fwd.
+ * Errors and device flags: as ab_attn_fwd; AB_ERR_UNSUPPORTED for another key_unit,
+ * AB_ERR_RANGE when n_ku > AB_MAX_BLOCKS.
+ */
+ab_status ab_attn_units_fwd(const void *q, const void *k, const void *v, ab_shape s, int key_unit,
+                            const int32_t *idx, const int32_t *cnt, const float *w, void *out,
+                            ab_dtype out_dtype, float *lse, int *dev_flag, void *stream);
+ab_status ab_attn_units_topk_fwd(const void *q, const void *k, const void *v, ab_shape s,
+                                 int key_unit, const int32_t *idx, const int32_t *cnt, void *out,
+                                 ab_dtype out_dtype, float *lse, int *dev_flag, void *stream);
 
 /*
  * ab_check_flag -- synchronise `stream`, copy *dev_flag to *host_flag and map it to a

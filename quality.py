@@ -18,6 +18,9 @@ Methods, each at the same budget K (blocks per query block):
   meanpool_topk  scores from one mean-pooled query per block (C = 1) -> top-k;
   ideal_topk     the K blocks with the largest true attention mass of the query block
                  (the best any top-k selection can do on mass recall).
+With --units, the same at the page's 4-token key units (third technique) for the same
+number of tensor-core tiles (32 units per 128-key tile): unit4_ibcs_sip,
+unit4_ibcs_topk, unit4_ideal_topk.
 
 Everything but the dense reference runs through the library's kernels; the reference
 (per-row block masses and O_dense) is plain fp32 PyTorch on the same device.
@@ -40,14 +43,14 @@ import torch  # noqa: E402
 
 
 def dense_reference(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, N: int,
-                    rows_per_chunk: int = 1024):
+                    rows_per_chunk: int = 1024, unit: int = 128):
     """Exact attention in fp32 for [B, H, N_pad, d] bf16 inputs on one device.
 
-    Returns (O_dense fp32 [B, H, N_pad, d], mass fp32 [B, H, N_pad, n_kb]) where
-    mass[..., i, j] is the softmax probability mass of query row i on key block j
-    (keys t >= N excluded). Rows i >= N are zero in both."""
+    Returns (O_dense fp32 [B, H, N_pad, d], mass fp32 [B, H, N_pad, N_pad / unit]) where
+    mass[..., i, j] is the softmax probability mass of query row i on key unit j of
+    `unit` tokens (keys t >= N excluded). Rows i >= N are zero in both."""
     B, H, N_pad, d = q.shape
-    nkb = N_pad // 128
+    nkb = N_pad // unit
     o = torch.zeros(B, H, N_pad, d, device=q.device, dtype=torch.float32)
     mass = torch.zeros(B, H, N_pad, nkb, device=q.device, dtype=torch.float32)
     scale = 1.0 / d ** 0.5
@@ -62,13 +65,14 @@ def dense_reference(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, N: int,
                 logits.masked_fill_(~key_ok, float("-inf"))
                 p = torch.softmax(logits, dim=-1)
                 o[b, h, r0:r1] = p @ vf
-                mass[b, h, r0:r1] = p.view(r1 - r0, nkb, 128).sum(-1)
+                mass[b, h, r0:r1] = p.view(r1 - r0, nkb, unit).sum(-1)
     return o, mass
 
 
 def mass_recall(mass: torch.Tensor, idx: torch.Tensor, cnt: torch.Tensor, N: int) -> float:
-    """Mean over valid query rows of the true softmax mass on the selected key blocks.
-    mass: [B, H, N_pad, n_kb]; idx: [B, H, n_qb, >= max cnt] (first cnt entries valid)."""
+    """Mean over valid query rows of the true softmax mass on the selected key units
+    (blocks of 128 or units of 4 tokens; query rows are grouped in blocks of 128).
+    mass: [B, H, N_pad, n_ku]; idx: [B, H, n_qb, >= max cnt] (first cnt entries valid)."""
     B, H, N_pad, nkb = mass.shape
     nqb = N_pad // 128
     sel = torch.zeros(B, H, nqb, nkb, device=mass.device, dtype=torch.float32)
@@ -92,7 +96,7 @@ def ideal_scores(mass: torch.Tensor) -> torch.Tensor:
     return mass.view(B, H, N_pad // 128, 128, nkb).mean(3).contiguous()
 
 
-def evaluate(w, heads: int, budgets, seeds: int, device="cuda"):
+def evaluate(w, heads: int, budgets, seeds: int, device="cuda", units: bool = False):
     import block_sparse_attention_ab_b200 as ab
     from block_sparse_attention_ab_b200 import synth
 
@@ -104,6 +108,11 @@ def evaluate(w, heads: int, budgets, seeds: int, device="cuda"):
     s_pool = ab.score(qc, kc, w.N, 1, 1)
     s_ideal = ideal_scores(mass)
     nkb = w.N_pad // 128
+    if units:
+        # the page's 4-token units at the same tile budget (32 units per 128-key tile)
+        mass4 = dense_reference(qc, kc, vc, w.N, unit=4)[1]
+        s_ibcs4 = ab.score(qc, kc, w.N, w.n_clusters, w.iters, unit=4)
+        s_ideal4 = ideal_scores(mass4)
     rows = []
     for frac in budgets:
         K = max(1, int(frac * nkb + 0.5))
@@ -123,6 +132,21 @@ def evaluate(w, heads: int, budgets, seeds: int, device="cuda"):
         res["ibcs_sip"] = {"mass_recall": round(float(np.mean(rec)), 5),
                            "attn_error": round(float(np.mean(err)), 5),
                            "mean_kept_blocks": round(float(np.mean(kept)), 2), "seeds": seeds}
+        if units:
+            K4 = 32 * K
+            for name, s4 in (("unit4_ibcs_topk", s_ibcs4), ("unit4_ideal_topk", s_ideal4)):
+                idx, cnt, _ = ab.select(s4, K4, "topk")
+                o = ab.attn_topk_fwd(qc, kc, vc, w.N, idx, cnt, out_dtype=torch.float32, unit=4)
+                res[name] = {"mass_recall": round(mass_recall(mass4, idx, cnt, w.N), 5),
+                             "attn_error": round(rel_error(o, o_ref, w.N), 5)}
+            rec, err = [], []
+            for sd in range(seeds):
+                idx, cnt, wt = ab.select(s_ibcs4, K4, "sip", w.sip_seed + sd)
+                o = ab.attn_fwd(qc, kc, vc, w.N, idx, cnt, wt, out_dtype=torch.float32, unit=4)
+                rec.append(mass_recall(mass4, idx, cnt, w.N))
+                err.append(rel_error(o, o_ref, w.N))
+            res["unit4_ibcs_sip"] = {"mass_recall": round(float(np.mean(rec)), 5),
+                                     "attn_error": round(float(np.mean(err)), 5), "seeds": seeds}
         rows.append(res)
     return rows
 
@@ -135,10 +159,12 @@ def main():
     ap.add_argument("--heads", type=int, default=2, help="first H heads only (0 = all)")
     ap.add_argument("--budgets", default="0.05,0.1,0.2,0.3")
     ap.add_argument("--seeds", type=int, default=4)
+    ap.add_argument("--units", action="store_true",
+                    help="also the page's 4-token key units at the same tile budget")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.config]
     budgets = [float(x) for x in args.budgets.split(",")]
-    rows = evaluate(w, args.heads, budgets, args.seeds)
+    rows = evaluate(w, args.heads, budgets, args.seeds, units=args.units)
     for r in rows:
         print(json.dumps({"workload": w.name, "heads": args.heads or w.H, **r}))
 

@@ -136,3 +136,36 @@ def test_product_package_does_not_reference_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle\b", text, re.M), f
                 assert "liboracle" not in text and "ab_oracle" not in text, f
+
+
+def test_unit_entry_points_reject_bad_units(L):
+    s = shape()
+    n = ctypes.c_size_t(0)
+    # key units: 128-token blocks or the page's 4-token units only
+    assert L.ab_score_units_workspace_size(s, 8, 8, ctypes.byref(n)) == 4
+    assert L.ab_attn_units_fwd(FAKE, FAKE, FAKE, s, 16, FAKE, FAKE, FAKE, FAKE, ab.AB_BF16, None,
+                               None, None) == 4
+    assert L.ab_attn_units_topk_fwd(FAKE, FAKE, FAKE, s, 2, FAKE, FAKE, FAKE, ab.AB_BF16, None,
+                                    None, None) == 4
+    # at most AB_MAX_BLOCKS units per head: 4-token units need N_pad <= 32768
+    big = shape(N=32896, N_pad=32896)
+    assert L.ab_score_units_workspace_size(big, 8, 4, ctypes.byref(n)) == 5
+    assert L.ab_attn_units_topk_fwd(FAKE, FAKE, FAKE, big, 4, FAKE, FAKE, FAKE, ab.AB_BF16, None,
+                                    None, None) == 5
+    assert L.ab_score_units(FAKE, FAKE, big, 8, 5, 4, FAKE, None, None, None, None, FAKE, 1 << 40,
+                            None, None) == 5
+    assert L.ab_attn_units_fwd(FAKE, FAKE, FAKE, s, 4, FAKE, FAKE, None, FAKE, ab.AB_BF16, None,
+                               None, None) == 1
+
+
+def test_unit_workspace_size(L):
+    n = ctypes.c_size_t(0)
+    assert L.ab_score_units_workspace_size(shape(), 8, 4, ctypes.byref(n)) == 0
+    nqb, nku = 8, 256
+    # mean keys [2, nku, 64] fp32, centroids and weights per query block, bf16 key terms
+    need = 2 * nku * 64 * 4 + 2 * nqb * 8 * 64 * 4 + 2 * nqb * 8 * 4 + 3 * 2 * nku * 64 * 2
+    assert need <= n.value <= need + 4 * 256
+    m = ctypes.c_size_t(0)
+    assert L.ab_score_units_workspace_size(shape(), 8, 128, ctypes.byref(m)) == 0
+    L.ab_score_workspace_size(shape(), 8, ctypes.byref(n))
+    assert m.value == n.value
