@@ -37,6 +37,10 @@ namespace ab {
 
 constexpr int kAttnThreads = 320;  // 8 softmax warps, 1 TMA warp, 1 MMA warp
 constexpr int kWarpTma = 8, kWarpMma = 9;
+// 4-token units: a second gather warp (on another SM sub-partition) copies half of every
+// K and V tile: warp 8 units 0..15, warp 10 units 16..31; warp 8 also loads Q
+constexpr int kWarpGather2 = 10;
+constexpr int attn_threads(bool units) { return units ? kAttnThreads + 32 : kAttnThreads; }
 constexpr int kTmemCols = 512;
 constexpr int kSBufs = 3;  // S / P buffers in TMEM, columns 128 b .. 128 b + 127
 constexpr int kColO = 384;
@@ -146,7 +150,7 @@ __device__ __forceinline__ int block_index(const AttnParams &p, int r, int i, bo
 }
 
 template <int D, bool kWeighted, bool kOutF32, bool kUnits>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(attn_threads(kUnits), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p)
 {
@@ -178,8 +182,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&o_full[b], 1);
         }
         for (int s = 0; s < L::kStages; ++s) {
-            // TMA: one arrive with the tile's byte count; units: one cp.async arrive per lane
-            mbar_init(&kv_full[s], kUnits ? 32 : 1);
+            // TMA: one arrive with the tile's byte count; units: one cp.async arrive per
+            // lane of the two gather warps
+            mbar_init(&kv_full[s], kUnits ? 64 : 1);
             mbar_init(&kv_empty[s], 1);
         }
         mbar_init(drain, 1);
@@ -195,11 +200,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kWarpTma) {
+    if (warp == kWarpTma || (kUnits && warp == kWarpGather2)) {
         // ------------------------------ TMA producer ------------------------------
+        // 4-token units: warps 8 and 10 both walk every ring position in order (so each
+        // warp's stage waits stay within one phase) and each copies its half of the
+        // tile's units; only warp 8 loads Q.
+        const bool do_q = warp == kWarpTma;
+        const int unit_half = warp == kWarpTma ? 0 : 1;
         // The whole warp runs the control flow (warp-uniform values); one elected lane
         // issues each copy.
-        if (elect_one()) {
+        if (elect_one() && do_q) {
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
@@ -212,6 +222,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag));
         };
         auto load_q = [&](const Cursor &c) -> bool {
+            if (!do_q) return true;
             const int b = c.seq & 1;
             if (!wait(&q_empty[b], ((c.seq >> 1) & 1) ^ 1)) return false;
             uint8_t *dst = smem + L::kQOff + b * L::kTileBytes;
@@ -239,7 +250,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (slot < cnt) {
                     u = __ldg(p.idx + (size_t)c.r * p.nkb + slot);
                     if (u < 0 || u >= p.nkb) {
-                        if (tm == &tmK) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
+                        if (tm == &tmK && unit_half == 0) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
                         u = -1;
                     }
                 }
@@ -247,7 +258,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const uint32_t dst = smem_u32(smem + L::kKVOff + s * L::kTileBytes);
                 const int rr = lane >> 3, c8 = lane & 7;
 #pragma unroll 4
-                for (int su = 0; su < 32; ++su) {
+                for (int su = unit_half * 16; su < unit_half * 16 + 16; ++su) {
                     const int us = __shfl_sync(0xffffffffu, u, su);
                     const int tok = us * 4 + rr;
                     const bool valid = us >= 0 && tok < p.N;
@@ -738,7 +749,7 @@ static cudaError_t launch_attn_t(const AttnLaunch &a, cudaStream_t st)
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = a.grid_override > 0 ? a.grid_override : (p.n_items < sms ? p.n_items : sms);
-    attn_fwd_kernel<D, W, F32, U4><<<grid, kAttnThreads, smem, st>>>(tq, tk, tv, p);
+    attn_fwd_kernel<D, W, F32, U4><<<grid, attn_threads(U4), smem, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
