@@ -44,7 +44,7 @@ constexpr int attn_threads(bool units) { return units ? kAttnThreads + 32 : kAtt
 constexpr int kTmemCols = 512;
 constexpr int kSBufs = 3;  // S / P buffers in TMEM, columns 128 b .. 128 b + 127
 constexpr int kColO = 384;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 256 without a rescale
+constexpr float kRescaleThreshold = 20.0f;  // log2 units: P stays <= 2^20 without a rescale (bf16 P and fp32 l / O hold that with room to spare)
 
 struct AttnParams {
     const int32_t *idx;

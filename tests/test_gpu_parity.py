@@ -236,7 +236,9 @@ def test_attn_hand_plans(orc, out_dtype):
     late block with a much larger logit than the first one."""
     N, d, H = 6 * 128, 128, 2
     q, k, v = _inputs(N, H=H, d=d, seed=5)
-    k[0, 0, 5 * 128:6 * 128] *= 6  # block 5 of head 0 dominates: forces a rescale
+    # block 5 of head 0 dominates: its logits exceed the running max of the earlier blocks
+    # by more than the lazy-rescale threshold (20 in log2 units), forcing O rescales
+    k[0, 0, 5 * 128:6 * 128] *= 12
     nb = 6
     idx = torch.full((1, H, nb, nb), -1, dtype=torch.int32)
     cnt = torch.zeros(1, H, nb, dtype=torch.int32)
