@@ -77,6 +77,7 @@ def lib():
         L.ab_score_units.argtypes = [P, P, S, I, I, I, P, P, P, P, P, P, ctypes.c_size_t, P, P]
         L.ab_attn_units_fwd.argtypes = [P, P, P, S, I, P, P, P, P, I, P, P, P]
         L.ab_attn_units_topk_fwd.argtypes = [P, P, P, S, I, P, P, P, I, P, P, P]
+        L.ab_selftest_bounded_wait.argtypes = [I, I, P, P, P]
         L.ab_check_flag.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
         L.ab_status_str.argtypes = [I]
         L.ab_status_str.restype = ctypes.c_char_p
@@ -85,7 +86,8 @@ def lib():
         L.ab_last_cuda_error.restype = ctypes.c_char_p
         for name in ("ab_score_workspace_size", "ab_score", "ab_score_noalloc", "ab_select", "ab_attn_fwd",
                      "ab_attn_topk_fwd", "ab_check_flag", "ab_version", "ab_score_units_workspace_size",
-                     "ab_score_units", "ab_attn_units_fwd", "ab_attn_units_topk_fwd"):
+                     "ab_score_units", "ab_attn_units_fwd", "ab_attn_units_topk_fwd",
+                     "ab_selftest_bounded_wait"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -252,6 +254,17 @@ def attn_topk_fwd(q, k, v, N: int, idx, cnt, want_lse: bool = False,
                                             _ptr(lse), _ptr(dev_flag), _stream()),
                "ab_attn_units_topk_fwd")
     return (o, lse) if want_lse else o
+
+
+def selftest_bounded_wait(limit_us: int, complete: bool, device="cuda"):
+    """Run the bounded-wait self test (include/ab_attn.h); returns (flag bits, done) with
+    done = 1 when the wait succeeded and 2 when it gave up."""
+    flag = torch.zeros(1, dtype=torch.int32, device=device)
+    done = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(lib().ab_selftest_bounded_wait(int(limit_us), int(bool(complete)), _ptr(flag), _ptr(done),
+                                          _stream()), "ab_selftest_bounded_wait")
+    bits = check_flag(flag)
+    return bits, int(done.item())
 
 
 def check_flag(dev_flag: torch.Tensor) -> int:

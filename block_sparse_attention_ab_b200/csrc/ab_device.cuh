@@ -68,10 +68,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait until the phase with the given parity has completed. Gives up after
-// kWaitLimitNs, or at once when *abort is set by another role; returns false then.
+// Wait until the phase with the given parity has completed. Gives up after limit_ns
+// (kWaitLimitNs in the kernels), or at once when *abort is set by another role; returns
+// false then, with *abort set and AB_FLAG_TIMEOUT raised on a timeout.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int *flag)
+                                          int *flag, uint64_t limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
@@ -80,7 +81,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (mbar_try_wait(bar, parity)) return true;
         if ((spin & 63u) == 0) {
             if (*abort) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 *abort = 1;
                 raise_flag(flag, AB_FLAG_TIMEOUT);
                 return false;

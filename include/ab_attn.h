@@ -163,6 +163,21 @@ ab_status ab_score_units(const void *q, const void *k, ab_shape s, int n_cluster
                          size_t workspace_bytes, int *dev_flag, void *stream);
 
 /*
+ * ab_selftest_bounded_wait -- exercises the failure path every pipeline of the library
+ * relies on, without a GPU fault. The method's pages have no counterpart; it exists so
+ * that a test can make an in-kernel wait run out. One CTA initialises an mbarrier that
+ * expects one arrival and waits on it with the library's bounded wait (limit limit_us
+ * microseconds, 1..1e6). With complete = 0 nothing arrives: the wait gives up after the
+ * limit, ORs AB_FLAG_TIMEOUT into *dev_flag and the kernel returns normally (*dev_done
+ * = 2), leaving the context usable. With complete != 0 the CTA arrives first and the
+ * wait succeeds (*dev_done = 1, no flag). dev_flag, dev_done: device ints owned by the
+ * caller. Asynchronous on `stream`; read the result with ab_check_flag.
+ * Errors: AB_ERR_NULL, AB_ERR_RANGE, AB_ERR_CUDA (launch).
+ */
+ab_status ab_selftest_bounded_wait(int limit_us, int complete, int *dev_flag, int *dev_done,
+                                   void *stream);
+
+/*
  * ab_select -- choose key blocks per query block (page section «Три приёма
  * AB-Attention», second technique SIP; section «Где ломаются прежние разреженные
  * схемы» for top-k).
