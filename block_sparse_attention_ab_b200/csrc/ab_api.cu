@@ -8,6 +8,19 @@
 #include "../../include/ab_attn.h"
 #include "ab_kernels.h"
 
+namespace ab {
+
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+ab_status status_of(cudaError_t e)
+{
+    if (e == cudaSuccess) return AB_OK;
+    g_last_cuda_error = e;
+    return AB_ERR_CUDA;
+}
+
+}  // namespace ab
+
 namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -39,14 +52,7 @@ ab_status check_unit(const ab_shape &s, int unit)
     return AB_OK;
 }
 
-thread_local cudaError_t g_last_cuda_error = cudaSuccess;
-
-ab_status cuda_status(cudaError_t e)
-{
-    if (e == cudaSuccess) return AB_OK;
-    g_last_cuda_error = e;
-    return AB_ERR_CUDA;
-}
+ab_status cuda_status(cudaError_t e) { return ab::status_of(e); }
 
 ab_status attn_common(const void *q, const void *k, const void *v, ab_shape s, int unit,
                       const int32_t *idx, const int32_t *cnt, const float *w, void *out,
@@ -240,7 +246,7 @@ const char *ab_status_str(ab_status s)
     return "AB_ERR_UNKNOWN";
 }
 
-const char *ab_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda_error); }
+const char *ab_last_cuda_error(void) { return cudaGetErrorString(ab::g_last_cuda_error); }
 
 int ab_version(void) { return 100; }
 

@@ -4,7 +4,12 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "../../include/ab_attn.h"
+
 namespace ab {
+
+// AB_OK, or AB_ERR_CUDA with the error kept for ab_last_cuda_error (ab_api.cu).
+ab_status status_of(cudaError_t e);
 
 // IBCS scoring (score_kernels.cu)
 // Device scratch of the scoring pass, each region 256-byte aligned: mean keys fp32

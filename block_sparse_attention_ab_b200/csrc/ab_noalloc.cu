@@ -77,5 +77,5 @@ extern "C" ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, 
                               dev_flag, cs);
     if (e == cudaSuccess)
         e = ab::launch_score(ce, cw, kt, scores, BH, nb, nb, nb, s.d, n_clusters, dev_flag, cs);
-    return e == cudaSuccess ? AB_OK : AB_ERR_CUDA;
+    return ab::status_of(e);
 }

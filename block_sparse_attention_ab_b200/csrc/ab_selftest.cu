@@ -5,6 +5,7 @@
 
 #include "../../include/ab_attn.h"
 #include "ab_device.cuh"
+#include "ab_kernels.h"
 
 namespace {
 
@@ -37,5 +38,5 @@ extern "C" ab_status ab_selftest_bounded_wait(int limit_us, int complete, int *d
     if (limit_us < 1 || limit_us > 1000000) return AB_ERR_RANGE;
     bounded_wait_kernel<<<1, 64, 0, (cudaStream_t)stream>>>(
         dev_flag, dev_done, (uint64_t)limit_us * 1000ull, complete ? 1 : 0);
-    return cudaGetLastError() == cudaSuccess ? AB_OK : AB_ERR_CUDA;
+    return ab::status_of(cudaGetLastError());
 }
