@@ -8,19 +8,23 @@
 // (CTA c takes items c, c + grid, ...), so concurrently running CTAs share a head's
 // K/V in L2. Per CTA, 320 threads in three roles:
 //   warps 0-7  softmax: warps q and q+4 own query rows 32q..32q+31 (TMEM lanes), warp
-//              q the first 64 key columns of each S row and warp q+4 the last 64; they
-//              read S from TMEM, run the online softmax in the log2 domain with the
-//              block's log2(w) added, write P (bf16) back over S, lazily rescale their
-//              half of O, and normalise and store their half of each output row;
+//              q the first 64 key columns of each S row and warp q+4 the last 64. Each
+//              warp runs its own online softmax (log2 domain, the block's log2(w)
+//              added) over its columns into its own O accumulator, writes P (bf16) back
+//              over its S columns and lazily rescales its O; at the end of a work item
+//              the two merge their (max, sum) once and each normalises and stores half
+//              of every output row from both accumulators;
 //   warp 8     TMA producer: Q tile (double buffered) and a ring of K / V tiles
 //              fetched by block index with 3-D tensor maps whose row extent is N, so
 //              rows past the sequence end arrive as zeros;
 //   warp 9     TMEM owner and MMA issuer: S = Q K^T (both operands from shared
-//              memory) into S buffer g mod 3, O += P V (P from TMEM).
-// Issue order of the MMA warp over the CTA's whole block stream g = 0, 1, ...:
-//   S(0), S(1), S(2), PV(0), S(3), PV(1), S(4), ...  S runs three blocks ahead, so the
+//              memory) into S buffer g mod kSB, O_h += P_h V_h for the two key halves h
+//              (P from TMEM).
+// TMEM: kSB S buffers of 128 columns (2 for d = 128, 3 for d = 64), then O_0 and O_1
+// (d fp32 columns each). Issue order of the MMA warp over the CTA's block stream:
+//   S(0), .., S(kSB - 1), PV(0), S(kSB), PV(1), ...  S runs kSB blocks ahead, so the
 // softmax never waits for a QK^T product, and nothing in the softmax waits for a PV
-// product except an O rescale (PV(g-1)) and the end of an item (PV(g)).
+// product except an O rescale (PV_h(g-1)) and the end of an item (PV(g)).
 // Every wait is bounded (2 s); on a timeout the roles unwind, drain their own
 // asynchronous work and the CTA frees its TMEM before returning.
 #include <cmath>
@@ -42,8 +46,16 @@ constexpr int kWarpTma = 8, kWarpMma = 9;
 constexpr int kWarpGather2 = 10;
 constexpr int attn_threads(bool units) { return units ? kAttnThreads + 32 : kAttnThreads; }
 constexpr int kTmemCols = 512;
-constexpr int kSBufs = 3;  // S / P buffers in TMEM, columns 128 b .. 128 b + 127
-constexpr int kColO = 384;
+constexpr int kSBufsMax = 3;
+// TMEM columns: S / P buffers (128 b .. 128 b + 127), then the O accumulator(s) of D
+// fp32 columns each. Shared softmax rows (blocks): 3 S buffers and one O. Split halves
+// (4-token units): O_0 and O_1 (O_h at kColO + h D), with 2 S buffers for D = 128.
+template <int D, bool kSplit>
+struct TmemPlan {
+    static constexpr int kSBufs = (kSplit && D == 128) ? 2 : 3;
+    static constexpr int kColO = kSBufs * 128;
+    static_assert(kColO + (kSplit ? 2 : 1) * D <= kTmemCols, "TMEM plan exceeds 512 columns");
+};
 constexpr float kRescaleThreshold = 20.0f;  // log2 units: P stays <= 2^20 without a rescale (bf16 P and fp32 l / O hold that with room to spare)
 
 struct AttnParams {
@@ -84,12 +96,13 @@ struct AttnSmem {
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[3], p_full[3],
-    // o_full[3], drain
-    static constexpr int kNumBars = 2 + 2 + kStages + kStages + 3 * kSBufs + 1;
+    // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[3], p_full[2][3],
+    // o_full[2][3], drain
+    static constexpr int kNumBars = 2 + 2 + kStages + kStages + 5 * kSBufsMax + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kXchOff = kMiscOff + 16;  // softmax exchange: float [2][2][128] + [2][128]
-    static constexpr int kBytes = kXchOff + (2 * 2 * 128 + 2 * 128) * 4;
+    // softmax exchange: float row max [2 blocks][2 halves][128], m [2][128], l [2][128]
+    static constexpr int kXchOff = kMiscOff + 16;
+    static constexpr int kBytes = kXchOff + (2 * 2 * 128 + 2 * 128 + 2 * 128) * 4;
     static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
 };
 
@@ -155,6 +168,12 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p)
 {
     using L = AttnSmem<D>;
+    // 4-token units: the two softmax halves of a row keep separate maxima and O
+    // accumulators (their per-unit masks and weights make the shared-max exchange the
+    // longer path); blocks: one shared row max per block and one O
+    constexpr bool kSplit = kUnits;
+    constexpr int kSB = TmemPlan<D, kSplit>::kSBufs;
+    constexpr int kColO = TmemPlan<D, kSplit>::kColO;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem_1024(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
@@ -163,9 +182,9 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
     uint64_t *kv_full = bars + 4;
     uint64_t *kv_empty = kv_full + L::kStages;
     uint64_t *s_full = kv_empty + L::kStages;
-    uint64_t *p_full = s_full + kSBufs;
-    uint64_t *o_full = p_full + kSBufs;
-    uint64_t *drain = o_full + kSBufs;
+    uint64_t *p_full = s_full + kSBufsMax;  // [h][b]: P_h of the block in S buffer b is in TMEM
+    uint64_t *o_full = p_full + 2 * kSBufsMax;  // [h][b]: PV_h of that block is complete
+    uint64_t *drain = o_full + 2 * kSBufsMax;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
 
@@ -176,10 +195,12 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             mbar_init(&q_full[b], 1);
             mbar_init(&q_empty[b], 1);
         }
-        for (int b = 0; b < kSBufs; ++b) {
+        for (int b = 0; b < kSB; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 256);
-            mbar_init(&o_full[b], 1);
+            for (int h = 0; h < (kSplit ? 2 : 1); ++h) {
+                mbar_init(&p_full[h * kSBufsMax + b], kSplit ? 128 : 256);
+                mbar_init(&o_full[h * kSBufsMax + b], 1);
+            }
         }
         for (int s = 0; s < L::kStages; ++s) {
             // TMA: one arrive with the tile's byte count; units: one cp.async arrive per
@@ -286,8 +307,8 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             ++kv_pos;
             return true;
         };
-        // tile order = the MMA warp's consumption order: K of the first kSBufs blocks,
-        // then V(g), K(g + kSBufs), V(g + 1), ...; a Q tile precedes its item's first K
+        // tile order = the MMA warp's consumption order: K of the first kSB blocks,
+        // then V(g), K(g + kSB), V(g + 1), ...; a Q tile precedes its item's first K
         Cursor kc = cursor_first(p), vc = kc;
         auto next_k = [&]() -> bool {
             bool r = true;
@@ -296,7 +317,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             cursor_next(kc, p);
             return r;
         };
-        for (int a = 0; a < kSBufs && ok && kc.r < p.n_items; ++a) ok = next_k();
+        for (int a = 0; a < kSB && ok && kc.r < p.n_items; ++a) ok = next_k();
         while (ok && vc.r < p.n_items) {
             ok = load_kv(vc, &tmV);
             cursor_next(vc, p);
@@ -336,14 +357,14 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             tc_fence_after();
             const uint64_t qd = q_desc0 + (uint64_t)qbuf * kTileDesc;
             const uint64_t kd = k_desc0 + (uint64_t)s * kTileDesc;
-            const uint32_t d_tmem = tmem + (g % kSBufs) * 128;
+            const uint32_t d_tmem = tmem + (g % kSB) * 128;
             if (elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
                     mma_ss(d_tmem, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&s_full[g % kSBufs]);
+                mma_commit(&s_full[g % kSB]);
                 mma_commit(&kv_empty[s]);
                 if (c.i == c.n - 1) mma_commit(&q_empty[qbuf]);
             }
@@ -353,38 +374,82 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         };
         Cursor sc = cursor_first(p), pc = sc;  // next S to issue, next PV to issue
         int gs = 0;                              // index of the next S
-        for (int a = 0; a < kSBufs && ok && sc.r < p.n_items; ++a) {
+        for (int a = 0; a < kSB && ok && sc.r < p.n_items; ++a) {
             ok = issue_s(sc, gs++);
             cursor_next(sc, p);
         }
         for (int g = 0; ok && pc.r < p.n_items; ++g) {
-            // O (+)= P(g) V(g)
-            if (!wait(&p_full[g % kSBufs], (g / kSBufs) & 1)) {
-                ok = false;
-                break;
-            }
-            const int s = kv_pos % L::kStages;
-            if (!wait(&kv_full[s], (kv_pos / L::kStages) & 1)) {
-                ok = false;
-                break;
-            }
-            if constexpr (kUnits) fence_proxy_async_smem();  // tile written by cp.async
-            tc_fence_after();
-            const uint64_t vd = v_desc0 + (uint64_t)s * kTileDesc;
-            const uint32_t p_tmem = tmem + (g % kSBufs) * 128;
-            const uint32_t acc0 = pc.i > 0 ? 1u : 0u;
-            if (elect_one()) {
+            const int b = g % kSB;
+            const uint32_t par = (g / kSB) & 1;
+            const bool first = pc.i == 0;
+            const uint32_t p_tmem = tmem + b * 128;
+            const uint32_t acc0 = first ? 0u : 1u;
+            if constexpr (!kSplit) {
+                // O (+)= P(g) V(g)
+                if (!wait(&p_full[b], par)) {
+                    ok = false;
+                    break;
+                }
+                const int s = kv_pos % L::kStages;
+                if (!wait(&kv_full[s], (kv_pos / L::kStages) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t vd = v_desc0 + (uint64_t)s * kTileDesc;
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < 128 / 16; ++kk)
-                    mma_ts(tmem + kColO, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)),
-                           idesc_pv, kk > 0 ? 1u : acc0);
-                mma_commit(&kv_empty[s]);
-                mma_commit(&o_full[g % kSBufs]);
+                    for (int kk = 0; kk < 128 / 16; ++kk)
+                        mma_ts(tmem + kColO, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)),
+                               idesc_pv, kk > 0 ? 1u : acc0);
+                    mma_commit(&kv_empty[s]);
+                    mma_commit(&o_full[b]);
+                }
+                __syncwarp();
+            } else {
+                // O_h (+)= P_h(g) V_h(g), h = 0, 1: the block's keys 64 h .. 64 h + 63 (P_h
+                // in TMEM columns 64 h .. 64 h + 31 of S buffer g mod kSB, V_h = V tile
+                // rows 64 h ..). An item's first PVs overwrite O_0 and O_1, which both
+                // softmax halves read in the previous item's epilogue: they wait for both
+                // P halves.
+                if ((first && !wait(&p_full[kSBufsMax + b], par)) || !wait(&p_full[b], par)) {
+                    ok = false;
+                    break;
+                }
+                const int s = kv_pos % L::kStages;
+                if (!wait(&kv_full[s], (kv_pos / L::kStages) & 1)) {
+                    ok = false;
+                    break;
+                }
+                if constexpr (kUnits) fence_proxy_async_smem();  // tile written by cp.async
+                tc_fence_after();
+                const uint64_t vd = v_desc0 + (uint64_t)s * kTileDesc;
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + kColO, p_tmem + kk * 8, vd + (uint64_t)(kk * (2048 >> 4)),
+                               idesc_pv, kk > 0 ? 1u : acc0);
+                    mma_commit(&o_full[b]);
+                }
+                __syncwarp();
+                if (!first && !wait(&p_full[kSBufsMax + b], par)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + kColO + D, p_tmem + 64 + kk * 8,
+                               vd + (uint64_t)((4 + kk) * (2048 >> 4)), idesc_pv, kk > 0 ? 1u : acc0);
+                    mma_commit(&kv_empty[s]);
+                    mma_commit(&o_full[kSBufsMax + b]);
+                }
+                __syncwarp();
             }
-            __syncwarp();
             ++kv_pos;
             cursor_next(pc, p);
-            // S(g + kSBufs) reuses the buffer whose P(g) was just consumed (in order)
+            // S(g + kSB) reuses the buffer whose P(g) was just consumed (in order)
             if (sc.r < p.n_items) {
                 ok = issue_s(sc, gs++);
                 cursor_next(sc, p);
@@ -399,38 +464,59 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         }
     } else {
         // -------------------------------- softmax ---------------------------------
-        // Warps q and q + 4 share TMEM lanes 32q..32q+31 (query rows); warp q takes S
-        // columns 0..63 of those rows, warp q + 4 columns 64..127. The row max is
-        // exchanged through shared memory across a 64-thread named barrier; warp q + 4
-        // writes P into columns 32..63, which warp q reads as S, only after it.
+        // Warps q and q + 4 share TMEM lanes 32q..32q+31 (query rows); warp q (half
+        // h = 0) takes S columns 0..63 of each block, warp q + 4 (h = 1) columns 64..127.
+        // Shared rows (blocks): the two exchange their block row max through shared
+        // memory across a 64-thread named barrier and run one online softmax into one O;
+        // warp q + 4 writes P into columns 32..63, which warp q reads as S, only after
+        // that barrier. Split halves (units): each warp runs its own online softmax over
+        // its columns (running max m_h, sum l_h) into its own accumulator O_h += P_h V_h,
+        // writing P_h over its own S columns 64 h .. 64 h + 31, so the two never wait for
+        // each other inside an item; at the end of an item they exchange (m, l) once and
+        // each writes half of the output columns from both accumulators:
+        //   O = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / (l_0 2^(m_0 - m) + l_1 2^(m_1 - m)),
+        //   m = max(m_0, m_1).
         // These warps never leave their loops early: after a failed (timed-out) wait
         // they skip the remaining waits but keep the same sequence of named barriers,
         // so a pair can never be left waiting for its partner.
         const int quad = warp & 3, half = warp >> 2;
         const int row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t col_o_own = kColO + (kSplit ? half * D : half * (D / 2));
+        const uint32_t col_o_oth = kColO + (half ^ 1) * D;  // split halves only
         float *xmax_sh = reinterpret_cast<float *>(smem + L::kXchOff);  // [2][2][128]
-        float *xl_sh = xmax_sh + 2 * 2 * 128;                            // [2][128]
+        float *xm_sh = xmax_sh + 2 * 2 * 128;                            // [2][128]
+        float *xl_sh = xm_sh + 2 * 128;                                  // [2][128]
+        const int hb = kSplit ? half * kSBufsMax : 0;
+        uint64_t *p_own = p_full + hb;
+        uint64_t *o_own = o_full + hb, *o_oth = o_full + (half ^ 1) * kSBufsMax;
         auto pair_sync = [&]() {
             tc_fence_before();
             asm volatile("bar.sync %0, 64;" ::"r"(1 + quad) : "memory");
             tc_fence_after();
         };
         int g = 0;
-        int o_seen = 0;  // PV completions observed so far
+        int o_seen = 0, o_seen_oth = 0;  // PV_h completions observed so far (own, other half)
         bool ok = true;
         auto wait_bar = [&](uint64_t *bar, uint32_t parity) {
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag));
         };
-        // wait until PV(k) is complete (k = g - 1 for a rescale, k = g at the end of an
-        // item). PV(k) completes phase k / 3 of o_full[k mod 3]. A parity wait is exact
-        // only within one phase of the barrier's state: PV(k - 3) is complete (S(g) was
-        // issued after PV(g - 3) and has completed) and PV(k + 3) cannot complete
-        // before P(k + 3) exists, so it is exact here.
+        // wait until PV_h(k) is complete (own half: k = g - 1 for a rescale; both halves:
+        // k = g at the end of an item). PV_h(k) completes phase k / kSB of o_full[h][k mod
+        // kSB]. A parity wait is exact only within one phase of the barrier's state:
+        // PV_h(k - kSB) is complete (S(g) was issued after it and has completed), and
+        // PV_h(k + kSB) cannot complete first: for the own half it needs P_h(k + kSB),
+        // which this warp has not written; for the other half at the end of an item it
+        // comes after the next item's first PV, which waits for this warp's next P.
         auto wait_o = [&](int k) {
             if (o_seen > k) return;
-            wait_bar(&o_full[k % kSBufs], (k / kSBufs) & 1);
+            wait_bar(&o_own[k % kSB], (k / kSB) & 1);
             o_seen = k + 1;
+        };
+        auto wait_o_oth = [&](int k) {
+            if (o_seen_oth > k) return;
+            wait_bar(&o_oth[k % kSB], (k / kSB) & 1);
+            o_seen_oth = k + 1;
         };
         auto lw_of = [&](float wj) -> float {  // log2 of a block weight (0 for top-k)
             if (!kWeighted) return 0.f;
@@ -522,8 +608,8 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                     }
                 }
                 const int nvalid = min(128, p.N - j * 128) - half * 64;  // blocks: valid columns here
-                const uint32_t s_col = (g % kSBufs) * 128;
-                wait_bar(&s_full[g % kSBufs], (g / kSBufs) & 1);
+                const uint32_t s_col = (g % kSB) * 128;
+                wait_bar(&s_full[g % kSB], (g / kSB) & 1);
                 tc_fence_after();
                 // the destination registers are only read after tcgen05.wait::ld
                 uint32_t su[64];
@@ -557,8 +643,8 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                     for (int e = 0; e < 64; ++e)
                         if (e >= nvalid) sv[e] = -INFINITY;
                 }
-                // row max: 8 independent chains of three-input max, then a tree; the two
-                // halves exchange theirs
+                // this half's row max: 8 independent chains of three-input max, then a tree;
+                // shared rows exchange theirs
                 float mx[8];
 #pragma unroll
                 for (int t = 0; t < 8; ++t) {
@@ -569,9 +655,12 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                 }
                 mx[0] = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
                               fmaxf(mx[6], mx[7]));
-                xmax_sh[((g & 1) * 2 + half) * 128 + row] = mx[0];
-                pair_sync();
-                const float smax = fmaxf(mx[0], xmax_sh[((g & 1) * 2 + (half ^ 1)) * 128 + row]);
+                float smax = mx[0];
+                if constexpr (!kSplit) {
+                    xmax_sh[((g & 1) * 2 + half) * 128 + row] = mx[0];
+                    pair_sync();
+                    smax = fmaxf(mx[0], xmax_sh[((g & 1) * 2 + (half ^ 1)) * 128 + row]);
+                }
                 float lw_n1 = 0.f;
                 if constexpr (kUnits) {
                     if (i + 1 < n) lw_n1 = unit_lw(j_n1, w_n1, nv_n);
@@ -588,14 +677,15 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                     rescale = true;
                 }
                 if (__any_sync(0xffffffffu, rescale)) {
-                    // O *= 2^(m_run - m_new) on the rows that need it; PV(g-1) must be done
+                    // O (split: O_h) *= 2^(m_run - m_new) on the rows that need it, this
+                    // warp's columns of it; PV(g-1) must be done
                     wait_o(g - 1);
                     tc_fence_after();
                     const float f = rescale ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll 1
-                    for (int ch = 0; ch < kHalfD / 32; ++ch) {
+                    for (int ch = 0; ch < (kSplit ? D : D / 2) / 32; ++ch) {
                         uint32_t r32[32];
-                        const uint32_t oc = kColO + half * kHalfD + ch * 32;
+                        const uint32_t oc = col_o_own + ch * 32;
                         tmem_ld32(tmem + lane_off + oc, r32);
                         tmem_wait_ld();
 #pragma unroll
@@ -609,10 +699,11 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                     }
                 }
                 // P = 2^(s * scale_log2 + lw - m_run) in fp32 pairs, packed to bf16 over
-                // the S columns; the first kSoftPairs pairs use the FMA-pipe exp2
-                // units: a row may have seen no valid key yet (every kept unit past the
-                // sequence end); its P is then 0, not NaN
-                const float m_ref = (kUnits && m_run == -INFINITY) ? 0.f : m_run;
+                // the S columns; the first kSoftPairs pairs use the FMA-pipe exp2.
+                // A half row may have seen no valid key yet (its columns of the block
+                // past the sequence end, or every kept unit there); its P is then 0, not
+                // NaN
+                const float m_ref = m_run == -INFINITY ? 0.f : m_run;
                 const float bias = kUnits ? -m_ref : lw - m_ref;
                 const uint64_t bias2 = f2_pack(bias, bias);
                 uint64_t ls2[4] = {0, 0, 0, 0};
@@ -632,14 +723,14 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                     ls2[e & 3] = f2_add(ls2[e & 3], f2_pack(pr.x, pr.y));
                     pk[e] = pack_bf16x2(pr.x, pr.y);
                 }
-                tmem_st32(tmem + lane_off + s_col + half * 32, pk);
+                tmem_st32(tmem + lane_off + s_col + half * (kSplit ? 64 : 32), pk);
                 {
                     const float2 a = f2_unpack(f2_add(f2_add(ls2[0], ls2[1]), f2_add(ls2[2], ls2[3])));
                     l_run += a.x + a.y;
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&p_full[g % kSBufs]);
+                mbar_arrive(&p_own[g % kSB]);
                 if (i + 1 < n) {
                     j = kUnits ? 0 : clamp_j(j_n1);
                     lw = lw_n1;
@@ -649,46 +740,58 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                 }
 
                 if (i == n - 1) {
-                    // epilogue: O / l (l summed over both halves), straight to global memory
+                    // epilogue: the item's last PV(s) done, (m, l) exchanged, this warp's
+                    // half of the output columns (split halves: from O_0 and O_1) divided
+                    // by l, straight to global memory
                     wait_o(g);
+                    if constexpr (kSplit) wait_o_oth(g);
+                    xm_sh[half * 128 + row] = m_run;
                     xl_sh[half * 128 + row] = l_run;
                     pair_sync();
-                    const float l_tot = l_run + xl_sh[(half ^ 1) * 128 + row];
+                    const float m_o = xm_sh[(half ^ 1) * 128 + row];
+                    const float l_o = xl_sh[(half ^ 1) * 128 + row];
+                    // shared rows: one max, l = l_0 + l_1; split halves: weight of each
+                    // accumulator 2^(m_h - m), 0 for a half that saw no key
+                    const float m_tot = kSplit ? fmaxf(m_run, m_o) : m_run;
+                    const float a_own = !kSplit ? 1.f : (m_run == -INFINITY ? 0.f : fast_exp2(m_run - m_tot));
+                    const float a_oth = !kSplit ? 1.f : (m_o == -INFINITY ? 0.f : fast_exp2(m_o - m_tot));
+                    const float l_tot = kSplit ? l_run * a_own + l_o * a_oth : l_run + l_o;
                     const float inv = (tok < p.N && l_tot > 0.f) ? 1.0f / l_tot : 0.f;
+                    const float c_own = a_own * inv, c_oth = a_oth * inv;
 #pragma unroll 1
                     for (int ch = 0; ch < kHalfD / 32; ++ch) {
-                        uint32_t r32[32];
-                        tmem_ld32(tmem + lane_off + kColO + half * kHalfD + ch * 32, r32);
-                        tmem_wait_ld();
+                        uint32_t ra[32], rb[32];
+                        float o[32];
+                        if constexpr (kSplit) {
+                            tmem_ld32(tmem + lane_off + col_o_own + half * kHalfD + ch * 32, ra);
+                            tmem_ld32(tmem + lane_off + col_o_oth + half * kHalfD + ch * 32, rb);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                o[e] = fmaf(__uint_as_float(ra[e]), c_own, __uint_as_float(rb[e]) * c_oth);
+                        } else {
+                            tmem_ld32(tmem + lane_off + col_o_own + ch * 32, ra);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(ra[e]) * inv;
+                        }
                         if (kOutF32) {
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                uint4 v;
-                                v.x = __float_as_uint(__uint_as_float(r32[4 * e + 0]) * inv);
-                                v.y = __float_as_uint(__uint_as_float(r32[4 * e + 1]) * inv);
-                                v.z = __float_as_uint(__uint_as_float(r32[4 * e + 2]) * inv);
-                                v.w = __float_as_uint(__uint_as_float(r32[4 * e + 3]) * inv);
-                                o4[ch * 8 + e] = v;
-                            }
+                            for (int e = 0; e < 8; ++e)
+                                o4[ch * 8 + e] = make_uint4(__float_as_uint(o[4 * e + 0]), __float_as_uint(o[4 * e + 1]),
+                                                            __float_as_uint(o[4 * e + 2]), __float_as_uint(o[4 * e + 3]));
                         } else {
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                uint4 v;
-                                v.x = pack_bf16x2(__uint_as_float(r32[8 * e + 0]) * inv,
-                                                  __uint_as_float(r32[8 * e + 1]) * inv);
-                                v.y = pack_bf16x2(__uint_as_float(r32[8 * e + 2]) * inv,
-                                                  __uint_as_float(r32[8 * e + 3]) * inv);
-                                v.z = pack_bf16x2(__uint_as_float(r32[8 * e + 4]) * inv,
-                                                  __uint_as_float(r32[8 * e + 5]) * inv);
-                                v.w = pack_bf16x2(__uint_as_float(r32[8 * e + 6]) * inv,
-                                                  __uint_as_float(r32[8 * e + 7]) * inv);
-                                o4[ch * 4 + e] = v;
-                            }
+                            for (int e = 0; e < 4; ++e)
+                                o4[ch * 4 + e] = make_uint4(pack_bf16x2(o[8 * e + 0], o[8 * e + 1]),
+                                                            pack_bf16x2(o[8 * e + 2], o[8 * e + 3]),
+                                                            pack_bf16x2(o[8 * e + 4], o[8 * e + 5]),
+                                                            pack_bf16x2(o[8 * e + 6], o[8 * e + 7]));
                         }
                     }
                     if (p.lse && half == 0)
                         p.lse[(size_t)bh * p.N_pad + tok] =
-                            tok < p.N ? (l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f
+                            tok < p.N ? (l_tot > 0.f ? (m_tot + log2f(l_tot)) * 0.69314718055994531f
                                                      : -INFINITY)
                                       : 0.f;
                 }
