@@ -90,6 +90,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// The same bounded wait for a warp off the critical path: between polls it sleeps
+// (~sleep_ns), so that it takes no issue slots from the warps sharing its SM
+// sub-partition.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                 int *flag, unsigned sleep_ns = 500,
+                                                 uint64_t limit_ns = kWaitLimitNs)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            *abort = 1;
+            raise_flag(flag, AB_FLAG_TIMEOUT);
+            return false;
+        }
+        __nanosleep(sleep_ns);
+        if (mbar_try_wait(bar, parity)) return true;
+    }
+}
+
 // Bounded wait that ignores the abort flag: used only while unwinding, to let copies
 // and MMAs already in flight land before the CTA releases its memory.
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity)

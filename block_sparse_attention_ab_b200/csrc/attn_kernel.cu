@@ -27,6 +27,7 @@
 // product except an O rescale (PV_h(g-1)) and the end of an item (PV(g)).
 // Every wait is bounded (2 s); on a timeout the roles unwind, drain their own
 // asynchronous work and the CTA frees its TMEM before returning.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cuda.h>
@@ -39,14 +40,16 @@
 
 namespace ab {
 
-constexpr int kAttnThreads = 320;  // 8 softmax warps, 1 TMA warp, 1 MMA warp
 constexpr int kWarpTma = 8, kWarpMma = 9;
 // 4-token units: a second gather warp (on another SM sub-partition) copies half of every
 // K and V tile: warp 8 units 0..15, warp 10 units 16..31; warp 8 also loads Q
 constexpr int kWarpGather2 = 10;
-constexpr int attn_threads(bool units) { return units ? kAttnThreads + 32 : kAttnThreads; }
+// the item scheduler: warp 10 (key blocks) or 11 (units)
+constexpr int sched_warp(bool units) { return units ? 11 : 10; }
+constexpr int attn_threads(bool units) { return (sched_warp(units) + 1) * 32; }
 constexpr int kTmemCols = 512;
 constexpr int kSBufsMax = 3;
+constexpr int kRing = 16;  // work items published ahead to the roles (more than any role's lead)
 // TMEM columns: S / P buffers (128 b .. 128 b + 127), then the O accumulator(s) of D
 // fp32 columns each. Shared softmax rows (blocks): 3 S buffers and one O. Split halves
 // (4-token units): O_0 and O_1 (O_h at kColO + h D), with 2 S buffers for D = 128.
@@ -70,7 +73,9 @@ struct AttnParams {
     int nkb;       // entries per idx / w row: key blocks (N_pad / 128) or key units (N_pad / 4)
     int per_tile;  // selected entries per 128-key tile: 1 (blocks) or 32 (units)
     int n_items;
-    float scale_log2;  // log2(e) / sqrt(d)
+    float scale_log2;       // log2(e) / sqrt(d)
+    unsigned int *counter;  // [2]: items claimed, CTAs finished (zero at launch; the last
+                            // CTA to finish sets both back to zero)
 };
 
 // 4-token key units: one 16-byte cp.async per lane (zero fill when src_bytes == 0) and
@@ -97,59 +102,101 @@ struct AttnSmem {
     static constexpr int kKVOff = 2 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
     // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[3], p_full[2][3],
-    // o_full[2][3], drain
-    static constexpr int kNumBars = 2 + 2 + kStages + kStages + 5 * kSBufsMax + 1;
+    // o_full[2][3], drain, ring_full[R], ring_empty[R], started
+    static constexpr int kNumBars = 2 + 2 + kStages + kStages + 5 * kSBufsMax + 1 + 2 * kRing + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     // softmax exchange: float row max [2 blocks][2 halves][128], m [2][128], l [2][128]
     static constexpr int kXchOff = kMiscOff + 16;
-    static constexpr int kBytes = kXchOff + (2 * 2 * 128 + 2 * 128 + 2 * 128) * 4;
+    static constexpr int kRingOff = kXchOff + (2 * 2 * 128 + 2 * 128 + 2 * 128) * 4;  // int [R][2]
+    static constexpr int kItemXchOff = kRingOff + kRing * 8;  // softmax pairs: int [2][2][4]
+    static constexpr int kBytes = kItemXchOff + 2 * 2 * 4 * 4;
     static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B
 };
 
-// The per-CTA stream of (item, block) pairs shared by the three roles.
+// Work items are handed out dynamically. A scheduler warp per CTA takes the CTA's first
+// item c = blockIdx.x and then claims each further item from a global counter (r =
+// gridDim.x + the counter's old value; r >= n_items ends the CTA's stream), one item
+// ahead of the CTA's K loads: claim t + 1 waits until the TMA warp has started item t.
+// It writes the output of an empty item itself (O = 0, lse = -inf) and publishes the
+// others in a ring of kRing entries in shared memory, from which every role reads the
+// CTA's item sequence, so all roles walk the same items in the same order. A CTA takes
+// a new item only when it is nearly done with the last, so the CTAs finish together
+// however unevenly the selected blocks are spread over the items (a fixed assignment of
+// items c, c + grid, ... leaves the CTAs whose items hold the most blocks running last).
+// Claims follow the natural head-major order, so the CTAs running at any time still work
+// on neighbouring items and share a head's K/V in L2.
+struct ItemRing {
+    volatile int *items;     // [kRing][2]: item t of the sequence and its clamped entry count,
+                             // in entry t mod kRing
+    uint64_t *full, *empty;  // [kRing] each: entry published; entry read by every reader
+    uint64_t *started;       // one phase per item the TMA warp's K loads enter (t >= 1)
+    volatile int *abort;
+    int *flag;
+};
+
+// Item t of the sequence and its entry count once published; one arrive per reading warp
+// releases the entry. False (and r = n_items) when the wait failed (timeout or abort).
+__device__ __forceinline__ bool ring_read(const ItemRing &q, int n_items, int t, int &r, int &cnt)
+{
+    const int slot = t % kRing;
+    r = n_items;
+    cnt = 0;
+    if (!__all_sync(0xffffffffu, mbar_wait(&q.full[slot], (t / kRing) & 1, q.abort, q.flag))) return false;
+    r = q.items[2 * slot];
+    cnt = q.items[2 * slot + 1];
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&q.empty[slot]);
+    return true;
+}
+
+// One role's walk over the CTA's (item, tile) stream.
 struct Cursor {
     int r;    // work item (flat (b*H + h)*nqb + qb); >= n_items when done
     int i;    // tile position within the item
-    int n;    // tiles of the item: selected entries (clamped to [0, nkb]) / per_tile, rounded up
-    int seq;  // index of the item among this CTA's non-empty items
+    int n;    // tiles of the item: cnt / per_tile, rounded up
+    int seq;  // index of the item among this CTA's items
+    int cnt;  // selected entries of item r, clamped to [0, nkb]
+    int t;    // position of item r in the CTA's item sequence
 };
 
-__device__ __forceinline__ int load_cnt(const AttnParams &p, int r)
+// Read item t of the sequence into the cursor. `lead`: the TMA warp's K cursor, which
+// tells the scheduler each time it starts an item (the scheduler then claims the next).
+__device__ __forceinline__ bool cursor_load(Cursor &c, const AttnParams &p, const ItemRing &q, bool lead)
 {
-    const int c = __ldg(p.cnt + r);
-    return c < 0 ? 0 : (c > p.nkb ? p.nkb : c);
+    const bool ok = ring_read(q, p.n_items, c.t, c.r, c.cnt);
+    c.n = (c.cnt + p.per_tile - 1) / p.per_tile;
+    c.i = 0;
+    if (lead && c.t >= 1 && c.r < p.n_items) {
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(q.started);
+    }
+    return ok;
 }
 
-__device__ __forceinline__ int load_tiles(const AttnParams &p, int r)
-{
-    return (load_cnt(p, r) + p.per_tile - 1) / p.per_tile;
-}
-
-__device__ __forceinline__ void cursor_seek(Cursor &c, const AttnParams &p)
+// Move past finished items.
+__device__ __forceinline__ bool cursor_seek(Cursor &c, const AttnParams &p, const ItemRing &q,
+                                            bool lead)
 {
     while (c.r < p.n_items && c.i >= c.n) {
         if (c.n > 0) ++c.seq;
-        c.r += gridDim.x;
-        c.i = 0;
-        c.n = c.r < p.n_items ? load_tiles(p, c.r) : 0;
+        ++c.t;
+        if (!cursor_load(c, p, q, lead)) return false;
     }
+    return true;
 }
 
-__device__ __forceinline__ Cursor cursor_first(const AttnParams &p)
+__device__ __forceinline__ bool cursor_first(Cursor &c, const AttnParams &p, const ItemRing &q,
+                                             bool lead)
 {
-    Cursor c;
-    c.r = blockIdx.x;
-    c.i = 0;
     c.seq = 0;
-    c.n = c.r < p.n_items ? load_tiles(p, c.r) : 0;
-    cursor_seek(c, p);
-    return c;
+    c.t = 0;
+    return cursor_load(c, p, q, lead) && cursor_seek(c, p, q, lead);
 }
 
-__device__ __forceinline__ void cursor_next(Cursor &c, const AttnParams &p)
+__device__ __forceinline__ bool cursor_next(Cursor &c, const AttnParams &p, const ItemRing &q, bool lead)
 {
     ++c.i;
-    cursor_seek(c, p);
+    return cursor_seek(c, p, q, lead);
 }
 
 __device__ __forceinline__ int block_index(const AttnParams &p, int r, int i, bool report)
@@ -185,10 +232,21 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
     uint64_t *p_full = s_full + kSBufsMax;  // [h][b]: P_h of the block in S buffer b is in TMEM
     uint64_t *o_full = p_full + 2 * kSBufsMax;  // [h][b]: PV_h of that block is complete
     uint64_t *drain = o_full + 2 * kSBufsMax;
+    uint64_t *ring_full = drain + 1, *ring_empty = ring_full + kRing, *started = ring_empty + kRing;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMiscOff);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMiscOff + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    ItemRing iq;
+    iq.items = reinterpret_cast<volatile int *>(smem + L::kRingOff);
+    iq.full = ring_full;
+    iq.empty = ring_empty;
+    iq.started = started;
+    iq.abort = abort_flag;
+    iq.flag = p.flag;
+    // readers of every ring entry, one arrive each: the K and V cursors of warp 8 (and of
+    // warp 10 for units), the S and PV cursors of the MMA warp, the 8 softmax warps
+    constexpr int kRingReaders = 2 + (kUnits ? 2 : 0) + 2 + 8;
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
@@ -209,6 +267,11 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             mbar_init(&kv_empty[s], 1);
         }
         mbar_init(drain, 1);
+        for (int e = 0; e < kRing; ++e) {
+            mbar_init(&ring_full[e], 1);
+            mbar_init(&ring_empty[e], kRingReaders);
+        }
+        mbar_init(started, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -265,7 +328,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                 // gather 32 units of 4 key rows into tile rows 4 s' .. 4 s' + 3, in the
                 // 128-byte-swizzled layout the MMA descriptors read; one warp
                 // instruction copies one unit's 4 rows x 64 columns (lane = row, chunk)
-                const int cnt = load_cnt(p, c.r);
+                const int cnt = c.cnt;
                 const int slot = c.i * 32 + lane;
                 int u = -1;
                 if (slot < cnt) {
@@ -309,18 +372,20 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         };
         // tile order = the MMA warp's consumption order: K of the first kSB blocks,
         // then V(g), K(g + kSB), V(g + 1), ...; a Q tile precedes its item's first K
-        Cursor kc = cursor_first(p), vc = kc;
+        // warp 8's K cursor tells the scheduler when it starts an item
+        Cursor kc, vc;
+        ok = cursor_first(kc, p, iq, warp == kWarpTma);
+        ok = cursor_first(vc, p, iq, false) && ok;
         auto next_k = [&]() -> bool {
             bool r = true;
             if (kc.i == 0) r = load_q(kc);
             r = r && load_kv(kc, &tmK);
-            cursor_next(kc, p);
-            return r;
+            return cursor_next(kc, p, iq, warp == kWarpTma) && r;
         };
         for (int a = 0; a < kSB && ok && kc.r < p.n_items; ++a) ok = next_k();
         while (ok && vc.r < p.n_items) {
             ok = load_kv(vc, &tmV);
-            cursor_next(vc, p);
+            ok = cursor_next(vc, p, iq, false) && ok;
             if (ok && kc.r < p.n_items) ok = next_k();
         }
         if (!ok) {
@@ -372,11 +437,13 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             ++kv_pos;
             return true;
         };
-        Cursor sc = cursor_first(p), pc = sc;  // next S to issue, next PV to issue
-        int gs = 0;                              // index of the next S
+        Cursor sc, pc;  // next S to issue, next PV to issue
+        ok = cursor_first(sc, p, iq, false);
+        ok = cursor_first(pc, p, iq, false) && ok;
+        int gs = 0;  // index of the next S
         for (int a = 0; a < kSB && ok && sc.r < p.n_items; ++a) {
             ok = issue_s(sc, gs++);
-            cursor_next(sc, p);
+            ok = cursor_next(sc, p, iq, false) && ok;
         }
         for (int g = 0; ok && pc.r < p.n_items; ++g) {
             const int b = g % kSB;
@@ -448,11 +515,11 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                 __syncwarp();
             }
             ++kv_pos;
-            cursor_next(pc, p);
+            ok = cursor_next(pc, p, iq, false);
             // S(g + kSB) reuses the buffer whose P(g) was just consumed (in order)
-            if (sc.r < p.n_items) {
+            if (ok && sc.r < p.n_items) {
                 ok = issue_s(sc, gs++);
-                cursor_next(sc, p);
+                ok = cursor_next(sc, p, iq, false) && ok;
             }
         }
         if (!ok) {
@@ -461,6 +528,58 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                 drain_wait(drain, 0);
             }
             __syncwarp();
+        }
+    } else if (warp == sched_warp(kUnits)) {
+        // ------------------------------ item scheduler ----------------------------
+        // Entry 0: the CTA's first item; entry t >= 2 once the K loads have entered item
+        // t - 1; empty items get their output here (O = 0; lse = -inf, 0 on padding rows)
+        // and are not published. Its waits sleep between polls: it shares an SM
+        // sub-partition with two softmax warps.
+        bool ok = true;
+        auto claim = [&]() -> int {
+            int c = 0;
+            if (lane == 0) c = (int)min(atomicAdd(p.counter, 1u), (unsigned)p.n_items);
+            c = __shfl_sync(0xffffffffu, c, 0);
+            return min((int)gridDim.x + c, p.n_items);
+        };
+        auto write_empty = [&](int r) {
+            const int bh = r / p.nqb, qb = r % p.nqb;
+            constexpr int kVecs = D * (kOutF32 ? 4 : 2) / 16;  // uint4 per output row
+            for (int rr = lane; rr < 128; rr += 32) {
+                const int tok = qb * 128 + rr;
+                const size_t off = ((size_t)bh * p.N_pad + tok) * D;
+                uint4 *o4 = kOutF32 ? reinterpret_cast<uint4 *>(static_cast<float *>(p.out) + off)
+                                    : reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + off);
+#pragma unroll 4
+                for (int e = 0; e < kVecs; ++e) o4[e] = make_uint4(0, 0, 0, 0);
+                if (p.lse) p.lse[(size_t)bh * p.N_pad + tok] = tok < p.N ? -INFINITY : 0.f;
+            }
+        };
+        int r = blockIdx.x < (unsigned)p.n_items ? (int)blockIdx.x : p.n_items;
+        for (int t = 0; ok; ++t) {
+            if (t >= 2) ok = __all_sync(0xffffffffu, mbar_wait_sleepy(started, (t - 2) & 1, abort_flag, p.flag));
+            if (!ok) break;
+            if (t > 0) r = claim();
+            int c_raw = 0;
+            while (r < p.n_items) {
+                c_raw = __ldg(p.cnt + r);
+                if ((c_raw < 0 || c_raw > p.nkb) && lane == 0) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
+                if (c_raw > 0) break;
+                write_empty(r);
+                r = claim();
+            }
+            // entry t once every reader has read its previous use
+            const int slot = t % kRing;
+            if (t >= kRing &&
+                !__all_sync(0xffffffffu, mbar_wait_sleepy(&ring_empty[slot], ((t / kRing) - 1) & 1, abort_flag, p.flag)))
+                break;
+            if (lane == 0) {
+                iq.items[2 * slot] = r;
+                iq.items[2 * slot + 1] = r < p.n_items ? min(c_raw, p.nkb) : 0;
+                mbar_arrive(&ring_full[slot]);  // release: the entry is visible to a reader's acquire
+            }
+            __syncwarp();
+            if (r >= p.n_items) break;
         }
     } else {
         // -------------------------------- softmax ---------------------------------
@@ -528,8 +647,22 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         constexpr int kHalfD = D / 2;
         constexpr int kSoftPairs = 6;  // of 32 pairs per block: exp2 on the FMA pipe
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
-        for (int r = blockIdx.x; r < p.n_items; r += gridDim.x) {
-            const int cnt_r = load_cnt(p, r);
+        // Item t of the CTA's sequence from the ring. The two warps of a pair take the
+        // smaller of their two reads (n_items after a failed wait), so they always walk
+        // the same items and meet at the same named barriers.
+        int *item_xch = reinterpret_cast<int *>(smem + L::kItemXchOff);  // [2 parities][2][4]
+        int t_item = 0, cnt_item = 0;
+        auto next_item = [&]() -> int {
+            int r2;
+            ring_read(iq, p.n_items, t_item, r2, cnt_item);
+            item_xch[((t_item & 1) * 2 + half) * 4 + quad] = r2;
+            pair_sync();
+            r2 = min(r2, item_xch[((t_item & 1) * 2 + (half ^ 1)) * 4 + quad]);
+            ++t_item;
+            return r2;
+        };
+        for (int r = next_item(); r < p.n_items; r = next_item()) {
+            const int cnt_r = cnt_item;
             const int n = kUnits ? (cnt_r + 31) / 32 : cnt_r;  // 128-key tiles of this item
             const int bh = r / p.nqb, qb = r % p.nqb;
             const int tok = qb * 128 + row;
@@ -538,10 +671,6 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             uint4 *o4 = kOutF32 ? reinterpret_cast<uint4 *>(static_cast<float *>(p.out) + orow_off)
                                 : reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + orow_off);
             constexpr int kRowVecs = kOutF32 ? kHalfD / 4 : kHalfD / 8;
-            if (warp == 0 && lane == 0) {
-                const int c = __ldg(p.cnt + r);
-                if (c < 0 || c > p.nkb) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
-            }
             if (n == 0) {
 #pragma unroll
                 for (int e = 0; e < kRowVecs; ++e) o4[e] = make_uint4(0, 0, 0, 0);
@@ -806,6 +935,16 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if (threadIdx.x == 0) {
+        // the last CTA to finish (all claims are made) returns the counter to zero for
+        // the next launch that uses it
+        __threadfence();
+        if (atomicAdd(p.counter + 1, 1u) == gridDim.x - 1) {
+            p.counter[0] = 0;
+            p.counter[1] = 0;
+            __threadfence();
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------------
@@ -817,6 +956,23 @@ static bool make_tmap(CUtensorMap *tm, const void *base, int BH, int N, int N_pa
 {
     return make_tmap_bf16_3d(tm, base, (uint64_t)d, (uint64_t)N, (uint64_t)BH, (uint64_t)d * 2,
                              (uint64_t)N_pad * d * 2, 64, 128);
+}
+
+// Claim counters of the item scheduler, one pair per launch slot: a launch takes the next
+// slot in turn and its last CTA leaves the pair at zero, so launches on one stream reuse a
+// slot safely and up to kCounterSlots launches can run at once on different streams.
+constexpr unsigned kCounterSlots = 4096;
+__device__ unsigned int g_item_counters[kCounterSlots][2];
+static std::atomic<unsigned> g_counter_next{0};
+
+static cudaError_t counter_slot(unsigned int **slot)
+{
+    void *base = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&base, g_item_counters);
+    if (e != cudaSuccess) return e;
+    const unsigned k = g_counter_next.fetch_add(1, std::memory_order_relaxed) % kCounterSlots;
+    *slot = static_cast<unsigned int *>(base) + 2 * k;
+    return cudaSuccess;
 }
 
 template <int D, bool W, bool F32, bool U4>
@@ -844,8 +1000,10 @@ static cudaError_t launch_attn_t(const AttnLaunch &a, cudaStream_t st)
     p.per_tile = U4 ? 32 : 1;
     p.n_items = a.B * a.H * p.nqb;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    cudaError_t e = counter_slot(&p.counter);
+    if (e != cudaSuccess) return e;
     const int smem = AttnSmem<D>::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, W, F32, U4>,
+    e = cudaFuncSetAttribute(attn_fwd_kernel<D, W, F32, U4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
