@@ -223,6 +223,10 @@ ab_status ab_select(const float *scores, int B, int H, int nqb, int nkb, int bud
  *           -inf for an empty selection).
  * Device-side: an idx/cnt outside range sets AB_FLAG_BAD_INDEX (the block is clamped
  * into range), a bad weight sets AB_FLAG_BAD_WEIGHT.
+ * Scheduling: the kernel hands the (b, h, query block) items to its persistent CTAs
+ * from a claim counter; each call takes the next of 4096 library-owned counters in turn
+ * and leaves it at zero when it ends, so calls on one stream (or captured in one graph)
+ * need nothing, and up to 4096 calls may run concurrently on different streams.
  * Errors: AB_ERR_NULL, AB_ERR_SHAPE, AB_ERR_DTYPE (inputs not bf16, or out_dtype not
  * AB_BF16 / AB_F32), AB_ERR_UNSUPPORTED, AB_ERR_ALIGN, AB_ERR_CUDA.
  */
