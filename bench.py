@@ -45,18 +45,29 @@ import torch  # noqa: E402
 L2_BYTES = 126 * 2**20
 
 
+def kernel_source_hash(csrc: str) -> str:
+    """First 16 hex digits of a SHA-256 over the attention kernel's sources with comments
+    and blank lines removed, so that an edit of comments alone keeps the hash."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in ("attn_kernel.cu", "ab_device.cuh"):
+        text = open(os.path.join(csrc, f), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln).encode())
+    return h.hexdigest()[:16]
+
+
 def attn_traffic_from_profile():
     """DRAM bytes per attention launch recorded in profiles/attn_fwd_wan13b.md, or None
     when the kernel source changed since that capture (hash mismatch)."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", "attn_fwd_wan13b.md")
     csrc = os.path.join(ROOT, "block_sparse_attention_ab_b200", "csrc")
     try:
         rec = dict(line.split(":", 1) for line in open(path) if line.startswith(("traffic_bytes", "kernel_source")))
-        h = hashlib.sha256()
-        for f in ("attn_kernel.cu", "ab_device.cuh"):
-            h.update(open(os.path.join(csrc, f), "rb").read())
-        if h.hexdigest()[:16] != rec["kernel_source_sha256_16"].strip():
+        if kernel_source_hash(csrc) != rec["kernel_source_sha256_16"].strip():
             return None
         return float(rec["traffic_bytes_per_launch"])
     except (OSError, KeyError, ValueError):

@@ -4,27 +4,32 @@
 // which keeps the computation ordinary softmax attention with a logit shift; the
 // kernel gathers the chosen key/value blocks by index, tokens stay in order).
 //
-// One persistent CTA per SM walks work items (b, h, query block) in head-major order
-// (CTA c takes items c, c + grid, ...), so concurrently running CTAs share a head's
-// K/V in L2. Per CTA, 320 threads in three roles:
+// One persistent CTA per SM works through (b, h, query block) items, claimed one at a
+// time from a global counter in head-major order (see the item scheduler below), so the
+// CTAs running at any time share a head's K/V in L2 and finish together. Per CTA, 352
+// threads (384 for 4-token units) in four roles:
 //   warps 0-7  softmax: warps q and q+4 own query rows 32q..32q+31 (TMEM lanes), warp
-//              q the first 64 key columns of each S row and warp q+4 the last 64. Each
-//              warp runs its own online softmax (log2 domain, the block's log2(w)
-//              added) over its columns into its own O accumulator, writes P (bf16) back
-//              over its S columns and lazily rescales its O; at the end of a work item
-//              the two merge their (max, sum) once and each normalises and stores half
-//              of every output row from both accumulators;
+//              q the first 64 key columns of each S row and warp q+4 the last 64; the
+//              online softmax runs in the log2 domain with the block's log2(w) added,
+//              writes P (bf16) back over S and lazily rescales O. Key blocks: the two
+//              warps exchange each block's row max and share one O; 4-token units: each
+//              warp keeps its own max, sum and O accumulator and the two merge once per
+//              item. Each warp normalises and stores half of every output row;
 //   warp 8     TMA producer: Q tile (double buffered) and a ring of K / V tiles
 //              fetched by block index with 3-D tensor maps whose row extent is N, so
-//              rows past the sequence end arrive as zeros;
+//              rows past the sequence end arrive as zeros (units: warps 8 and 10 gather
+//              the tiles with cp.async);
 //   warp 9     TMEM owner and MMA issuer: S = Q K^T (both operands from shared
-//              memory) into S buffer g mod kSB, O_h += P_h V_h for the two key halves h
-//              (P from TMEM).
-// TMEM: kSB S buffers of 128 columns (2 for d = 128, 3 for d = 64), then O_0 and O_1
-// (d fp32 columns each). Issue order of the MMA warp over the CTA's block stream:
+//              memory) into S buffer g mod kSB, O (+)= P V with P read from TMEM (units:
+//              O_h += P_h V_h for the two key halves h);
+//   warp 10    item scheduler (warp 11 for units): claims the items and publishes them
+//              to the other roles through a ring in shared memory.
+// TMEM: kSB S buffers of 128 columns, then the O accumulator(s) (d fp32 columns each):
+// 3 S buffers and one O for key blocks; O_0 and O_1 for units, with 2 S buffers at
+// d = 128. Issue order of the MMA warp over the CTA's block stream:
 //   S(0), .., S(kSB - 1), PV(0), S(kSB), PV(1), ...  S runs kSB blocks ahead, so the
 // softmax never waits for a QK^T product, and nothing in the softmax waits for a PV
-// product except an O rescale (PV_h(g-1)) and the end of an item (PV(g)).
+// product except an O rescale (PV(g-1)) and the end of an item (PV(g)).
 // Every wait is bounded (2 s); on a timeout the roles unwind, drain their own
 // asynchronous work and the CTA frees its TMEM before returning.
 #include <atomic>
