@@ -2,31 +2,49 @@
 
 One step = one pass of the method over one batch of synthetic input: IBCS scoring
 (mean keys, per-block k-means, block scores) -> SIP selection -> HT-weighted block-sparse
-attention. The top-k mode (top-k selection -> unweighted sparse attention) is timed in
-the same run with the same protocol and reported beside it.
+attention.
 
-Workload (default): Wan2.1-1.3B-shaped 480p clip, B=1, H=12, N=21x30x52=32760 tokens
-(padded to 32768), d=128, bf16, budget 10% of key blocks (26 of 256), 8 clusters, 5
-k-means iterations; synthetic inputs from block_sparse_attention_ab_b200.synth.
+Headline workload (the largest single-GPU configuration): the long-context stress case,
+B=1, H=24, N=64^3=262144 tokens, d=128, bf16, attention mass concentrated on 2% of the
+key blocks, SIP budget 10% of the key blocks (205 of 2048), 8 clusters, 5 k-means
+iterations; synthetic inputs from block_sparse_attention_ab_b200.synth.
 
 Metric: dense-equivalent TFLOPS = 4 B H N^2 d / step time (N valid tokens), plus the
 sparse-attention kernel's ms/call and its tensor-pipe roofline on selected-block FLOPs
-(4 * 128 * 128 * d per kept (query block, key block) pair).
+(4 * 128 * 128 * d per kept (query block, key block) pair) and the scoring pass's HBM
+roofline.
 
-Also reported, each in its own timed region after the main one: the amortised step
-with plan reuse (score + SIP select once every --reuse steps, attention every step: the
-pages' deployment schedule), the same path with the pages' 4-token key units at the same
-tile budget (units gathered 32 per 128-key tile), and the same attention kernel run dense
-(every key block kept), the comparison the pages make against dense attention.
+Timed region of the headline: K steps back to back, CUDA events on the launching stream,
+bracketed by synchronize (+ barrier for N > 1); per-stage events inside it. The inputs
+(Q+K+V = 4.8 GB) are far larger than the 126 MB L2, so no flush is needed there.
+
+Also reported, each in its own timed region after the headline (per-call CUDA events,
+median and min; "cold" = a 256 MB buffer written before each call to flush L2):
+  topk           the same step in the top-k mode at the same budget;
+  budget_sweep   SIP at every budget of the long-context workload (5..30%);
+  workloads      the Wan2.1-1.3B, Wan2.1-14B (8/11/20%, top-k 11%) and HunyuanVideo
+                 720p (10%, SIP and top-k) shaped workloads, per stage;
+  plan_reuse     score + SIP select once every --reuse steps, attention every step;
+  schedule50     the pages' deployment schedule: 50 sampler steps, the first 10 dense
+                 (the same kernel with every key block kept), then sparse with the plan
+                 refreshed every 4 steps;
+  dense_attn     the attention kernel with every key block kept;
+  units4         the pages' 4-token key units at the same tile budget;
+  e2e            the headline step through the public API with host buffers (pinned
+                 H2D of Q, K, V and D2H of O inside the timed region);
+  cpu_baseline   the CPU oracle on a bounded sample of the headline workload,
+                 extrapolated to a whole step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-For N > 1 run under torchrun: every rank runs the same workload on its own data (weak
-scaling, no data-path collective); the step time is the max over ranks.
+For N > 1 run under torchrun: every rank runs the headline workload on its own data
+(weak scaling over independent batches, no data-path collective); the step time is the
+max over ranks.
 """
 
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -43,6 +61,13 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 L2_BYTES = 126 * 2**20
+FLUSH_BYTES = 256 * 2**20
+METRIC = "sparse attn ms/call & dense-equiv TFLOPS on 1xB200; % tensor-pipe & HBM roofline"
+UNIT = "TFLOPS (dense-equivalent, whole step: score + SIP select + sparse attention)"
+HEADLINE = ("long", 0.10)
+# sources that decide the attention kernel's DRAM traffic (kernel, launch setup, maps)
+KERNEL_FILES = ("attn_kernel.cu", "ab_device.cuh", "tmap_host.h", "ab_api.cu", "ab_kernels.h")
+TRAFFIC_PROFILE = "attn_fwd_long.md"
 
 
 def kernel_source_hash(csrc: str) -> str:
@@ -51,7 +76,7 @@ def kernel_source_hash(csrc: str) -> str:
     import hashlib
     import re
     h = hashlib.sha256()
-    for f in ("attn_kernel.cu", "ab_device.cuh"):
+    for f in KERNEL_FILES:
         text = open(os.path.join(csrc, f), encoding="utf-8").read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)
@@ -60,16 +85,19 @@ def kernel_source_hash(csrc: str) -> str:
     return h.hexdigest()[:16]
 
 
-def attn_traffic_from_profile():
-    """DRAM bytes per attention launch recorded in profiles/attn_fwd_wan13b.md, or None
-    when the kernel source changed since that capture (hash mismatch)."""
-    path = os.path.join(ROOT, "profiles", "attn_fwd_wan13b.md")
-    csrc = os.path.join(ROOT, "block_sparse_attention_ab_b200", "csrc")
+def attn_traffic_from_profile(heads_full: int, path: str = None, csrc: str = None):
+    """DRAM bytes per headline attention launch from the ncu record in profiles/ (a
+    capture of fewer heads, scaled by heads_full / heads_captured: every head reads its
+    own Q, K, V and writes its own O), or None when the kernel sources changed since that
+    capture (hash mismatch) or there is no record."""
+    path = path or os.path.join(ROOT, "profiles", TRAFFIC_PROFILE)
+    csrc = csrc or os.path.join(ROOT, "block_sparse_attention_ab_b200", "csrc")
+    keys = ("traffic_bytes_per_launch", "kernel_source_sha256_16", "heads_captured")
     try:
-        rec = dict(line.split(":", 1) for line in open(path) if line.startswith(("traffic_bytes", "kernel_source")))
+        rec = dict(line.split(":", 1) for line in open(path) if line.startswith(keys))
         if kernel_source_hash(csrc) != rec["kernel_source_sha256_16"].strip():
             return None
-        return float(rec["traffic_bytes_per_launch"])
+        return float(rec["traffic_bytes_per_launch"]) * heads_full / int(rec["heads_captured"])
     except (OSError, KeyError, ValueError):
         return None
 
@@ -153,7 +181,6 @@ def workload(name: str):
 def rank_workload(name: str, rank: int, world: int, heads: int = 0):
     """The workload a rank runs: every rank gets the same shape on its own data (weak
     scaling over independent batches; the method has no cross-rank exchange)."""
-    import dataclasses
     w = workload(name)
     if heads:
         w = dataclasses.replace(w, H=heads)
@@ -179,54 +206,150 @@ def selected_flops(sum_cnt: int, d: int) -> float:
     return 4.0 * 128 * 128 * d * sum_cnt
 
 
+def score_bytes(w) -> float:
+    """Algorithmic HBM bytes of one scoring pass: read Q and K once, write the scores."""
+    return 2.0 * w.B * w.H * w.N_pad * w.d * 2 + 4.0 * w.B * w.H * w.n_blocks ** 2
+
+
+def stats(ts):
+    return {"median": round(statistics.median(ts), 4), "min": round(min(ts), 4),
+            "mean": round(float(np.mean(ts)), 4)}
+
+
+def tflops(flop, ms):
+    return round(flop / (ms * 1e-3) / 1e12, 2)
+
+
 # ------------------------------------------------------------------------ our arm ----
+
+class Runner:
+    """Device buffers and the three calls of the path for one workload."""
+
+    def __init__(self, ab, w, dev, keep_host=False):
+        from block_sparse_attention_ab_b200 import synth
+        self.ab, self.w, self.dev = ab, w, dev
+        q, k, v = synth.make_qkv(w)
+        if keep_host:
+            self.host = tuple(t.pin_memory() for t in (q, k, v))
+        self.q, self.k, self.v = (t.to(dev) for t in (q, k, v))
+        del q, k, v
+        B, H, N_pad, d = self.q.shape
+        nb = N_pad // 128
+        self.nb, self.d = nb, d
+        shape = ab.make_shape(self.q, w.N)
+        self.ws = torch.empty(ab.score_workspace_bytes(shape, w.n_clusters), device=dev, dtype=torch.uint8)
+        self.scores = torch.empty(B, H, nb, nb, device=dev, dtype=torch.float32)
+        self.idx = torch.empty(B, H, nb, nb, device=dev, dtype=torch.int32)
+        self.cnt = torch.empty(B, H, nb, device=dev, dtype=torch.int32)
+        self.wt = torch.empty(B, H, nb, nb, device=dev, dtype=torch.float32)
+        self.out = torch.empty_like(self.q)
+        self.flag = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def score(self):
+        w = self.w
+        self.ab.score(self.q, self.k, w.N, w.n_clusters, w.iters, workspace=self.ws, out=self.scores)
+
+    def select(self, K, mode, seed=None):
+        seed = self.w.sip_seed if seed is None else seed
+        self.ab.select(self.scores, K, mode, seed, dev_flag=self.flag,
+                       out=(self.idx, self.cnt, self.wt))
+
+    def attn(self, mode):
+        w, ab = self.w, self.ab
+        if mode == "sip":
+            ab.attn_fwd(self.q, self.k, self.v, w.N, self.idx, self.cnt, self.wt,
+                        dev_flag=self.flag, out=self.out)
+        else:
+            ab.attn_topk_fwd(self.q, self.k, self.v, w.N, self.idx, self.cnt,
+                             dev_flag=self.flag, out=self.out)
+
+    def check(self, what):
+        if self.ab.check_flag(self.flag) != 0:
+            raise RuntimeError(f"device flag raised during the benchmark ({what})")
+
+    def sum_cnt(self):
+        return int(self.cnt.sum().item())
+
+
+def ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+def time_calls(fn, calls, flush=None):
+    """Per-call CUDA-event times (ms) of `calls` calls of fn, each preceded by flush()
+    (outside the events) when given."""
+    pairs = [(ev(), ev()) for _ in range(calls)]
+    for a, b in pairs:
+        if flush is not None:
+            flush()
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in pairs]
+
+
+def case_measure(r, K, mode, calls, flush, cold=True, seed=None):
+    """Stage times of one (workload, mode, budget) case: scoring, selection, attention,
+    warm (back to back) and cold (L2 flushed before each call)."""
+    d = r.d
+    r.score()
+    r.select(K, mode, seed)
+    r.attn(mode)
+    torch.cuda.synchronize()
+    sc = time_calls(r.score, calls)
+    se = time_calls(lambda: r.select(K, mode, seed), calls)
+    at = time_calls(lambda: r.attn(mode), calls)
+    res = {"budget": K, "sum_cnt": r.sum_cnt(),
+           "score_ms": stats(sc), "select_ms": stats(se), "attn_ms": stats(at)}
+    if cold:
+        res["cold"] = {"score_ms": stats(time_calls(r.score, calls, flush)),
+                       "select_ms": stats(time_calls(lambda: r.select(K, mode, seed), calls, flush)),
+                       "attn_ms": stats(time_calls(lambda: r.attn(mode), calls, flush))}
+    r.check(f"{r.w.name} {mode} {K}")
+    a_ms = res["attn_ms"]["median"]
+    step = res["score_ms"]["median"] + res["select_ms"]["median"] + a_ms
+    res["step_ms"] = round(step, 4)
+    res["step_dense_equiv_tflops"] = tflops(dense_equiv_flops(r.w), step)
+    res["attn_selected_tflops"] = tflops(selected_flops(res["sum_cnt"], d), a_ms)
+    return res
+
 
 def run_ours(args, rank, world, local_rank):
     import block_sparse_attention_ab_b200 as ab
-    from block_sparse_attention_ab_b200 import build, synth
+    from block_sparse_attention_ab_b200 import build
 
     build.build()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    peaks = measured_peaks()
     w = rank_workload(args.config, rank, world, args.heads)
-    K = w.budget_blocks(w.budgets[0])
-    q, k, v = synth.make_qkv(w)
-    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
-    qc, kc, vc = (t.to(dev) for t in (q, k, v))
-    B, H, N_pad, d = qc.shape
-    nb = N_pad // 128
-    shape = ab.make_shape(qc, w.N)
-    ws = torch.empty(ab.score_workspace_bytes(shape, w.n_clusters), device=dev, dtype=torch.uint8)
-    scores = torch.empty(B, H, nb, nb, device=dev, dtype=torch.float32)
-    idx = torch.empty(B, H, nb, nb, device=dev, dtype=torch.int32)
-    cnt = torch.empty(B, H, nb, device=dev, dtype=torch.int32)
-    wt = torch.empty(B, H, nb, nb, device=dev, dtype=torch.float32)
-    out = torch.empty_like(qc)
-    flag = torch.zeros(1, dtype=torch.int32, device=dev)
+    frac = args.budget if args.budget is not None else (
+        HEADLINE[1] if args.config == HEADLINE[0] else w.budgets[0])
+    K = w.budget_blocks(frac)
+    r = Runner(ab, w, dev, keep_host=True)
+    q, d, nb = r.q, r.d, r.nb
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def ev():
-        return torch.cuda.Event(enable_timing=True)
-
-    def step(events=None, mode="sip"):
-        if events:
-            events[0].record()
-        ab.score(qc, kc, w.N, w.n_clusters, w.iters, workspace=ws, out=scores)
-        if events:
-            events[1].record()
-        ab.select(scores, K, mode, w.sip_seed, dev_flag=flag, out=(idx, cnt, wt))
-        if events:
-            events[2].record()
-        if mode == "sip":
-            ab.attn_fwd(qc, kc, vc, w.N, idx, cnt, wt, dev_flag=flag, out=out)
-        else:
-            ab.attn_topk_fwd(qc, kc, vc, w.N, idx, cnt, dev_flag=flag, out=out)
-        if events:
-            events[3].record()
+    def flush():
+        flush_buf.fill_(1)
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
+    def step(events=None, mode="sip"):
+        if events:
+            events[0].record()
+        r.score()
+        if events:
+            events[1].record()
+        r.select(K, mode)
+        if events:
+            events[2].record()
+        r.attn(mode)
+        if events:
+            events[3].record()
 
     def timed(mode):
         for _ in range(args.warmup):
@@ -247,23 +370,40 @@ def run_ours(args, rank, world, local_rank):
                            e[2].elapsed_time(e[3])] for e in per])
         return total, stage
 
+    # ---- headline: K timed steps, clocks sampled over them
     clocks = ClockSampler(local_rank)
     clocks.start()
     total_ms, stage_ms = timed("sip")
     clk = clocks.stop()
-    sum_cnt = int(cnt.sum().item())
-    if ab.check_flag(flag) != 0:
-        raise RuntimeError("device flag raised during the benchmark")
-    topk_total, topk_stage = timed("topk")
-    topk_cnt = int(cnt.sum().item())
+    sum_cnt = r.sum_cnt()
+    r.check("headline")
+    ms_step = max_over_ranks(total_ms / args.steps, world, dev)
+    attn_med = float(np.median(stage_ms[:, 2]))
+    attn_ms = max_over_ranks(attn_med, world, dev)
+    score_med = float(np.median(stage_ms[:, 0]))
+    dense = dense_equiv_flops(w)
+    sel = selected_flops(sum_cnt, d)
+    calls = max(3, min(args.steps, args.calls))
 
-    # plan reuse (the pages' deployment schedule): score + SIP select once every
-    # `reuse` steps, attention every step with the plan in force
+    # ---- top-k at the same budget, same protocol
+    topk_total, topk_stage = timed("topk")
+    topk_cnt = r.sum_cnt()
+    r.check("topk")
+    topk_ms = max_over_ranks(topk_total / args.steps, world, dev)
+
+    # ---- cold per-stage numbers of the headline (L2 flushed before each call)
+    r.select(K, "sip")
+    torch.cuda.synchronize()
+    cold = {"score_ms": stats(time_calls(r.score, calls, flush)),
+            "select_ms": stats(time_calls(lambda: r.select(K, "sip"), calls, flush)),
+            "attn_ms": stats(time_calls(lambda: r.attn("sip"), calls, flush))}
+
+    # ---- plan reuse and the pages' 50-step schedule
     def reuse_step(i):
         if i % args.reuse == 0:
-            ab.score(qc, kc, w.N, w.n_clusters, w.iters, workspace=ws, out=scores)
-            ab.select(scores, K, "sip", w.sip_seed + i // args.reuse, dev_flag=flag, out=(idx, cnt, wt))
-        ab.attn_fwd(qc, kc, vc, w.N, idx, cnt, wt, dev_flag=flag, out=out)
+            r.score()
+            r.select(K, "sip", w.sip_seed + i // args.reuse)
+        r.attn("sip")
 
     for i in range(args.warmup * args.reuse):
         reuse_step(i)
@@ -278,99 +418,33 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     reuse_ms = max_over_ranks(a.elapsed_time(b) / args.steps, world, dev)
 
-    # dense comparison: the same attention kernel with every key block kept (top-k at
-    # budget n_kb, all weights 1)
-    ab.select(scores, nb, "topk", out=(idx, cnt, wt))
-    dense_calls = max(3, args.steps // 30)
-    for _ in range(2):
-        ab.attn_topk_fwd(qc, kc, vc, w.N, idx, cnt, dev_flag=flag, out=out)
-    torch.cuda.synchronize()
-    barrier()
-    a, b = ev(), ev()
-    a.record()
-    for _ in range(dense_calls):
-        ab.attn_topk_fwd(qc, kc, vc, w.N, idx, cnt, dev_flag=flag, out=out)
-    b.record()
-    torch.cuda.synchronize()
-    barrier()
-    dense_ms = max_over_ranks(a.elapsed_time(b) / dense_calls, world, dev)
-    dense_pairs = int(cnt.sum().item())
-    if ab.check_flag(flag) != 0:
-        raise RuntimeError("device flag raised during the benchmark")
+    extras = {}
+    if not args.headline_only and world == 1:
+        extras["schedule50"] = schedule50(r, K, args)
+        extras["dense_attn"] = dense_attn(r, peaks, calls=max(1, min(3, args.steps)))
+        sweep = {}
+        for f in w.budgets:
+            Kf = w.budget_blocks(f)
+            sweep[f"{round(100 * f)}%"] = case_measure(r, Kf, "sip", calls, flush, cold=False)
+        extras["budget_sweep"] = sweep
 
-    # the page's 4-token key units at the same tile budget (32 units per 128-key tile):
-    # unit scores -> SIP over units -> attention over the gathered units
-    units = None
-    if N_pad // 4 <= 8192:
-        K4 = 32 * K
-        nku = N_pad // 4
-        ws4 = torch.empty(ab.score_workspace_bytes(shape, w.n_clusters, 4), device=dev, dtype=torch.uint8)
-        scores4 = torch.empty(B, H, nb, nku, device=dev, dtype=torch.float32)
-        idx4 = torch.empty(B, H, nb, nku, device=dev, dtype=torch.int32)
-        cnt4 = torch.empty(B, H, nb, device=dev, dtype=torch.int32)
-        wt4 = torch.empty(B, H, nb, nku, device=dev, dtype=torch.float32)
-
-        def unit_step(e=None):
-            if e:
-                e[0].record()
-            ab.score(qc, kc, w.N, w.n_clusters, w.iters, workspace=ws4, out=scores4, unit=4)
-            if e:
-                e[1].record()
-            ab.select(scores4, K4, "sip", w.sip_seed, dev_flag=flag, out=(idx4, cnt4, wt4))
-            if e:
-                e[2].record()
-            ab.attn_fwd(qc, kc, vc, w.N, idx4, cnt4, wt4, dev_flag=flag, out=out, unit=4)
-            if e:
-                e[3].record()
-
-        unit_iters = max(3, args.steps // 30)
-        for _ in range(2):
-            unit_step()
-        torch.cuda.synchronize()
-        barrier()
-        per4 = [[ev() for _ in range(4)] for _ in range(unit_iters)]
-        for i in range(unit_iters):
-            unit_step(per4[i])
-        torch.cuda.synchronize()
-        barrier()
-        st4 = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])]
-                        for e in per4])
-        tiles4 = int(((cnt4 + 31) // 32).sum().item())
-        attn4 = max_over_ranks(float(np.mean(st4[:, 2])), world, dev)
-        if ab.check_flag(flag) != 0:
-            raise RuntimeError("device flag raised during the unit benchmark")
-        units = {"unit_tokens": 4, "budget_units": K4, "tiles": tiles4,
-                 "kept_units": int(cnt4.sum().item()),
-                 "score_ms": round(float(np.mean(st4[:, 0])), 4),
-                 "select_ms": round(float(np.mean(st4[:, 1])), 4),
-                 "attn_ms": round(attn4, 4),
-                 "ms_per_step": round(max_over_ranks(float(np.mean(st4.sum(1))), world, dev), 4),
-                 "attn_tile_tflops": round(selected_flops(tiles4, d) / (attn4 * 1e-3) / 1e12, 2),
-                 "note": "SIP over 4-token key units, gathered 32 per 128-key tile"}
-
-    ms_step = max_over_ranks(total_ms / args.steps, world, dev)
-    attn_ms = float(np.mean(stage_ms[:, 2]))
-    dense = dense_equiv_flops(w)
-    sel = selected_flops(sum_cnt, d)
-    peaks = measured_peaks()
-
-    # end to end through the public API with host buffers: pinned H2D of Q, K, V,
-    # the whole path, D2H of the output; all inside the timed region
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    # ---- end to end through the public API with host buffers
+    qh, kh, vh = r.host
+    out_h = torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory()
 
     def e2e_step():
         qd = qh.to(dev, non_blocking=True)
         kd = kh.to(dev, non_blocking=True)
         vd = vh.to(dev, non_blocking=True)
-        s = ab.score(qd, kd, w.N, w.n_clusters, w.iters, workspace=ws, out=scores)
-        ab.select(s, K, "sip", w.sip_seed, out=(idx, cnt, wt))
-        o = ab.attn_fwd(qd, kd, vd, w.N, idx, cnt, wt, out=out)
+        s = ab.score(qd, kd, w.N, w.n_clusters, w.iters, workspace=r.ws, out=r.scores)
+        ab.select(s, K, "sip", w.sip_seed, out=(r.idx, r.cnt, r.wt))
+        o = ab.attn_fwd(qd, kd, vd, w.N, r.idx, r.cnt, r.wt, out=r.out)
         out_h.copy_(o, non_blocking=True)
 
-    for _ in range(max(1, args.warmup)):
+    for _ in range(max(1, min(args.warmup, 3))):
         e2e_step()
     torch.cuda.synchronize()
-    e2e_steps = max(1, min(args.steps, 10))
+    e2e_steps = max(1, min(args.steps, 5))
     barrier()
     a, b = ev(), ev()
     a.record()
@@ -382,11 +456,16 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world, dev)
     h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
     d2h = out_h.numel() * out_h.element_size()
+    del out_h
 
+    traffic = args.traffic if args.traffic is not None else (
+        attn_traffic_from_profile(w.B * w.H) if (w.name == HEADLINE[0] and K == w.budget_blocks(HEADLINE[1])) else None)
+    achieved = sel / (attn_ms * 1e-3) / 1e12
+    sbytes = score_bytes(w)
     res = {
-        "metric": "sparse attn ms/call & dense-equiv TFLOPS on 1xB200; % tensor-pipe & HBM roofline",
+        "metric": METRIC,
         "value": round(world * dense / (ms_step * 1e-3) / 1e12, 2),
-        "unit": "TFLOPS (dense-equivalent, whole step: score + SIP select + sparse attention)",
+        "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -395,130 +474,316 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded generator shaped like Wan2.1-1.3B 480p attention; no weights or prompts)",
+        "data": f"synthetic (seeded generator shaped like {w.name} video-DiT attention; no weights or prompts)",
         "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} (N_pad={w.N_pad}) d={w.d}, "
-                               f"budget {K}/{nb} key blocks, C={w.n_clusters}, T={w.iters}",
+                               f"SIP budget {K}/{nb} key blocks ({round(100 * frac)}%), "
+                               f"C={w.n_clusters}, T={w.iters}",
                    "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world}",
-                   "l2": f"inputs Q+K+V = {3 * q.numel() * 2 / 1e6:.0f} MB > 126 MB L2 (no flush)"},
-        "attn_ms_per_call": round(max_over_ranks(attn_ms, world, dev), 4),
-        "attn_dense_equiv_tflops": round(dense / (attn_ms * 1e-3) / 1e12, 2),
-        "attn_selected_tflops": round(sel / (attn_ms * 1e-3) / 1e12, 2),
-        "stage_ms": {"score": round(float(np.mean(stage_ms[:, 0])), 4),
-                     "select_sip": round(float(np.mean(stage_ms[:, 1])), 4),
-                     "attn_sip": round(attn_ms, 4)},
+                   "l2": f"inputs Q+K+V = {3 * q.numel() * 2 / 1e9:.2f} GB > 126 MB L2 (no flush "
+                         f"in the timed steps; 'cold' stage numbers flush a 256 MB buffer before each call)"},
+        "attn_ms_per_call": round(attn_ms, 4),
+        "attn_dense_equiv_tflops": tflops(dense, attn_ms),
+        "attn_selected_tflops": round(achieved, 2),
+        "stage_ms": {"score": stats(list(stage_ms[:, 0])), "select_sip": stats(list(stage_ms[:, 1])),
+                     "attn_sip": stats(list(stage_ms[:, 2]))},
+        "stage_ms_cold": cold,
         "sum_cnt": sum_cnt,
-        "topk": {"ms_per_step": round(topk_total / args.steps, 4),
-                 "attn_ms_per_call": round(float(np.mean(topk_stage[:, 2])), 4),
-                 "select_ms": round(float(np.mean(topk_stage[:, 1])), 4),
-                 "attn_selected_tflops": round(selected_flops(topk_cnt, d) /
-                                               (float(np.mean(topk_stage[:, 2])) * 1e-3) / 1e12, 2),
+        "topk": {"ms_per_step": round(topk_ms, 4),
+                 "value": round(world * dense / (topk_ms * 1e-3) / 1e12, 2),
+                 "attn_ms": stats(list(topk_stage[:, 2])),
+                 "select_ms": stats(list(topk_stage[:, 1])),
+                 "attn_selected_tflops": tflops(selected_flops(topk_cnt, d),
+                                                float(np.median(topk_stage[:, 2]))),
                  "sum_cnt": topk_cnt},
         "roofline": {"bound": "tensor",
                      "kernel": "attn_fwd_kernel<128, weighted, bf16 out>",
-                     "achieved": round(sel / (attn_ms * 1e-3) / 1e12, 2),
+                     "achieved": round(achieved, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(sel / (attn_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} bf16 dense burst",
-                     "traffic": args.traffic if args.traffic is not None else attn_traffic_from_profile(),
-                     "algorithmic_bytes": 4 * q.numel() * 2},
-        "score_roofline": {"bound": "hbm",
-                           "achieved": round((2 * q.numel() * 2 + scores.numel() * 4) /
-                                             (float(np.mean(stage_ms[:, 0])) * 1e-3) / 1e9, 1),
+                     "traffic": traffic,
+                     "algorithmic_bytes": 4 * q.numel() * 2,
+                     "per_launch": f"4*128*128*d FLOP x sum_cnt = {sel / 1e12:.2f} TFLOP; median of "
+                                   f"{args.steps} CUDA-event timed launches"},
+        "score_roofline": {"bound": "hbm", "bytes": sbytes,
+                           "achieved": round(sbytes / (score_med * 1e-3) / 1e9, 1),
                            "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": round((2 * q.numel() * 2 + scores.numel() * 4) /
-                                         (float(np.mean(stage_ms[:, 0])) * 1e-3) / 1e9 /
-                                         peaks["hbm_gbs"], 4)},
+                           "frac": round(sbytes / (score_med * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
         "plan_reuse": {"every": args.reuse,
                        "ms_per_step": round(reuse_ms, 4),
                        "value": round(world * dense / (reuse_ms * 1e-3) / 1e12, 2),
                        "unit": "TFLOPS (dense-equivalent)",
                        "schedule": f"score + SIP select once per {args.reuse} steps, attention every step"},
-        "units4": units,
-        "dense_attn": {"ms_per_call": round(dense_ms, 4), "sum_cnt": dense_pairs,
-                       "tflops": round(selected_flops(dense_pairs, d) / (dense_ms * 1e-3) / 1e12, 2),
-                       "frac": round(selected_flops(dense_pairs, d) / (dense_ms * 1e-3) / 1e12 /
-                                     peaks["bf16_tflops"], 4),
-                       "note": "same kernel, every key block kept (budget n_kb, weights 1)"},
+        **extras,
         "e2e": {"value": round(world * dense / (e2e_ms * 1e-3) / 1e12, 2),
-                "unit": "TFLOPS (dense-equivalent, host buffers in and out)",
+                "unit": UNIT,
+                "what": "public API with host buffers: pinned H2D of Q, K, V, the whole path, D2H of O",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": 5 * args.steps,
         "clocks": clk,
     }
+    del r, flush_buf
+    torch.cuda.empty_cache()
+    if not args.headline_only and world == 1:
+        res["workloads"] = other_workloads(ab, dev, args, peaks, calls)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, q, k, v, K, seconds=args.cpu_seconds)
+        res["cpu_baseline"] = cpu_baseline(w, K, seconds=args.cpu_seconds)
     return res
+
+
+def schedule50(r, K, args, steps=50, dense_steps=10, every=4):
+    """The pages' deployment schedule over one 50-step sampling run: the first 10 steps
+    attend densely (the same kernel, every key block kept), the rest run the sparse path
+    with score + SIP select every `every` steps and attention every step. Reported: the
+    per-step average, beside dense-only and sparse-only per-step times from the same run."""
+    r.select(r.nb, "topk")  # every block kept: the plan of the dense steps
+    ts = []
+    for i in range(steps):
+        a, b = ev(), ev()
+        a.record()
+        if i < dense_steps:
+            r.attn("topk")
+        else:
+            j = i - dense_steps
+            if j % every == 0:
+                r.score()
+                r.select(K, "sip", r.w.sip_seed + j // every)
+            r.attn("sip")
+        b.record()
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    t = [a.elapsed_time(b) for a, b in ts]
+    r.check("schedule50")
+    total = sum(t)
+    dense_ms = statistics.median(t[:dense_steps])
+    sparse = t[dense_steps:]
+    dense_equiv = dense_equiv_flops(r.w)
+    return {"steps": steps, "dense_steps": dense_steps, "plan_every": every,
+            "ms_per_step": round(total / steps, 4),
+            "value": tflops(dense_equiv, total / steps),
+            "dense_step_ms": round(dense_ms, 4),
+            "sparse_step_ms_mean": round(float(np.mean(sparse)), 4),
+            "speedup_vs_dense": round(dense_ms * steps / total, 3),
+            "note": "first transformer block dense on the pages: a model-level factor, not modelled"}
+
+
+def dense_attn(r, peaks, calls):
+    """The attention kernel with every key block kept (top-k at budget n_kb, weights 1)."""
+    r.select(r.nb, "topk")
+    r.attn("topk")
+    torch.cuda.synchronize()
+    t = time_calls(lambda: r.attn("topk"), calls)
+    r.check("dense")
+    pairs = r.sum_cnt()
+    ms = statistics.median(t)
+    tf = selected_flops(pairs, r.d) / (ms * 1e-3) / 1e12
+    return {"ms_per_call": round(ms, 4), "sum_cnt": pairs, "tflops": round(tf, 2),
+            "frac": round(tf / peaks["bf16_tflops"], 4),
+            "note": "same kernel, every key block kept (budget n_kb, weights 1)"}
+
+
+def units4(r, K, calls):
+    """The pages' 4-token key units at the same tile budget (32 units per 128-key tile):
+    unit scores -> SIP over units -> attention over the gathered units."""
+    ab, w, dev = r.ab, r.w, r.dev
+    B, H, N_pad, d = r.q.shape
+    nb, nku = r.nb, N_pad // 4
+    K4 = 32 * K
+    shape = ab.make_shape(r.q, w.N)
+    ws4 = torch.empty(ab.score_workspace_bytes(shape, w.n_clusters, 4), device=dev, dtype=torch.uint8)
+    scores4 = torch.empty(B, H, nb, nku, device=dev, dtype=torch.float32)
+    idx4 = torch.empty(B, H, nb, nku, device=dev, dtype=torch.int32)
+    cnt4 = torch.empty(B, H, nb, device=dev, dtype=torch.int32)
+    wt4 = torch.empty(B, H, nb, nku, device=dev, dtype=torch.float32)
+
+    def sc():
+        ab.score(r.q, r.k, w.N, w.n_clusters, w.iters, workspace=ws4, out=scores4, unit=4)
+
+    def se():
+        ab.select(scores4, K4, "sip", w.sip_seed, dev_flag=r.flag, out=(idx4, cnt4, wt4))
+
+    def at():
+        ab.attn_fwd(r.q, r.k, r.v, w.N, idx4, cnt4, wt4, dev_flag=r.flag, out=r.out, unit=4)
+
+    sc()
+    se()
+    at()
+    torch.cuda.synchronize()
+    t_sc, t_se, t_at = (stats(time_calls(f, calls)) for f in (sc, se, at))
+    r.check("units4")
+    tiles = int(((cnt4 + 31) // 32).sum().item())
+    step = t_sc["median"] + t_se["median"] + t_at["median"]
+    return {"unit_tokens": 4, "budget_units": K4, "tiles": tiles,
+            "kept_units": int(cnt4.sum().item()),
+            "score_ms": t_sc, "select_ms": t_se, "attn_ms": t_at,
+            "ms_per_step": round(step, 4),
+            "attn_tile_tflops": tflops(selected_flops(tiles, d), t_at["median"]),
+            "note": "SIP over 4-token key units, gathered 32 per 128-key tile"}
+
+
+def other_workloads(ab, dev, args, peaks, calls):
+    """Per-stage numbers of the other named workloads (each case warm and cold)."""
+    flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    out = {}
+    for name in ("hunyuan720", "wan14b", "wan13b"):
+        w = workload(name)
+        r = Runner(ab, w, dev)
+        rec = {"shape": f"B={w.B} H={w.H} N={w.N} (N_pad={w.N_pad}) d={w.d}"}
+        for f in w.budgets:
+            K = w.budget_blocks(f)
+            rec[f"sip_{round(100 * f)}%"] = case_measure(r, K, "sip", calls, flush)
+        Kt = w.budget_blocks(w.topk_budget)
+        rec[f"topk_{round(100 * w.topk_budget)}%"] = case_measure(r, Kt, "topk", calls, flush)
+        s0 = rec[f"sip_{round(100 * w.budgets[0])}%"]
+        sbytes = score_bytes(w)
+        rec["score_roofline"] = {"bound": "hbm", "bytes": sbytes,
+                                 "achieved": round(sbytes / (s0["score_ms"]["median"] * 1e-3) / 1e9, 1),
+                                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                 "frac": round(sbytes / (s0["score_ms"]["median"] * 1e-3) / 1e9 /
+                                               peaks["hbm_gbs"], 4)}
+        a_tf = s0["attn_selected_tflops"]
+        rec["attn_roofline"] = {"bound": "tensor", "achieved": a_tf, "peak": peaks["bf16_tflops"],
+                                "unit": "TFLOP/s", "frac": round(a_tf / peaks["bf16_tflops"], 4)}
+        if name in ("wan13b", "hunyuan720"):
+            rec["dense_attn"] = dense_attn(r, peaks, calls=max(1, min(3, calls)))
+        if w.N_pad // 4 <= ab.MAX_UNITS:
+            try:
+                rec["units4"] = units4(r, w.budget_blocks(w.budgets[0]), calls)
+            except ab.AbError as e:  # the library rejects the size: report it
+                rec["units4"] = {"unavailable": str(e)}
+        out[name] = rec
+        del r
+        torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------- CPU oracle leg ----
 
-def cpu_baseline(w, q, k, v, K, seconds: float = 15.0, max_heads: int = 0):
-    """Time the oracle, as it stands, on a bounded sample of the same workload: whole
-    heads (IBCS scoring, SIP selection and the attention of every query block), one head
-    at a time until `seconds` have been spent; scaled to all B*H heads of one step."""
+_HEAD_CACHE = {}
+
+
+def _head_data(w, h):
+    from block_sparse_attention_ab_b200 import synth
+    key = (w.name, w.data_seed, h)
+    if key not in _HEAD_CACHE:
+        _HEAD_CACHE.clear()
+        _HEAD_CACHE[key] = synth.make_qkv(w, heads=[h])
+    return _HEAD_CACHE[key]
+
+
+def _oracle_sample(w, K, n_items, seed, heads=(0,)):
+    """Time the oracle, as it stands, on `n_items` (head, query block) items of workload w
+    drawn from `heads`: per head its mean keys; per item the k-means of its query block,
+    its score row, its SIP row and its attention. Returns (seconds per head of mean keys,
+    seconds per item, threads used, detail)."""
     import oracle
 
-    t_heads = []
-    detail = None
-    for h in range(w.H):
-        qs, ks, vs = q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1]
+    rng = np.random.default_rng(seed)
+    nb = w.n_blocks
+    t_mk, t_item, n_done = 0.0, 0.0, 0
+    parts = np.zeros(4)
+    for h in heads:
+        q, k, v = _head_data(w, h)
         t0 = time.perf_counter()
-        cent, wts, _, _, _ = oracle.kmeans(qs, w.N, w.n_clusters, w.iters)
-        s = oracle.score(cent, wts, oracle.mean_key(ks, w.N))
-        t1 = time.perf_counter()
-        idx, cnt, wt, _, _ = oracle.sip(s.astype(np.float32), K, w.sip_seed, with_p=False)
-        t2 = time.perf_counter()
-        oracle.attn_rows(qs, ks, vs, w.N, idx, cnt, wt)
-        t3 = time.perf_counter()
-        t_heads.append(t3 - t0)
-        detail = (t1 - t0, t2 - t1, t3 - t2)
-        if sum(t_heads) >= seconds or (max_heads and len(t_heads) >= max_heads):
-            break
-    per_head = sum(t_heads) / len(t_heads)
-    step_s = w.B * w.H * per_head
+        kbar = oracle.mean_key(k, w.N)
+        t_mk += time.perf_counter() - t0
+        qbs = rng.choice(nb, size=max(1, n_items // len(heads)), replace=False)
+        t0 = time.perf_counter()
+        rows = []
+        idx = np.full((1, 1, nb, nb), -1, dtype=np.int32)
+        cnt = np.zeros((1, 1, nb), dtype=np.int32)
+        wt = np.zeros((1, 1, nb, nb), dtype=np.float32)
+        for qb in qbs:
+            nv = min(128, w.N - qb * 128)
+            qblk = torch.zeros(1, 1, 128, w.d, dtype=q.dtype)
+            qblk[0, 0, :nv] = q[0, 0, qb * 128: qb * 128 + nv]
+            t1 = time.perf_counter()
+            cent, wts, _, _, _ = oracle.kmeans(qblk, nv, w.n_clusters, w.iters)
+            s = oracle.score(cent, wts, kbar)
+            t2 = time.perf_counter()
+            i_, c_, w_, _, _ = oracle.sip(s.astype(np.float32), K, w.sip_seed, with_p=False)
+            t3 = time.perf_counter()
+            idx[0, 0, qb], cnt[0, 0, qb], wt[0, 0, qb] = i_[0, 0, 0], c_[0, 0, 0], w_[0, 0, 0]
+            rows.append(int(qb))
+            parts[0] += t2 - t1
+            parts[1] += t3 - t2
+        t4 = time.perf_counter()
+        oracle.attn_rows(q, k, v, w.N, idx, cnt, wt, rows=np.array(rows, dtype=np.int64))
+        t5 = time.perf_counter()
+        parts[2] += t5 - t4
+        t_item += t5 - t0
+        n_done += len(rows)
+    detail = (f"k-means+score {parts[0] / n_done * 1e3:.1f} ms, SIP {parts[1] / n_done * 1e3:.2f} ms, "
+              f"attention {parts[2] / n_done * 1e3:.1f} ms per item (attention of the items in one "
+              f"call, one OpenMP thread per item)")
+    threads = min(oracle.num_threads(), max(1, n_items // len(heads)))
+    return t_mk / len(heads), t_item / n_done, threads, detail, n_done
+
+
+def cpu_baseline(w, K, seconds: float = 15.0, n_items: int = 64):
+    """The oracle as it stands on a bounded sample of the workload: the mean keys of one
+    head and `n_items` (head 0, query block) items (k-means, score row, SIP row,
+    attention), extrapolated to all B*H heads and B*H*n_qb items of one step. The SIP draw
+    of a sampled item uses counter (j, 0, 0, 0) (the item scored alone), a different but
+    equally distributed draw."""
+    t_mk, t_item, threads, detail, n = _oracle_sample(w, K, n_items, seed=12345)
+    items = w.B * w.H * w.n_blocks
+    step_s = w.B * w.H * t_mk + items * t_item
     return {"value": round(dense_equiv_flops(w) / step_s / 1e12, 6),
             "unit": "TFLOPS (dense-equivalent, whole step)",
-            "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": (f"{len(t_heads)} of {w.B * w.H} (batch, head) slices of the workload, each "
-                       f"complete: scoring {detail[0]:.2f} s, SIP {detail[1]:.3f} s, attention of "
-                       f"all {w.n_blocks} query blocks {detail[2]:.2f} s (last slice); "
-                       f"{sum(t_heads):.1f} s of CPU time, scaled by {w.B * w.H}/{len(t_heads)}"),
+            "cores": threads, "kind": "oracle", "extrapolated": True,
+            "sample": (f"{n} of {items} (head, query block) items of {w.name} at {K}/{w.n_blocks} "
+                       f"blocks plus the mean keys of 1 of {w.B * w.H} heads, extrapolated to one "
+                       f"whole step: {detail}"),
             "est_step_s": round(step_s, 2)}
 
 
 def run_reference(args, rank, world):
-    """Reference arm: the CPU oracle on the same workload and metric, each step a bounded
-    sample scaled to one whole step."""
+    """Reference arm: the CPU oracle on the same workload and metric. Each step times a
+    bounded sample (the mean keys of one head and a batch of items), extrapolated to one
+    whole step; the line says so."""
     if rank != 0:
         return None
     w = workload(args.config)
-    from block_sparse_attention_ab_b200 import synth
-    q, k, v = synth.make_qkv(w, heads=[0])
-    K = w.budget_blocks(w.budgets[0])
-    # each step: one complete (batch, head) slice, scaled to the whole step
-    for _ in range(args.warmup):
-        cpu_baseline(w, q, k, v, K, seconds=0.0, max_heads=1)
-    vals = []
-    last = None
-    for _ in range(args.steps):
-        last = cpu_baseline(w, q, k, v, K, seconds=0.0, max_heads=1)
-        vals.append(last["est_step_s"])
+    frac = args.budget if args.budget is not None else (
+        HEADLINE[1] if args.config == HEADLINE[0] else w.budgets[0])
+    K = w.budget_blocks(frac)
+    per_step = 16
+    for i in range(args.warmup):
+        _oracle_sample(w, K, 4, seed=1000 + i)
+    vals, last = [], None
+    for i in range(args.steps):
+        t_mk, t_item, threads, detail, n = _oracle_sample(w, K, per_step, seed=i)
+        step_s = w.B * w.H * t_mk + w.B * w.H * w.n_blocks * t_item
+        vals.append(step_s)
+        last = (threads, detail, n)
     ms = statistics.median(vals) * 1e3
     value = dense_equiv_flops(w) / (ms * 1e-3) / 1e12
+    sample = (f"each step: mean keys of 1 of {w.B * w.H} heads and {last[2]} of "
+              f"{w.B * w.H * w.n_blocks} (head, query block) items, extrapolated to one whole "
+              f"step ({last[1]})")
     return {
         "impl": "reference",
-        "metric": "sparse attn ms/call & dense-equiv TFLOPS on 1xB200; % tensor-pipe & HBM roofline",
+        "metric": METRIC,
         "value": round(value, 6),
-        "unit": "TFLOPS (dense-equivalent, whole step: score + SIP select + sparse attention)",
+        "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": round(ms, 2),
+        "timing": "extrapolated from a bounded sample per step (not a measured whole step)",
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} budget {K}/{w.n_blocks}",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} (N_pad={w.N_pad}) d={w.d}, "
+                               f"SIP budget {K}/{w.n_blocks} key blocks ({round(100 * frac)}%), "
+                               f"C={w.n_clusters}, T={w.iters}",
                    "global_batch": w.B, "seq_len": w.N, "parallelism": "dp1"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS (dense-equivalent, whole step)",
-                         "cores": last["cores"], "kind": "oracle", "sample": last["sample"]},
-        "e2e": {"value": round(value, 6), "unit": "TFLOPS (dense-equivalent, whole step)",
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": last[0],
+                         "kind": "oracle", "extrapolated": True, "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": UNIT,
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -526,13 +791,19 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="wan13b")
+    ap.add_argument("--config", default=HEADLINE[0])
+    ap.add_argument("--budget", type=float, default=None,
+                    help="SIP budget as a fraction of the key blocks (default: 10%% for long, "
+                         "else the workload's first budget)")
     ap.add_argument("--heads", type=int, default=0, help="override head count (profiling)")
+    ap.add_argument("--calls", type=int, default=10, help="per-call samples of the extra cases")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the extra cases and workloads (profiling runs)")
     ap.add_argument("--reuse", type=int, default=4,
                     help="plan reuse period for the amortised-step measurement")
     ap.add_argument("--traffic", type=float, default=None,

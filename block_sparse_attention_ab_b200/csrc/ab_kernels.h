@@ -63,5 +63,8 @@ struct AttnLaunch {
     int grid_override;  // > 0: number of CTAs (tests); 0: one per SM
 };
 cudaError_t launch_attn(const AttnLaunch &a, cudaStream_t st);
+// Tests: the next attention launch uses claim slot `slot` (0..4095) instead of the next
+// slot in turn.
+void force_next_counter_slot(int slot);
 
 }  // namespace ab

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <mutex>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "../../include/ab_attn.h"
 #include "ab_kernels.h"
@@ -25,24 +26,29 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Device address of g_scratch on the current device. In host code the symbol is only a
 // host-side stand-in, so the address is looked up once per device (with that device
 // current) and cached.
+// A failed lookup keeps its CUDA error for ab_last_cuda_error; a device ordinal past the
+// cache (more than kMaxDevices GPUs) is AB_ERR_RANGE.
 ab_status scratch_on_current_device(void **out)
 {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AB_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return ab::status_of(e);
+    if (dev < 0 || dev >= kMaxDevices) return AB_ERR_RANGE;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
     if (!g_scratch_addr[dev]) {
         void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_scratch) != cudaSuccess || !ptr) return AB_ERR_CUDA;
+        e = cudaGetSymbolAddress(&ptr, g_scratch);
+        if (e != cudaSuccess) return ab::status_of(e);
+        if (!ptr) return ab::status_of(cudaErrorInvalidSymbol);
         g_scratch_addr[dev] = ptr;
     }
     *out = g_scratch_addr[dev];
     return AB_OK;
 }
 
-}  // namespace
-
-extern "C" ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, int n_clusters,
-                                      int iters, float *scores, int *dev_flag, void *stream)
+// The body of ab_score_noalloc.
+ab_status score_noalloc(const void *q, const void *k, ab_shape s, int n_clusters, int iters,
+                        float *scores, int *dev_flag, void *stream)
 {
     if (!q || !k || !scores) return AB_ERR_NULL;
     if (s.B <= 0 || s.H <= 0 || s.N <= 0 || s.N_pad <= 0 || s.d <= 0) return AB_ERR_SHAPE;
@@ -78,4 +84,15 @@ extern "C" ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, 
     if (e == cudaSuccess)
         e = ab::launch_score(ce, cw, kt, scores, BH, nb, nb, nb, s.d, n_clusters, dev_flag, cs);
     return ab::status_of(e);
+}
+
+}  // namespace
+
+extern "C" ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, int n_clusters,
+                                      int iters, float *scores, int *dev_flag, void *stream)
+{
+    nvtxRangePushA("ab_score_noalloc");
+    const ab_status st = score_noalloc(q, k, s, n_clusters, iters, scores, dev_flag, stream);
+    nvtxRangePop();
+    return st;
 }

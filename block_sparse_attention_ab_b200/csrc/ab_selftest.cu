@@ -1,5 +1,7 @@
-// ab_selftest.cu -- ab_selftest_bounded_wait: exercises the bounded mbarrier wait that
-// every pipeline of the library relies on, without a GPU fault (see include/ab_attn.h).
+// ab_selftest.cu -- test entry points (see include/ab_attn.h): ab_selftest_bounded_wait
+// exercises the bounded mbarrier wait that every pipeline of the library relies on,
+// without a GPU fault; ab_selftest_force_counter_slot steers the next attention call
+// onto a chosen claim slot.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -39,4 +41,11 @@ extern "C" ab_status ab_selftest_bounded_wait(int limit_us, int complete, int *d
     bounded_wait_kernel<<<1, 64, 0, (cudaStream_t)stream>>>(
         dev_flag, dev_done, (uint64_t)limit_us * 1000ull, complete ? 1 : 0);
     return ab::status_of(cudaGetLastError());
+}
+
+extern "C" ab_status ab_selftest_force_counter_slot(int slot)
+{
+    if (slot < 0 || slot >= 4096) return AB_ERR_RANGE;
+    ab::force_next_counter_slot(slot);
+    return AB_OK;
 }

@@ -79,9 +79,35 @@ struct AttnParams {
     int per_tile;  // selected entries per 128-key tile: 1 (blocks) or 32 (units)
     int n_items;
     float scale_log2;       // log2(e) / sqrt(d)
-    unsigned int *counter;  // [2]: items claimed, CTAs finished (zero at launch; the last
-                            // CTA to finish sets both back to zero)
+    unsigned int *counter;  // claim slot [4]: items claimed, owner tag (zeroed on the
+                            // launch's stream just before the kernel)
+    unsigned int tag;       // this launch's owner tag (never 0 or kSlotPoison)
 };
+
+// A claim slot is zeroed on the launch's stream right before the kernel; the first CTA
+// to arrive writes the launch's tag into it. A CTA that finds another tag (or, at a
+// claim or at its exit, a slot that no longer carries its tag) knows that a second
+// launch is using the same slot at the same time: it raises AB_FLAG_SCHED_COLLISION and
+// poisons the slot, so that the other launch finds out too.
+constexpr unsigned kSlotPoison = 0xFFFFFFFFu;
+
+__device__ __forceinline__ void slot_collision(const AttnParams &p)
+{
+    raise_flag(p.flag, AB_FLAG_SCHED_COLLISION);
+    atomicExch(p.counter + 1, kSlotPoison);
+}
+
+__device__ __forceinline__ void slot_join(const AttnParams &p)
+{
+    const unsigned old = atomicCAS(p.counter + 1, 0u, p.tag);
+    if (old != 0u && old != p.tag) slot_collision(p);
+}
+
+__device__ __forceinline__ void slot_check(const AttnParams &p)
+{
+    __threadfence();
+    if (atomicOr(p.counter + 1, 0u) != p.tag) slot_collision(p);
+}
 
 // 4-token key units: one 16-byte cp.async per lane (zero fill when src_bytes == 0) and
 // an arrive on an mbarrier when this thread's earlier cp.async copies have landed.
@@ -541,9 +567,13 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         // and are not published. Its waits sleep between polls: it shares an SM
         // sub-partition with two softmax warps.
         bool ok = true;
+        if (lane == 0) slot_join(p);
         auto claim = [&]() -> int {
             int c = 0;
-            if (lane == 0) c = (int)min(atomicAdd(p.counter, 1u), (unsigned)p.n_items);
+            if (lane == 0) {
+                c = (int)min(atomicAdd(p.counter, 1u), (unsigned)p.n_items);
+                slot_check(p);
+            }
             c = __shfl_sync(0xffffffffu, c, 0);
             return min((int)gridDim.x + c, p.n_items);
         };
@@ -940,16 +970,8 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    if (threadIdx.x == 0) {
-        // the last CTA to finish (all claims are made) returns the counter to zero for
-        // the next launch that uses it
-        __threadfence();
-        if (atomicAdd(p.counter + 1, 1u) == gridDim.x - 1) {
-            p.counter[0] = 0;
-            p.counter[1] = 0;
-            __threadfence();
-        }
-    }
+    // every claim of this CTA is made: the slot must still carry this launch's tag
+    if (threadIdx.x == 0) slot_check(p);
 }
 
 // ---------------------------------------------------------------------------------
@@ -963,22 +985,29 @@ static bool make_tmap(CUtensorMap *tm, const void *base, int BH, int N, int N_pa
                              (uint64_t)N_pad * d * 2, 64, 128);
 }
 
-// Claim counters of the item scheduler, one pair per launch slot: a launch takes the next
-// slot in turn and its last CTA leaves the pair at zero, so launches on one stream reuse a
-// slot safely and up to kCounterSlots launches can run at once on different streams.
+// Claim slots of the item scheduler (16 bytes each: items claimed, owner tag, two unused
+// words). A launch takes the next slot in turn, zeroes it on its own stream just before
+// the kernel and tags it with its launch number; launches that share a slot while both
+// run are detected (slot_join / slot_check).
 constexpr unsigned kCounterSlots = 4096;
-__device__ unsigned int g_item_counters[kCounterSlots][2];
-static std::atomic<unsigned> g_counter_next{0};
+__device__ unsigned int g_item_counters[kCounterSlots][4];
+static std::atomic<unsigned long long> g_counter_next{0};
+static std::atomic<int> g_forced_slot{-1};
 
-static cudaError_t counter_slot(unsigned int **slot)
+static cudaError_t counter_slot(cudaStream_t st, unsigned int **slot, unsigned *tag)
 {
     void *base = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&base, g_item_counters);
+    cudaError_t e = cudaGetSymbolAddress(&base, g_item_counters);
     if (e != cudaSuccess) return e;
-    const unsigned k = g_counter_next.fetch_add(1, std::memory_order_relaxed) % kCounterSlots;
-    *slot = static_cast<unsigned int *>(base) + 2 * k;
-    return cudaSuccess;
+    const unsigned long long gen = g_counter_next.fetch_add(1, std::memory_order_relaxed);
+    const int forced = g_forced_slot.exchange(-1);
+    const unsigned k = forced >= 0 ? (unsigned)forced : (unsigned)(gen % kCounterSlots);
+    *slot = static_cast<unsigned int *>(base) + 4 * k;
+    *tag = 1u + (unsigned)(gen % 0xFFFFFFFEull);  // 1 .. 0xFFFFFFFE: never 0 or kSlotPoison
+    return cudaMemsetAsync(*slot, 0, 4 * sizeof(unsigned int), st);
 }
+
+void force_next_counter_slot(int slot) { g_forced_slot.store(slot % (int)kCounterSlots); }
 
 template <int D, bool W, bool F32, bool U4>
 static cudaError_t launch_attn_t(const AttnLaunch &a, cudaStream_t st)
@@ -1005,7 +1034,7 @@ static cudaError_t launch_attn_t(const AttnLaunch &a, cudaStream_t st)
     p.per_tile = U4 ? 32 : 1;
     p.n_items = a.B * a.H * p.nqb;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
-    cudaError_t e = counter_slot(&p.counter);
+    cudaError_t e = counter_slot(st, &p.counter, &p.tag);
     if (e != cudaSuccess) return e;
     const int smem = AttnSmem<D>::kAlloc;
     e = cudaFuncSetAttribute(attn_fwd_kernel<D, W, F32, U4>,

@@ -3,7 +3,8 @@
 // SIP (AB-Attention news page, section «Три приёма AB-Attention», second technique):
 // inclusion probability p_j = min(1, c s_j) with sum p_j = K, the top blocks always
 // kept, each kept block weighted by 1/p_j. Solved exactly in integers on the fixed
-// point u_j = floor(s_j 2^50) so every implementation reproduces the same bits; draws
+// point u_j = floor(s_j 2^50) so every implementation reproduces the same bits (a row
+// whose exact sum U = sum u_j needs more than 64 bits is rejected as invalid); draws
 // from Philox4x32-10 (Salmon et al., SC'11) keyed by the seed, counter (j, qb, h, b).
 // Top-k (section «Где ломаются прежние разреженные схемы»): the K largest scores, ties
 // to the lower index, found by an MSB-first radix select on the score bits.
@@ -125,23 +126,27 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
     const float *s = scores + row * nkb;
     const int tid = threadIdx.x;
 
-    // pass 0: validate, U = sum u_j, number of positive u_j
-    unsigned long long U = 0, npos = 0, nbad = 0;
+    // pass 0: validate, U = sum u_j, number of positive u_j. U is summed exactly as
+    // U_hi = sum (u_j >> 12) and U_lo = sum (u_j & 0xfff) (neither can overflow), and a row
+    // whose U needs more than 64 bits is rejected like a bad score.
+    unsigned long long u_hi = 0, u_lo = 0, counts = 0;  // counts: positive | bad << 32
     for (int j = tid; j < nkb; j += kSelThreads) {
         const float v = s[j];
         inS[j] = 0;
         if (!score_ok(v)) {
-            ++nbad;
+            counts += 1ull << 32;
             continue;
         }
         const uint64_t u = fixed50(v);
-        U += u;
-        npos += u > 0;
+        u_hi += u >> 12;
+        u_lo += u & 0xfffull;
+        counts += u > 0;
     }
-    Sum3 t = block_sum3(U, npos, nbad, red);
-    U = t.a;
-    npos = t.b;
-    if (t.c != 0) {
+    Sum3 t = block_sum3(u_hi, u_lo, counts, red);
+    const unsigned long long top = t.a + (t.b >> 12);  // U = top * 2^12 + (U_lo mod 2^12)
+    unsigned long long U = (top << 12) | (t.b & 0xfffull);
+    unsigned long long npos = t.c & 0xffffffffull;
+    if ((t.c >> 32) != 0 || top >= (1ull << 52)) {
         for (int j = tid; j < nkb; j += kSelThreads) {
             idx[row * nkb + j] = -1;
             w[row * nkb + j] = 0.f;

@@ -14,9 +14,14 @@
  *     them as absent) and are written as 0 on output.
  *   - n_qb = n_kb = N_pad / 128 query / key blocks of 128 tokens each.
  *   - Every pointer argument except `stream` is a DEVICE pointer on the current
- *     device, allocated and owned by the caller, 16-byte aligned. The library
- *     allocates no device memory and keeps no state between calls; the only
- *     host-side work is argument validation and building TMA tensor maps.
+ *     device, allocated and owned by the caller, 16-byte aligned. The calls allocate
+ *     no device memory; the host-side work is argument validation, building TMA tensor
+ *     maps and enqueueing kernels (and, for the attention calls, one 16-byte memset).
+ *   - Library-owned device state: two file-scope __device__ arrays exist once on every
+ *     GPU that loads the library, from load until process exit: the attention
+ *     kernels' 4096 claim slots (16 bytes each; see "Scheduling" at ab_attn_fwd) and
+ *     the AB_NOALLOC_SCRATCH_BYTES scratch of ab_score_noalloc. Nothing else persists
+ *     between calls.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
  *     enqueues work on it and returns; results are ready when the stream is.
  *   - Argument errors are reported synchronously by the return value and nothing is
@@ -63,10 +68,14 @@ typedef struct {
 } ab_shape;
 
 /* Bits OR-ed into *dev_flag by the kernels. */
-#define AB_FLAG_BAD_SCORE 1u  /* ab_select: a score is NaN, infinite, < 0 or > 2 */
+#define AB_FLAG_BAD_SCORE 1u  /* ab_select: a score is NaN, infinite, < 0 or > 2, or a
+                                 SIP row's exact fixed-point sum needs more than 64 bits */
 #define AB_FLAG_BAD_INDEX 2u  /* ab_attn_*: a cnt or idx entry outside its range */
 #define AB_FLAG_BAD_WEIGHT 4u /* ab_attn_fwd: a weight is NaN, infinite or <= 0 */
 #define AB_FLAG_TIMEOUT 8u    /* a bounded in-kernel wait gave up (pipeline stalled) */
+#define AB_FLAG_SCHED_COLLISION 16u /* ab_attn_*: another attention call used the same
+                                       claim slot while this one ran (see "Scheduling" at
+                                       ab_attn_fwd); this call's output is unreliable */
 
 /* Limits: head dim d in {64, 128}; 1 <= n_kb <= 8192 (N_pad <= 1,048,576). */
 #define AB_BLOCK 128
@@ -178,6 +187,15 @@ ab_status ab_selftest_bounded_wait(int limit_us, int complete, int *dev_flag, in
                                    void *stream);
 
 /*
+ * ab_selftest_force_counter_slot -- test hook with no counterpart on the method's pages:
+ * the next attention call (from any thread) takes claim slot `slot` instead of the next
+ * one in turn, so a test can make two concurrently running calls share a slot and
+ * check that the sharing is detected (AB_FLAG_SCHED_COLLISION). Errors: AB_ERR_RANGE
+ * unless 0 <= slot < 4096.
+ */
+ab_status ab_selftest_force_counter_slot(int slot);
+
+/*
  * ab_select -- choose key blocks per query block (page section «Три приёма
  * AB-Attention», second technique SIP; section «Где ломаются прежние разреженные
  * схемы» for top-k).
@@ -192,7 +210,8 @@ ab_status ab_selftest_bounded_wait(int limit_us, int complete, int *dev_flag, in
  *   with p = 1/4 counts four times.
  * AB_MODE_TOPK: the K blocks with the largest scores (ties to the lower index),
  *   weights 1.
- * scores : fp32 [B,H,nqb,nkb], every entry finite and in [0, 2].
+ * scores : fp32 [B,H,nqb,nkb], every entry finite and in [0, 2]; for SIP the row's
+ *          U = sum_j u_j must fit in 64 bits (a row sum below 2^14; IBCS rows sum to 1).
  * idx    : out, int32 [B,H,nqb,nkb]: kept block indices in ascending order in the
  *          first cnt entries of each row, -1 after them.
  * cnt    : out, int32 [B,H,nqb].
@@ -224,9 +243,18 @@ ab_status ab_select(const float *scores, int B, int H, int nqb, int nkb, int bud
  * Device-side: an idx/cnt outside range sets AB_FLAG_BAD_INDEX (the block is clamped
  * into range), a bad weight sets AB_FLAG_BAD_WEIGHT.
  * Scheduling: the kernel hands the (b, h, query block) items to its persistent CTAs
- * from a claim counter; each call takes the next of 4096 library-owned counters in turn
- * and leaves it at zero when it ends, so calls on one stream (or captured in one graph)
- * need nothing, and up to 4096 calls may run concurrently on different streams.
+ * from a claim slot. Each call takes the next of the 4096 library-owned slots in turn
+ * (process-wide, on the host), zeroes it with a memset on `stream` just before the
+ * kernel, and tags it with its own launch number. Calls on one stream never share a
+ * slot at the same time, nor do the replays of one CUDA graph executable (CUDA orders
+ * them). Two executions share a slot only if (a) more than 4096 attention calls are
+ * in flight at once across streams, or (b) two graph executables instantiated from
+ * ONE capture of a call run at the same time: a captured call keeps the slot and tag
+ * it took at capture. Case (b) repeats the same call on the same buffers and still
+ * writes the right output. In case (a) each CTA checks the slot's tag when it starts,
+ * at every claim and when it ends; a call that finds another call's tag raises
+ * AB_FLAG_SCHED_COLLISION and marks the slot so that the other call raises it too.
+ * Treat the output of a call that raised it as unreliable.
  * Errors: AB_ERR_NULL, AB_ERR_SHAPE, AB_ERR_DTYPE (inputs not bf16, or out_dtype not
  * AB_BF16 / AB_F32), AB_ERR_UNSUPPORTED, AB_ERR_ALIGN, AB_ERR_CUDA.
  */

@@ -133,7 +133,8 @@ int orc_mean_key(const uint16_t *K, int B, int H, int N, int N_pad, int d, doubl
  *            lowest c;
  *   update : c_c = mean of its members; an empty cluster keeps its centroid;
  *   output : centroids after the T-th update, weights = member count / n_v from the
- *            T-th assignment ("вес, равный доле запросов в кластере").
+ *            T-th assignment (each cluster weighted by its share of the block's queries:
+ *            AB-Attention news page, «Три приёма AB-Attention», first technique IBCS).
  * cent [B,H,nqb,C,d], wts [B,H,nqb,C], assign [B,H,N_pad] (optional; 255 on padding),
  * min_gap [B,H,nqb] (optional): the smallest relative gap (d2 - d1) / d2 between the
  * best and second-best distance seen by any query in any iteration (1 when C = 1).
@@ -293,7 +294,9 @@ int orc_score(const double *cent, const double *wts, const double *kbar, int B, 
  *   draw: Philox4x32-10, key (lo32 seed, hi32 seed), counter (kb, qb, h, b);
  *   R53 = ((x0 << 32) | x1) >> 11; keep iff (double)R53 < p_j * 2^53;
  *   kept blocks in ascending order, w_j = (float)(1 / p_j).
- * Returns 1 in *bad when a score is not finite or outside [0, 2].
+ * Returns 1 in *bad when a score is not finite or outside [0, 2], or when the exact sum
+ * U does not fit in 64 bits (sum of the row's scores of 2^14 or more: never for IBCS
+ * scores, whose rows sum to 1), so that every integer above stays exact.
  * ------------------------------------------------------------------------------ */
 static int sip_row(const float *s, int nkb, int K, uint64_t seed, int b, int h, int qb,
                    int32_t *idx, int32_t *cnt_out, float *w, double *p, uint64_t *u)
@@ -303,12 +306,14 @@ static int sip_row(const float *s, int nkb, int K, uint64_t seed, int b, int h, 
         if (!(v >= 0.0f && v <= 2.0f)) return 1;
         u[j] = (uint64_t)floor(ldexp((double)v, 50));
     }
-    uint64_t U = 0;
+    unsigned __int128 U128 = 0;
     int positive = 0;
     for (int j = 0; j < nkb; ++j) {
-        U += u[j];
+        U128 += u[j];
         positive += u[j] > 0;
     }
+    if (U128 >> 64) return 1;
+    const uint64_t U = (uint64_t)U128;
     unsigned char *inS = (unsigned char *)calloc((size_t)nkb, 1);
     if (!inS) return 2;
     uint64_t k = 0, R = 0;

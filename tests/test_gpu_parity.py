@@ -150,6 +150,21 @@ def test_select_flags_bad_scores(orc):
         assert np.all(idx.cpu().numpy()[0, 0, 1] == -1)
 
 
+def test_sip_rejects_rows_whose_exact_sum_overflows(orc):
+    # U = 8192 * 2^51 = 2^64 in row 0 (rejected on both sides); row 1 sums just below
+    s = np.full((1, 1, 2, 8192), 2.0, dtype=np.float32)
+    s[0, 0, 1, 0] = 1.75
+    flag = _flag()
+    idx, cnt, w, p = ab.select(torch.from_numpy(s).cuda(), 100, "sip", 0, want_p=True, dev_flag=flag)
+    assert ab.check_flag(flag) & ab.FLAG_BAD_SCORE
+    idx_r, cnt_r, w_r, p_r, bad_r = orc.sip(s, 100, 0)
+    assert bad_r[0, 0, 0] == 1
+    np.testing.assert_array_equal(cnt.cpu().numpy(), cnt_r)
+    np.testing.assert_array_equal(idx.cpu().numpy(), idx_r)
+    np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), w_r.view(np.uint32))
+    np.testing.assert_array_equal(p.cpu().numpy()[0, 0, 1].view(np.uint64), p_r[0, 0, 1].view(np.uint64))
+
+
 # -------------------------------------------------------------------- scoring --------
 
 @pytest.mark.parametrize("N,d,H,C", [(1024, 64, 2, 8), (3 * 128 + 77, 128, 3, 8),

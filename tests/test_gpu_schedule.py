@@ -6,8 +6,8 @@ empty items itself and hands the others to its roles through a ring in shared me
 Small problems give every CTA a single item, so these tests use more items than SMs
 (up to several per CTA), with many empty items, ragged counts and unit plans, and check
 every row against the oracle with the bounds of tests/test_gpu_parity.py. A run of more
-launches than there are counter slots checks that each launch leaves its claim counter
-at zero for the next launch that takes the slot.
+launches than there are claim slots checks that every reuse of a slot starts clean, and
+two calls forced onto one slot while both run check that the sharing is flagged.
 """
 
 import numpy as np
@@ -165,3 +165,42 @@ def test_counter_slots_wrap(orc):
     assert ab.check_flag(flag) == 0
     assert torch.equal(out, first)
     _check(orc, q, k, v, N, idx, cnt, w, first, lse, unit=128)
+
+
+def test_calls_sharing_a_claim_slot_are_flagged_or_correct(orc):
+    # Two calls forced onto the same claim slot, on two streams, so that they run at the
+    # same time: a call that finds the other's tag raises AB_FLAG_SCHED_COLLISION; a call
+    # that raises nothing must have written exactly what it writes alone.
+    lib = ab.lib()
+    runs = []
+    for seed, (N, H, max_cnt) in enumerate([(32768, 16, 64), (4000, 6, 8)]):
+        q, k, v = _inputs(N, H, seed=40 + seed)
+        B, _, N_pad, d = q.shape
+        nqb = N_pad // 128
+        idx, cnt, w = _plan(B, H, nqb, nqb, nqb, max_cnt, 0.1, seed=50 + seed)
+        t = [x.cuda() for x in (q, k, v)] + [torch.from_numpy(a).cuda() for a in (idx, cnt, w)]
+        alone = ab.attn_fwd(*t[:3], N, *t[3:], out_dtype=torch.float32)
+        runs.append((N, t, alone))
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    flags = [torch.zeros(1, dtype=torch.int32, device="cuda") for _ in runs]
+    outs = [torch.full_like(r[2], float("nan")) for r in runs]
+    for (N, t, _), s, f, o in zip(runs, streams, flags, outs):
+        with torch.cuda.stream(s):
+            assert lib.ab_selftest_force_counter_slot(77) == 0
+            ab.attn_fwd(*t[:3], N, *t[3:], dev_flag=f, out=o, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    seen = []
+    for (N, t, alone), f, o in zip(runs, flags, outs):
+        bits = ab.check_flag(f)
+        assert bits & ~ab.FLAG_SCHED_COLLISION == 0
+        if not bits & ab.FLAG_SCHED_COLLISION:
+            assert torch.equal(o, alone)
+        seen.append(bool(bits))
+    print("collision flagged per call:", seen)
+    # a slot forced once is used once: the next call is clean again
+    N, t, alone = runs[1]
+    f = torch.zeros(1, dtype=torch.int32, device="cuda")
+    again = ab.attn_fwd(*t[:3], N, *t[3:], dev_flag=f, out_dtype=torch.float32)
+    assert ab.check_flag(f) == 0 and torch.equal(again, alone)
+    assert lib.ab_selftest_force_counter_slot(4096) == 5  # AB_ERR_RANGE

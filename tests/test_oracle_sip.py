@@ -135,6 +135,19 @@ def test_sip_rejects_bad_scores(orc):
         assert np.all(idx == -1)
 
 
+def test_sip_rejects_rows_whose_exact_sum_overflows(orc):
+    # 8192 scores of 2.0: U = 8192 * 2^51 = 2^64 does not fit in 64 bits, so the row is
+    # invalid (the integers of the water-filling would wrap); one score less fits.
+    s = np.full((1, 1, 2, 8192), 2.0, dtype=np.float32)
+    s[0, 0, 1, 0] = 1.75
+    idx, cnt, w, p, bad = orc.sip(s, 100, 0)
+    assert bad[0, 0, 0] == 1 and cnt[0, 0, 0] == 0 and np.all(idx[0, 0, 0] == -1)
+    assert bad[0, 0, 1] == 0 and cnt[0, 0, 1] > 0
+    # nearly equal scores: p ~ K / n for each block and sum p = K
+    assert abs(p[0, 0, 1].sum() - 100) <= 1e-9 * 100
+    np.testing.assert_allclose(p[0, 0, 1, 1:], 100 / 8192, rtol=1e-3)
+
+
 def test_topk_reference_cases(orc):
     s = _row([0.1, 0.3, 0.3, 0.05, 0.25])
     idx, cnt, w = orc.topk(s, 2)
