@@ -25,7 +25,8 @@ from . import synth  # noqa: F401  (seeded input generators)
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libab_attn.so")
 BLOCK = 128
-MAX_UNITS = 8192  # AB_MAX_BLOCKS: selection entries per row (key blocks or key units)
+MAX_BLOCKS = 8192  # AB_MAX_BLOCKS: key blocks per head
+MAX_UNITS = 65536  # AB_MAX_UNITS: 4-token key units per head, and entries per selection row
 
 AB_F32 = 0
 AB_BF16 = 1
@@ -81,6 +82,7 @@ def lib():
         L.ab_attn_units_topk_fwd.argtypes = [P, P, P, S, I, P, P, P, I, P, P, P]
         L.ab_selftest_bounded_wait.argtypes = [I, I, P, P, P]
         L.ab_selftest_force_counter_slot.argtypes = [I]
+        L.ab_selftest_attn_wait_limit.argtypes = [P, P, P, S, I, P, P, P, P, I, P, P, I, P]
         L.ab_check_flag.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
         L.ab_status_str.argtypes = [I]
         L.ab_status_str.restype = ctypes.c_char_p
@@ -90,7 +92,8 @@ def lib():
         for name in ("ab_score_workspace_size", "ab_score", "ab_score_noalloc", "ab_select", "ab_attn_fwd",
                      "ab_attn_topk_fwd", "ab_check_flag", "ab_version", "ab_score_units_workspace_size",
                      "ab_score_units", "ab_attn_units_fwd", "ab_attn_units_topk_fwd",
-                     "ab_selftest_bounded_wait", "ab_selftest_force_counter_slot"):
+                     "ab_selftest_bounded_wait", "ab_selftest_force_counter_slot",
+                     "ab_selftest_attn_wait_limit"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib

@@ -51,12 +51,12 @@ ab::ScoreLayout score_layout(const ab_shape &s, int C, int unit = AB_BLOCK)
                             (size_t)s.d, (size_t)C);
 }
 
-// key units accepted by the unit entry points: 128-token blocks or 4-token units, with at
-// most AB_MAX_BLOCKS units per head
+// key units accepted by the unit entry points: 128-token blocks (at most AB_MAX_BLOCKS
+// per head, checked with the shape) or 4-token units (at most AB_MAX_UNITS per head)
 ab_status check_unit(const ab_shape &s, int unit)
 {
     if (unit != AB_BLOCK && unit != AB_UNIT4) return AB_ERR_UNSUPPORTED;
-    if (s.N_pad / unit > AB_MAX_BLOCKS) return AB_ERR_RANGE;
+    if (s.N_pad / unit > AB_MAX_UNITS) return AB_ERR_RANGE;
     return AB_OK;
 }
 
@@ -64,7 +64,8 @@ ab_status cuda_status(cudaError_t e) { return ab::status_of(e); }
 
 ab_status attn_common(const void *q, const void *k, const void *v, ab_shape s, int unit,
                       const int32_t *idx, const int32_t *cnt, const float *w, void *out,
-                      ab_dtype out_dtype, float *lse, int *dev_flag, void *stream)
+                      ab_dtype out_dtype, float *lse, int *dev_flag, void *stream,
+                      unsigned long long wait_ns = 0)
 {
     if (!q || !k || !v || !idx || !cnt || !out) return AB_ERR_NULL;
     ab_status st = check_shape(s);
@@ -93,6 +94,7 @@ ab_status attn_common(const void *q, const void *k, const void *v, ab_shape s, i
     a.d = s.d;
     a.unit = unit;
     a.grid_override = 0;
+    a.wait_ns = wait_ns;
     return cuda_status(ab::launch_attn(a, (cudaStream_t)stream));
 }
 
@@ -180,7 +182,7 @@ ab_status ab_select(const float *scores, int B, int H, int nqb, int nkb, int bud
     if (mode == AB_MODE_SIP && !w) return AB_ERR_NULL;
     if (mode != AB_MODE_SIP && mode != AB_MODE_TOPK) return AB_ERR_UNSUPPORTED;
     if (B <= 0 || H <= 0 || nqb <= 0 || nkb <= 0) return AB_ERR_SHAPE;
-    if (nkb > AB_MAX_BLOCKS || budget < 1) return AB_ERR_RANGE;
+    if (nkb > AB_MAX_UNITS || budget < 1) return AB_ERR_RANGE;
     if ((long long)B * H * nqb > 2147483647LL) return AB_ERR_RANGE;
     if (!aligned16(scores) || !aligned16(idx) || !aligned16(cnt) || (w && !aligned16(w)) ||
         (p && !aligned16(p)))
@@ -229,6 +231,18 @@ ab_status ab_attn_topk_fwd(const void *q, const void *k, const void *v, ab_shape
     NvtxRange nvtx("ab_attn_topk_fwd");
     return attn_common(q, k, v, s, AB_BLOCK, idx, cnt, nullptr, out, out_dtype, lse, dev_flag,
                        stream);
+}
+
+ab_status ab_selftest_attn_wait_limit(const void *q, const void *k, const void *v, ab_shape s,
+                                      int key_unit, const int32_t *idx, const int32_t *cnt,
+                                      const float *w, void *out, ab_dtype out_dtype, float *lse,
+                                      int *dev_flag, int limit_ns, void *stream)
+{
+    NvtxRange nvtx("ab_selftest_attn_wait_limit");
+    if (!dev_flag) return AB_ERR_NULL;
+    if (limit_ns < 1 || limit_ns > 1000000000) return AB_ERR_RANGE;
+    return attn_common(q, k, v, s, key_unit, idx, cnt, w, out, out_dtype, lse, dev_flag, stream,
+                       (unsigned long long)limit_ns);
 }
 
 ab_status ab_check_flag(const int *dev_flag, int *host_flag, void *stream)

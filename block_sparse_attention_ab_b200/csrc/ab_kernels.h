@@ -61,6 +61,7 @@ struct AttnLaunch {
     int B, H, N, N_pad, d;
     int unit;           // key unit of idx entries: 128 (key blocks) or 4 (gathered 4-token units)
     int grid_override;  // > 0: number of CTAs (tests); 0: one per SM
+    unsigned long long wait_ns;  // > 0: limit of the kernel's bounded waits (tests); 0: 2 s
 };
 cudaError_t launch_attn(const AttnLaunch &a, cudaStream_t st);
 // Tests: the next attention launch uses claim slot `slot` (0..4095) instead of the next

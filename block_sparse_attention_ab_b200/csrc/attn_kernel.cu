@@ -82,6 +82,7 @@ struct AttnParams {
     unsigned int *counter;  // claim slot [4]: items claimed, owner tag (zeroed on the
                             // launch's stream just before the kernel)
     unsigned int tag;       // this launch's owner tag (never 0 or kSlotPoison)
+    unsigned long long wait_ns;  // limit of every bounded wait (kWaitLimitNs; shorter in tests)
 };
 
 // A claim slot is zeroed on the launch's stream right before the kernel; the first CTA
@@ -163,6 +164,7 @@ struct ItemRing {
     uint64_t *started;       // one phase per item the TMA warp's K loads enter (t >= 1)
     volatile int *abort;
     int *flag;
+    unsigned long long wait_ns;
 };
 
 // Item t of the sequence and its entry count once published; one arrive per reading warp
@@ -172,7 +174,8 @@ __device__ __forceinline__ bool ring_read(const ItemRing &q, int n_items, int t,
     const int slot = t % kRing;
     r = n_items;
     cnt = 0;
-    if (!__all_sync(0xffffffffu, mbar_wait(&q.full[slot], (t / kRing) & 1, q.abort, q.flag))) return false;
+    if (!__all_sync(0xffffffffu, mbar_wait(&q.full[slot], (t / kRing) & 1, q.abort, q.flag, q.wait_ns)))
+        return false;
     r = q.items[2 * slot];
     cnt = q.items[2 * slot + 1];
     __syncwarp();
@@ -275,6 +278,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
     iq.started = started;
     iq.abort = abort_flag;
     iq.flag = p.flag;
+    iq.wait_ns = p.wait_ns;
     // readers of every ring entry, one arrive each: the K and V cursors of warp 8 (and of
     // warp 10 for units), the S and PV cursors of the MMA warp, the 8 softmax warps
     constexpr int kRingReaders = 2 + (kUnits ? 2 : 0) + 2 + 8;
@@ -334,7 +338,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         int q_loads = 0;
         bool ok = true;
         auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
-            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag));
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag, p.wait_ns));
         };
         auto load_q = [&](const Cursor &c) -> bool {
             if (!do_q) return true;
@@ -442,7 +446,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         int kv_pos = 0;
         bool ok = true;
         auto wait = [&](uint64_t *bar, uint32_t parity) -> bool {
-            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag));
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag, p.wait_ns));
         };
         auto issue_s = [&](const Cursor &c, int g) -> bool {
             const int qbuf = c.seq & 1;
@@ -592,7 +596,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         };
         int r = blockIdx.x < (unsigned)p.n_items ? (int)blockIdx.x : p.n_items;
         for (int t = 0; ok; ++t) {
-            if (t >= 2) ok = __all_sync(0xffffffffu, mbar_wait_sleepy(started, (t - 2) & 1, abort_flag, p.flag));
+            if (t >= 2) ok = __all_sync(0xffffffffu, mbar_wait_sleepy(started, (t - 2) & 1, abort_flag, p.flag, 500, p.wait_ns));
             if (!ok) break;
             if (t > 0) r = claim();
             int c_raw = 0;
@@ -606,7 +610,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             // entry t once every reader has read its previous use
             const int slot = t % kRing;
             if (t >= kRing &&
-                !__all_sync(0xffffffffu, mbar_wait_sleepy(&ring_empty[slot], ((t / kRing) - 1) & 1, abort_flag, p.flag)))
+                !__all_sync(0xffffffffu, mbar_wait_sleepy(&ring_empty[slot], ((t / kRing) - 1) & 1, abort_flag, p.flag, 500, p.wait_ns)))
                 break;
             if (lane == 0) {
                 iq.items[2 * slot] = r;
@@ -653,7 +657,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         int o_seen = 0, o_seen_oth = 0;  // PV_h completions observed so far (own, other half)
         bool ok = true;
         auto wait_bar = [&](uint64_t *bar, uint32_t parity) {
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag, p.wait_ns));
         };
         // wait until PV_h(k) is complete (own half: k = g - 1 for a rescale; both halves:
         // k = g at the end of an item). PV_h(k) completes phase k / kSB of o_full[h][k mod
@@ -1034,6 +1038,7 @@ static cudaError_t launch_attn_t(const AttnLaunch &a, cudaStream_t st)
     p.per_tile = U4 ? 32 : 1;
     p.n_items = a.B * a.H * p.nqb;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    p.wait_ns = a.wait_ns > 0 ? a.wait_ns : kWaitLimitNs;
     cudaError_t e = counter_slot(st, &p.counter, &p.tag);
     if (e != cudaSuccess) return e;
     const int smem = AttnSmem<D>::kAlloc;

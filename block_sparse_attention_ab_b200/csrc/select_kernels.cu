@@ -8,8 +8,9 @@
 // from Philox4x32-10 (Salmon et al., SC'11) keyed by the seed, counter (j, qb, h, b).
 // Top-k (section «Где ломаются прежние разреженные схемы»): the K largest scores, ties
 // to the lower index, found by an MSB-first radix select on the score bits.
-// One CTA of 256 threads per (b, h, qb) row; kept blocks are compacted in ascending
-// order with warp ballots and a block-wide prefix.
+// One CTA of 256 threads per (b, h, qb) row (rows of up to 65536 entries: key blocks or
+// 4-token key units); kept entries are compacted in ascending order with warp ballots and
+// a block-wide prefix.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -226,13 +227,26 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
     if (tid == 0) cnt[row] = base;
 }
 
+// Score bit patterns (order-preserving for s >= 0, -0 taken as +0): staged in shared
+// memory (kSmemKeys) or, for rows too long for it, read from the scores in global memory.
+template <bool kSmemKeys>
+struct TopkKeys {
+    uint32_t *sh;
+    const float *s;
+    __device__ __forceinline__ uint32_t operator[](int j) const
+    {
+        return kSmemKeys ? sh[j] : __float_as_uint(__ldg(s + j) + 0.0f);
+    }
+};
+
+template <bool kSmemKeys>
 __global__ void __launch_bounds__(kSelThreads) topk_kernel(const float *__restrict__ scores,
                                                           int nkb, int K,
                                                           int32_t *__restrict__ idx,
                                                           int32_t *__restrict__ cnt,
                                                           float *__restrict__ w, int *flag)
 {
-    extern __shared__ uint32_t keys[];  // nkb score bit patterns (order-preserving for s >= 0)
+    extern __shared__ uint32_t keys_sh[];  // kSmemKeys: nkb score bit patterns
     __shared__ unsigned long long red[kSelWarps][3];
     __shared__ int hist[256];
     __shared__ int wtot[kSelWarps];
@@ -243,11 +257,12 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const float *__restri
     const float *s = scores + row * nkb;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+    const TopkKeys<kSmemKeys> keys{keys_sh, s};
     unsigned long long nbad = 0;
     for (int j = tid; j < nkb; j += kSelThreads) {
         const float v = s[j];
         if (!score_ok(v)) ++nbad;
-        keys[j] = __float_as_uint(v + 0.0f);  // -0 -> +0
+        if (kSmemKeys) keys_sh[j] = __float_as_uint(v + 0.0f);  // -0 -> +0
     }
     const Sum3 t = block_sum3(nbad, 0, 0, red);
     if (t.a != 0) {
@@ -330,13 +345,25 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const float *__restri
     if (tid == 0) cnt[row] = base;
 }
 
+// Rows of more than 48 KB of per-row shared memory need the opt-in limit.
+constexpr size_t kTopkSmemKeysMax = 160 * 1024;
+
+template <typename Kern>
+static cudaError_t allow_smem(Kern kern, size_t bytes)
+{
+    if (bytes <= 48 * 1024) return cudaSuccess;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
 cudaError_t launch_sip(const float *scores, int B, int H, int nqb, int nkb, int K, uint64_t seed,
                        int32_t *idx, int32_t *cnt, float *w, double *p, int *flag, cudaStream_t st)
 {
     const unsigned rows = (unsigned)((size_t)B * H * nqb);
-    sip_kernel<<<rows, kSelThreads, (size_t)nkb, st>>>(scores, H, nqb, nkb, K, (uint32_t)seed,
-                                                       (uint32_t)(seed >> 32), idx, cnt, w, p,
-                                                       flag);
+    const size_t smem = (size_t)nkb;
+    cudaError_t e = allow_smem(sip_kernel, smem);
+    if (e != cudaSuccess) return e;
+    sip_kernel<<<rows, kSelThreads, smem, st>>>(scores, H, nqb, nkb, K, (uint32_t)seed,
+                                                (uint32_t)(seed >> 32), idx, cnt, w, p, flag);
     return cudaGetLastError();
 }
 
@@ -344,8 +371,14 @@ cudaError_t launch_topk(const float *scores, int B, int H, int nqb, int nkb, int
                         int32_t *cnt, float *w, int *flag, cudaStream_t st)
 {
     const unsigned rows = (unsigned)((size_t)B * H * nqb);
-    topk_kernel<<<rows, kSelThreads, (size_t)nkb * sizeof(uint32_t), st>>>(scores, nkb, K, idx,
-                                                                            cnt, w, flag);
+    const size_t smem = (size_t)nkb * sizeof(uint32_t);
+    if (smem <= kTopkSmemKeysMax) {
+        cudaError_t e = allow_smem(topk_kernel<true>, smem);
+        if (e != cudaSuccess) return e;
+        topk_kernel<true><<<rows, kSelThreads, smem, st>>>(scores, nkb, K, idx, cnt, w, flag);
+    } else {
+        topk_kernel<false><<<rows, kSelThreads, 0, st>>>(scores, nkb, K, idx, cnt, w, flag);
+    }
     return cudaGetLastError();
 }
 

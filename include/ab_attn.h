@@ -81,9 +81,10 @@ typedef struct {
 #define AB_BLOCK 128
 #define AB_MAX_BLOCKS 8192
 /* The page's fine-grained key/value selection unit (section «Три приёма AB-Attention»,
- * third technique): 4 tokens. With it at most AB_MAX_BLOCKS units per head
- * (N_pad <= 32768). */
+ * third technique): 4 tokens. With it at most AB_MAX_UNITS units per head
+ * (N_pad <= 262144); ab_select takes rows of up to AB_MAX_UNITS entries. */
 #define AB_UNIT4 4
+#define AB_MAX_UNITS 65536
 
 /*
  * ab_score_workspace_size -- bytes of device scratch ab_score() needs for shape `s`
@@ -159,11 +160,11 @@ ab_status ab_score_noalloc(const void *q, const void *k, ab_shape s, int n_clust
  * scores[qb][u] = sum_c w_c softmax_u(cent_c . kbar_u / sqrt(d)) over the units that
  * hold at least one valid token (u < ceil(N / key_unit)); the other units score 0.
  * With key_unit = AB_BLOCK this is ab_score.
- * scores : out, fp32 [B,H,n_qb,n_ku], n_ku = N_pad / key_unit (<= AB_MAX_BLOCKS).
+ * scores : out, fp32 [B,H,n_qb,n_ku], n_ku = N_pad / key_unit (<= AB_MAX_UNITS).
  * kbar   : optional out, fp32 [B,H,n_ku,d]. Other arguments as ab_score; the workspace
  *          needs ab_score_units_workspace_size() bytes.
  * Errors: as ab_score; AB_ERR_UNSUPPORTED for another key_unit, AB_ERR_RANGE when
- * n_ku > AB_MAX_BLOCKS.
+ * n_ku > AB_MAX_UNITS.
  */
 ab_status ab_score_units_workspace_size(ab_shape s, int n_clusters, int key_unit, size_t *bytes);
 ab_status ab_score_units(const void *q, const void *k, ab_shape s, int n_clusters, int iters,
@@ -185,6 +186,22 @@ ab_status ab_score_units(const void *q, const void *k, ab_shape s, int n_cluster
  */
 ab_status ab_selftest_bounded_wait(int limit_us, int complete, int *dev_flag, int *dev_done,
                                    void *stream);
+
+/*
+ * ab_selftest_attn_wait_limit -- test entry point with no counterpart on the method's
+ * pages: ab_attn_units_fwd (w != NULL) or ab_attn_units_topk_fwd (w == NULL) with every
+ * bounded wait inside the attention kernel limited to limit_ns nanoseconds (1..1e9)
+ * instead of 2 s, so that a test can make the kernel's own waits give up. A wait that
+ * gives up ORs AB_FLAG_TIMEOUT into *dev_flag (required here) and every role of the CTA
+ * unwinds: the producer and MMA warps let their copies and MMAs in flight land, the
+ * softmax warps run out their loops without waiting, and the CTA frees its tensor
+ * memory and returns, leaving the context usable. The output of such a call is
+ * undefined. Arguments and errors otherwise as ab_attn_units_fwd.
+ */
+ab_status ab_selftest_attn_wait_limit(const void *q, const void *k, const void *v, ab_shape s,
+                                      int key_unit, const int32_t *idx, const int32_t *cnt,
+                                      const float *w, void *out, ab_dtype out_dtype, float *lse,
+                                      int *dev_flag, int limit_ns, void *stream);
 
 /*
  * ab_selftest_force_counter_slot -- test hook with no counterpart on the method's pages:
@@ -219,7 +236,7 @@ ab_status ab_selftest_force_counter_slot(int slot);
  *          optional (NULL) for top-k.
  * p      : optional out, fp64 [B,H,nqb,nkb]: p_j by block index (SIP only).
  * A row with an invalid score sets AB_FLAG_BAD_SCORE and gets cnt = 0, idx = -1.
- * Errors: AB_ERR_NULL, AB_ERR_SHAPE, AB_ERR_RANGE (budget < 1, nkb > AB_MAX_BLOCKS),
+ * Errors: AB_ERR_NULL, AB_ERR_SHAPE, AB_ERR_RANGE (budget < 1, nkb > AB_MAX_UNITS),
  * AB_ERR_ALIGN, AB_ERR_CUDA.
  */
 ab_status ab_select(const float *scores, int B, int H, int nqb, int nkb, int budget,
@@ -285,7 +302,7 @@ ab_status ab_attn_topk_fwd(const void *q, const void *k, const void *v, ab_shape
  *         / sum_{u in sel} w_u sum_{t in u, t<N} e^{q_i.k_t/sqrt(d)}
  * With key_unit = AB_BLOCK these are ab_attn_fwd / ab_attn_topk_fwd.
  * Errors and device flags: as ab_attn_fwd; AB_ERR_UNSUPPORTED for another key_unit,
- * AB_ERR_RANGE when n_ku > AB_MAX_BLOCKS.
+ * AB_ERR_RANGE when n_ku > AB_MAX_UNITS.
  */
 ab_status ab_attn_units_fwd(const void *q, const void *k, const void *v, ab_shape s, int key_unit,
                             const int32_t *idx, const int32_t *cnt, const float *w, void *out,

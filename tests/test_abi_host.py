@@ -111,7 +111,7 @@ def test_select_argument_checks(L):
     assert L.ab_select(FAKE, 1, 1, 8, 8, 3, 7, u, FAKE, FAKE, FAKE, None, None, None) == 4
     assert L.ab_select(FAKE, 0, 1, 8, 8, 3, 0, u, FAKE, FAKE, FAKE, None, None, None) == 2
     assert L.ab_select(FAKE, 1, 1, 8, 8, 0, 0, u, FAKE, FAKE, FAKE, None, None, None) == 5
-    assert L.ab_select(FAKE, 1, 1, 8, 8193, 3, 1, u, FAKE, FAKE, None, None, None, None) == 5
+    assert L.ab_select(FAKE, 1, 1, 8, 65537, 3, 1, u, FAKE, FAKE, None, None, None, None) == 5
     assert L.ab_select(MISALIGNED, 1, 1, 8, 8, 3, 1, u, FAKE, FAKE, None, None, None, None) == 9
 
 
@@ -147,8 +147,10 @@ def test_unit_entry_points_reject_bad_units(L):
                                None, None) == 4
     assert L.ab_attn_units_topk_fwd(FAKE, FAKE, FAKE, s, 2, FAKE, FAKE, FAKE, ab.AB_BF16, None,
                                     None, None) == 4
-    # at most AB_MAX_BLOCKS units per head: 4-token units need N_pad <= 32768
-    big = shape(N=32896, N_pad=32896)
+    # at most AB_MAX_UNITS = 65536 units per head: 4-token units need N_pad <= 262144
+    ok = shape(N=262144, N_pad=262144)
+    assert L.ab_score_units_workspace_size(ok, 8, 4, ctypes.byref(n)) == 0
+    big = shape(N=262144 + 128, N_pad=262144 + 128)
     assert L.ab_score_units_workspace_size(big, 8, 4, ctypes.byref(n)) == 5
     assert L.ab_attn_units_topk_fwd(FAKE, FAKE, FAKE, big, 4, FAKE, FAKE, FAKE, ab.AB_BF16, None,
                                     None, None) == 5
@@ -156,6 +158,11 @@ def test_unit_entry_points_reject_bad_units(L):
                             None, None) == 5
     assert L.ab_attn_units_fwd(FAKE, FAKE, FAKE, s, 4, FAKE, FAKE, None, FAKE, ab.AB_BF16, None,
                                None, None) == 1
+
+
+def test_select_row_length_limit(L):
+    # rows of up to AB_MAX_UNITS entries; a longer row is rejected before any launch
+    assert L.ab_select(FAKE, 1, 1, 1, 65537, 4, 0, 0, FAKE, FAKE, FAKE, None, None, None) == 5
 
 
 def test_unit_workspace_size(L):

@@ -1,7 +1,9 @@
 """Failure detection without a GPU fault: an in-kernel wait on an mbarrier that nothing
 completes must give up after its limit, report AB_FLAG_TIMEOUT through the device flag
 and return, leaving the CUDA context usable for the next call (the bounded wait every
-pipeline role of the library uses)."""
+pipeline role of the library uses). The attention kernel itself is run with its waits
+limited to 1 us, so that its own unwind path (drains, softmax loops run out, tensor
+memory freed) runs and the next call on the same context still gives the right result."""
 
 import time
 
@@ -59,3 +61,67 @@ def test_selftest_argument_checks():
     assert L.ab_selftest_bounded_wait(0, 0, None, None, None) == 1
     flag = torch.zeros(1, dtype=torch.int32, device="cuda")
     assert L.ab_selftest_bounded_wait(0, 0, ab._ptr(flag), ab._ptr(flag), None) == 5
+
+
+def _attn_with_limit(q, k, v, N, idx, cnt, w, unit, limit_ns):
+    """ab_selftest_attn_wait_limit through the C ABI: the attention call with every wait
+    inside the kernel limited to limit_ns; returns (flag bits, out)."""
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+    code = ab.lib().ab_selftest_attn_wait_limit(
+        ab._ptr(q), ab._ptr(k), ab._ptr(v), ab.make_shape(q, N), unit, ab._ptr(idx), ab._ptr(cnt),
+        ab._ptr(w), ab._ptr(out), ab.AB_F32, None, ab._ptr(flag), int(limit_ns), ab._stream())
+    assert code == 0, ab.STATUS.get(code, code)
+    return ab.check_flag(flag), out
+
+
+@pytest.mark.parametrize("unit", [128, 4])
+def test_attention_wait_limit_runs_out(orc, unit):
+    # the attention kernel's own waits (TMA tiles, MMAs, the item ring) given 1 us: some
+    # wait gives up, the flag reports it, every CTA unwinds and returns, and the next
+    # call on the same context matches the oracle
+    g = torch.Generator().manual_seed(11)
+    N, H, d = 2000, 3, 128
+    N_pad = (N + 127) // 128 * 128
+    q, k, v = (torch.zeros(1, H, N_pad, d, dtype=torch.bfloat16) for _ in range(3))
+    for t in (q, k, v):
+        t[:, :, :N] = torch.randn(1, H, N, d, generator=g).to(torch.bfloat16)
+    nkb = N_pad // unit
+    n_valid = -(-N // unit)
+    nqb = N_pad // 128
+    rng = np.random.default_rng(unit)
+    idx = np.full((1, H, nqb, nkb), -1, dtype=np.int32)
+    cnt = np.zeros((1, H, nqb), dtype=np.int32)
+    w = np.zeros((1, H, nqb, nkb), dtype=np.float32)
+    for h in range(H):
+        for qb in range(nqb):
+            c = int(rng.integers(1, min(n_valid, 200) + 1))
+            idx[0, h, qb, :c] = np.sort(rng.choice(n_valid, c, replace=False))
+            cnt[0, h, qb] = c
+            w[0, h, qb, :c] = rng.uniform(1.0, 3.0, c)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    ic, cc, wc = (torch.from_numpy(a).cuda() for a in (idx, cnt, w))
+    # a generous limit: nothing gives up and the result is right
+    bits, good = _attn_with_limit(qc, kc, vc, N, ic, cc, wc, unit, 1_000_000_000)
+    assert bits == 0
+    t0 = time.perf_counter()
+    bits, _ = _attn_with_limit(qc, kc, vc, N, ic, cc, wc, unit, 1000)
+    assert time.perf_counter() - t0 < 10.0
+    assert bits & ab.FLAG_TIMEOUT and not bits & ~(ab.FLAG_TIMEOUT | ab.FLAG_BAD_INDEX)
+    # the context is usable: the normal call gives the result it gave before
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    again = ab.attn_fwd(qc, kc, vc, N, ic, cc, wc, dev_flag=flag, out_dtype=torch.float32, unit=unit)
+    assert ab.check_flag(flag) == 0
+    assert torch.equal(again, good)
+    ref, _, _, _ = orc.attn_rows(q, k, v, N, idx, cnt, w, unit=unit)
+    got = good.cpu().numpy().reshape(H * nqb, 128, d)
+    assert np.abs(got - ref).max() <= 1e-2
+
+
+def test_attention_wait_limit_argument_checks():
+    L = ab.lib()
+    z = torch.zeros(16, dtype=torch.int32, device="cuda")
+    s = ab.Shape(1, 1, 128, 128, 64, ab.AB_BF16)
+    p = ab._ptr(z)
+    assert L.ab_selftest_attn_wait_limit(p, p, p, s, 128, p, p, p, p, ab.AB_F32, None, None, 1000, None) == 1
+    assert L.ab_selftest_attn_wait_limit(p, p, p, s, 128, p, p, p, p, ab.AB_F32, None, p, 0, None) == 5

@@ -196,3 +196,77 @@ def test_unit_path_at_wan13b_size(orc):
     nqb = w.N_pad // 128
     sample = np.array([0 * nqb + 3, 0 * nqb + nqb - 1, 1 * nqb + 100, 1 * nqb + 7], dtype=np.int64)
     _compare(orc, q, k, v, w.N, idx, cnt, wt, out, lse, rows=sample)
+
+
+def test_unit_path_at_hunyuan720_size(orc):
+    """Two heads of the HunyuanVideo-720p-shaped workload (N = 118800 tokens, 29728 4-token
+    units per head, 29700 of them holding a valid token) at the bench's tile budget (93
+    tiles = 2976 units): unit scores on sampled rows against the oracle fed the GPU's own
+    centroids, weights and mean keys, the SIP and top-k plans bit-exact on sampled rows,
+    attention on sampled query blocks."""
+    w = synth.WORKLOADS["hunyuan720"]
+    q, k, v = synth.make_qkv(w, heads=[0, 1])
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    nqb, nku = w.N_pad // 128, w.N_pad // U
+    nvu = -(-w.N // U)
+    assert nku == 29728 and nvu == 29700
+    K = w.budget_blocks(w.budgets[0]) * 32
+    s, kbar, cent, cw, _ = ab.score(qc, kc, w.N, w.n_clusters, w.iters, unit=U, intermediates=True)
+    torch.cuda.synchronize()
+    s_np = s.cpu().numpy()
+    assert np.all(s_np[..., nvu:] == 0)
+    np.testing.assert_allclose(s_np.sum(-1), 1.0, rtol=2e-5)
+    rng = np.random.default_rng(3)
+    rows = np.sort(rng.choice(nqb, 5, replace=False))
+    ref = orc.score(cent.cpu().numpy().astype(np.float64)[:, :, rows],
+                    cw.cpu().numpy().astype(np.float64)[:, :, rows],
+                    kbar.cpu().numpy().astype(np.float64), n_valid=nvu)
+    got = s_np[:, :, rows]
+    assert np.all(np.abs(got - ref) <= SCORE_RTOL * np.abs(ref) + 1e-30)
+    sub = np.zeros_like(s_np)
+    sub[:, :, rows] = s_np[:, :, rows]
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for mode in ("topk", "sip"):
+        idx, cnt, wt = ab.select(s, K, mode, w.sip_seed, dev_flag=flag)
+        torch.cuda.synchronize()
+        if mode == "sip":
+            idx_r, cnt_r, w_r, _, _ = orc.sip(sub, K, w.sip_seed, with_p=False)
+            np.testing.assert_array_equal(wt.cpu().numpy()[:, :, rows].view(np.uint32),
+                                          w_r[:, :, rows].view(np.uint32))
+        else:
+            idx_r, cnt_r, _ = orc.topk(sub, K)
+        np.testing.assert_array_equal(cnt.cpu().numpy()[:, :, rows], cnt_r[:, :, rows])
+        np.testing.assert_array_equal(idx.cpu().numpy()[:, :, rows], idx_r[:, :, rows])
+    assert ab.check_flag(flag) == 0
+    out, lse = ab.attn_fwd(qc, kc, vc, w.N, idx, cnt, wt, want_lse=True, dev_flag=flag,
+                           out_dtype=torch.float32, unit=U)
+    torch.cuda.synchronize()
+    assert ab.check_flag(flag) == 0
+    sample = np.array([rows[0], nqb - 1, nqb + rows[2], nqb + rows[4]], dtype=np.int64)
+    _compare(orc, q, k, v, w.N, idx, cnt, wt, out, lse, rows=sample)
+
+
+@pytest.mark.parametrize("nku", [29728, 65536])
+def test_selection_rows_of_many_units(orc, nku):
+    """Selection rows of 4-token units up to the 65536-unit limit (the 262144-token shape):
+    top-k (scores staged in shared memory up to 40960 entries, read from global memory
+    beyond) and SIP (a 64 KB saturation map) bit-exact against the oracle, with ties."""
+    rng = np.random.default_rng(nku)
+    s = rng.random((1, 1, 3, nku), dtype=np.float32) ** 8
+    s[0, 0, 1, 100:2000] = s[0, 0, 1, 99]  # a long run of equal scores
+    s /= s.sum(-1, keepdims=True)
+    K = 2976 if nku < 65536 else 6560
+    sc = torch.from_numpy(s).cuda()
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx, cnt, _ = ab.select(sc, K, "topk", dev_flag=flag)
+    idx_r, cnt_r, _ = orc.topk(s, K)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), cnt_r)
+    np.testing.assert_array_equal(idx.cpu().numpy(), idx_r)
+    idx, cnt, wt, p = ab.select(sc, K, "sip", 5, want_p=True, dev_flag=flag)
+    idx_r, cnt_r, w_r, p_r, _ = orc.sip(s, K, 5)
+    torch.cuda.synchronize()
+    assert ab.check_flag(flag) == 0
+    np.testing.assert_array_equal(cnt.cpu().numpy(), cnt_r)
+    np.testing.assert_array_equal(idx.cpu().numpy(), idx_r)
+    np.testing.assert_array_equal(wt.cpu().numpy().view(np.uint32), w_r.view(np.uint32))
+    np.testing.assert_array_equal(p.cpu().numpy().view(np.uint64), p_r.view(np.uint64))
