@@ -77,11 +77,13 @@ def _attn_with_limit(q, k, v, N, idx, cnt, w, unit, limit_ns):
 
 @pytest.mark.parametrize("unit", [128, 4])
 def test_attention_wait_limit_runs_out(orc, unit):
-    # the attention kernel's own waits (TMA tiles, MMAs, the item ring) given 1 us: some
-    # wait gives up, the flag reports it, every CTA unwinds and returns, and the next
-    # call on the same context matches the oracle
+    # the attention kernel's own waits (TMA tiles, MMAs, the item ring) given 1 us: with
+    # more items than CTAs each CTA's item scheduler waits for its TMA warp to start the
+    # next item, which takes far longer, so that wait gives up; the flag reports it,
+    # every CTA unwinds and returns, and the next call on the same context matches the
+    # oracle
     g = torch.Generator().manual_seed(11)
-    N, H, d = 2000, 3, 128
+    N, H, d = 2000, 12, 128
     N_pad = (N + 127) // 128 * 128
     q, k, v = (torch.zeros(1, H, N_pad, d, dtype=torch.bfloat16) for _ in range(3))
     for t in (q, k, v):
@@ -95,7 +97,7 @@ def test_attention_wait_limit_runs_out(orc, unit):
     w = np.zeros((1, H, nqb, nkb), dtype=np.float32)
     for h in range(H):
         for qb in range(nqb):
-            c = int(rng.integers(1, min(n_valid, 200) + 1))
+            c = int(rng.integers(min(n_valid, 200) // 2, min(n_valid, 200) + 1))
             idx[0, h, qb, :c] = np.sort(rng.choice(n_valid, c, replace=False))
             cnt[0, h, qb] = c
             w[0, h, qb, :c] = rng.uniform(1.0, 3.0, c)
@@ -113,8 +115,9 @@ def test_attention_wait_limit_runs_out(orc, unit):
     again = ab.attn_fwd(qc, kc, vc, N, ic, cc, wc, dev_flag=flag, out_dtype=torch.float32, unit=unit)
     assert ab.check_flag(flag) == 0
     assert torch.equal(again, good)
-    ref, _, _, _ = orc.attn_rows(q, k, v, N, idx, cnt, w, unit=unit)
-    got = good.cpu().numpy().reshape(H * nqb, 128, d)
+    rows = np.arange(0, H * nqb, 7, dtype=np.int64)
+    ref, _, _, _ = orc.attn_rows(q, k, v, N, idx, cnt, w, rows=rows, unit=unit)
+    got = good.cpu().numpy().reshape(H * nqb, 128, d)[rows]
     assert np.abs(got - ref).max() <= 1e-2
 
 
