@@ -461,6 +461,10 @@ def run_ours(args, rank, world, local_rank):
     traffic = args.traffic if args.traffic is not None else (
         attn_traffic_from_profile(w.B * w.H) if (w.name == HEADLINE[0] and K == w.budget_blocks(HEADLINE[1])) else None)
     achieved = sel / (attn_ms * 1e-3) / 1e12
+    # the headline kernel is timed inside a long loop (seconds of continuous load under the
+    # power cap): its denominator is the sustained bf16 peak, the burst one otherwise
+    sustained = ms_step * args.steps >= 1000.0
+    peak_attn = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     sbytes = score_bytes(w)
     res = {
         "metric": METRIC,
@@ -498,9 +502,11 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor",
                      "kernel": "attn_fwd_kernel<128, weighted, bf16 out>",
                      "achieved": round(achieved, 2),
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(achieved / peaks["bf16_tflops"], 4),
-                     "peak_source": f"{peaks['source']} bf16 dense burst",
+                     "peak": peak_attn, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_attn, 4),
+                     "peak_source": (f"{peaks['source']} bf16 dense {'sustained' if sustained else 'burst'} "
+                                     f"(timed inside {ms_step * args.steps / 1e3:.1f} s of back-to-back steps)"),
+                     "frac_vs_burst": round(achieved / peaks["bf16_tflops"], 4),
                      "traffic": traffic,
                      "algorithmic_bytes": 4 * q.numel() * 2,
                      "per_launch": f"4*128*128*d FLOP x sum_cnt = {sel / 1e12:.2f} TFLOP; median of "
