@@ -684,7 +684,9 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         };
         auto clamp_j = [&](int j) { return j < 0 ? 0 : (j >= p.nkb ? p.nkb - 1 : j); };
         constexpr int kHalfD = D / 2;
-        constexpr int kSoftPairs = 6;  // of 32 pairs per block: exp2 on the FMA pipe
+        // pairs e with e % 5 == 4 (6 of 32 per block) take the FMA-pipe exp2, spread through
+        // the loop so that FMA-pipe and MUFU work interleave
+        constexpr int kSoftEvery = 5;
         const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
         // Item t of the CTA's sequence from the ring. The two warps of a pair take the
         // smaller of their two reads (n_items after a failed wait), so they always walk
@@ -867,7 +869,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                     }
                 }
                 // P = 2^(s * scale_log2 + lw - m_run) in fp32 pairs, packed to bf16 over
-                // the S columns; the first kSoftPairs pairs use the FMA-pipe exp2.
+                // the S columns; every fifth pair uses the FMA-pipe exp2.
                 // A half row may have seen no valid key yet (its columns of the block
                 // past the sequence end, or every kept unit there); its P is then 0, not
                 // NaN
@@ -881,7 +883,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
                     const uint64_t x2 = kUnits ? f2_add(f2_pack(sv[2 * e], sv[2 * e + 1]), bias2)
                                                : f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), scale2, bias2);
                     float2 pr;
-                    if (e < kSoftPairs) {
+                    if (e % kSoftEvery == kSoftEvery - 1) {
                         pr = soft_exp2_pair(x2);
                     } else {
                         const float2 xv = f2_unpack(x2);
