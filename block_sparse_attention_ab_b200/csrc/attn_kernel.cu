@@ -15,7 +15,7 @@
 //              warps exchange each block's row max and share one O; 4-token units: each
 //              warp keeps its own max, sum and O accumulator and the two merge once per
 //              item. Each warp normalises and stores half of every output row;
-//   warp 8     TMA producer: Q tile (double buffered) and a ring of K / V tiles
+//   warp 8     TMA producer: Q tile (double buffered; single for units) and a ring of K / V tiles
 //              fetched by block index with 3-D tensor maps whose row extent is N, so
 //              rows past the sequence end arrive as zeros (units: warps 8 and 10 gather
 //              the tiles with cp.async);
@@ -125,13 +125,18 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
                  : "memory");
 }
 
-template <int D>
+// Shared memory of one attention CTA. Key blocks: Q double-buffered (the next item's Q
+// loads during the current item) and a 4-stage K/V ring (d = 128). 4-token units: the
+// gather of a tile lands later than a TMA tile and items hold many tiles, so Q is single-
+// buffered and the ring gets the freed space (5 stages at d = 128).
+template <int D, bool kUnits>
 struct AttnSmem {
     static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
     static constexpr int kBoxes = D / 64;           // 64-column (128-byte) TMA boxes per tile
-    static constexpr int kStages = D == 128 ? 4 : 8;
+    static constexpr int kQBufs = kUnits ? 1 : 2;
+    static constexpr int kStages = D == 128 ? (kUnits ? 5 : 4) : (kUnits ? 9 : 8);
     static constexpr int kQOff = 0;
-    static constexpr int kKVOff = 2 * kTileBytes;
+    static constexpr int kKVOff = kQBufs * kTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
     // barriers: q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[3], p_full[2][3],
     // o_full[2][3], drain, ring_full[R], ring_empty[R], started
@@ -248,7 +253,7 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p)
 {
-    using L = AttnSmem<D>;
+    using L = AttnSmem<D, kUnits>;
     // 4-token units: the two softmax halves of a row keep separate maxima and O
     // accumulators (their per-unit masks and weights make the shared-max exchange the
     // longer path); blocks: one shared row max per block and one O
@@ -342,8 +347,8 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
         };
         auto load_q = [&](const Cursor &c) -> bool {
             if (!do_q) return true;
-            const int b = c.seq & 1;
-            if (!wait(&q_empty[b], ((c.seq >> 1) & 1) ^ 1)) return false;
+            const int b = c.seq % L::kQBufs;
+            if (!wait(&q_empty[b], ((c.seq / L::kQBufs) & 1) ^ 1)) return false;
             uint8_t *dst = smem + L::kQOff + b * L::kTileBytes;
             const int bh = c.r / p.nqb, qb = c.r % p.nqb;
             if (elect_one()) {
@@ -361,32 +366,38 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             if (!wait(&kv_empty[s], ((kv_pos / L::kStages) & 1) ^ 1)) return false;
             if constexpr (kUnits) {
                 // gather 32 units of 4 key rows into tile rows 4 s' .. 4 s' + 3, in the
-                // 128-byte-swizzled layout the MMA descriptors read; one warp
-                // instruction copies one unit's 4 rows x 64 columns (lane = row, chunk)
+                // 128-byte-swizzled layout the MMA descriptors read; this warp copies its
+                // 16 units, one warp instruction per unit and 64-column box (lane = row rr,
+                // 16-byte chunk c8). The loop over the units is unrolled, so each unit's
+                // destination (tile row 64 half + 4 k + rr, swizzle phase rr + 4 (k mod 2))
+                // is a per-lane base plus a constant: per unit one shuffle, one address
+                // and one validity test before the copies.
                 const int cnt = c.cnt;
-                const int slot = c.i * 32 + lane;
+                const int slot = c.i * 32 + unit_half * 16 + (lane & 15);
                 int u = -1;
                 if (slot < cnt) {
                     u = __ldg(p.idx + (size_t)c.r * p.nkb + slot);
                     if (u < 0 || u >= p.nkb) {
-                        if (tm == &tmK && unit_half == 0) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
+                        if (tm == &tmK && lane < 16) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
                         u = -1;
                     }
                 }
-                const __nv_bfloat16 *src = (tm == &tmK ? p.kg : p.vg) + (size_t)(c.r / p.nqb) * p.N_pad * D;
-                const uint32_t dst = smem_u32(smem + L::kKVOff + s * L::kTileBytes);
                 const int rr = lane >> 3, c8 = lane & 7;
-#pragma unroll 4
-                for (int su = unit_half * 16; su < unit_half * 16 + 16; ++su) {
-                    const int us = __shfl_sync(0xffffffffu, u, su);
-                    const int tok = us * 4 + rr;
-                    const bool valid = us >= 0 && tok < p.N;
-                    const int row = su * 4 + rr;
-                    const __nv_bfloat16 *g = src + (size_t)(valid ? tok : 0) * D + c8 * 8;
+                const char *src = reinterpret_cast<const char *>(tm == &tmK ? p.kg : p.vg) +
+                                  ((size_t)(c.r / p.nqb) * p.N_pad + rr) * (D * 2) + c8 * 16;
+                const uint32_t dst = smem_u32(smem + L::kKVOff + s * L::kTileBytes) +
+                                     (uint32_t)(unit_half * 64 + rr) * 128;
+                const uint32_t sw_even = (uint32_t)(c8 ^ rr) << 4, sw_odd = (uint32_t)(c8 ^ (rr + 4)) << 4;
+                const int rows_left = p.N - rr;  // unit us holds a valid row here iff 4 us < rows_left
 #pragma unroll
-                    for (int h = 0; h < L::kBoxes; ++h)
-                        cp_async_16(dst + h * 16384 + row * 128 + ((c8 ^ (row & 7)) << 4), g + h * 64,
-                                    valid ? 16u : 0u);
+                for (int k = 0; k < 16; ++k) {
+                    const int us = __shfl_sync(0xffffffffu, u, k);
+                    const bool valid = us >= 0 && us * 4 < rows_left;
+                    const char *g = src + (size_t)(valid ? us : 0) * (4 * D * 2);
+                    const uint32_t d0 = dst + k * 512 + ((k & 1) ? sw_odd : sw_even);
+                    const uint32_t nbytes = valid ? 16u : 0u;
+#pragma unroll
+                    for (int h = 0; h < L::kBoxes; ++h) cp_async_16(d0 + h * 16384, g + h * 128, nbytes);
                 }
                 cp_async_arrive_noinc(&kv_full[s]);
                 ++kv_pos;
@@ -427,8 +438,8 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             // drain: the last loads issued may still be in flight
             for (int k = kv_pos - L::kStages; k < kv_pos; ++k)
                 if (k >= 0) drain_wait(&kv_full[k % L::kStages], (k / L::kStages) & 1);
-            for (int k = q_loads - 2; k < q_loads; ++k)
-                if (k >= 0) drain_wait(&q_full[k & 1], (k >> 1) & 1);
+            for (int k = q_loads - L::kQBufs; k < q_loads; ++k)
+                if (k >= 0) drain_wait(&q_full[k % L::kQBufs], (k / L::kQBufs) & 1);
         }
     } else if (warp == kWarpMma) {
         // ------------------------------- MMA issuer -------------------------------
@@ -449,8 +460,8 @@ __global__ void __launch_bounds__(attn_threads(kUnits), 1)
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.flag, p.wait_ns));
         };
         auto issue_s = [&](const Cursor &c, int g) -> bool {
-            const int qbuf = c.seq & 1;
-            if (c.i == 0 && !wait(&q_full[qbuf], (c.seq >> 1) & 1)) return false;
+            const int qbuf = c.seq % L::kQBufs;
+            if (c.i == 0 && !wait(&q_full[qbuf], (c.seq / L::kQBufs) & 1)) return false;
             const int s = kv_pos % L::kStages;
             if (!wait(&kv_full[s], (kv_pos / L::kStages) & 1)) return false;
             if constexpr (kUnits) fence_proxy_async_smem();  // tile written by cp.async
@@ -1043,7 +1054,7 @@ static cudaError_t launch_attn_t(const AttnLaunch &a, cudaStream_t st)
     p.wait_ns = a.wait_ns > 0 ? a.wait_ns : kWaitLimitNs;
     cudaError_t e = counter_slot(st, &p.counter, &p.tag);
     if (e != cudaSuccess) return e;
-    const int smem = AttnSmem<D>::kAlloc;
+    const int smem = AttnSmem<D, U4>::kAlloc;
     e = cudaFuncSetAttribute(attn_fwd_kernel<D, W, F32, U4>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
