@@ -9,8 +9,9 @@
 // Top-k (section «Где ломаются прежние разреженные схемы»): the K largest scores, ties
 // to the lower index, found by an MSB-first radix select on the score bits.
 // One CTA of 256 threads per (b, h, qb) row (rows of up to 65536 entries: key blocks or
-// 4-token key units); kept entries are compacted in ascending order with warp ballots and
-// a block-wide prefix.
+// 4-token key units); kept entries are compacted in ascending order: each warp owns a
+// contiguous slab of the row and uses ballots, and one block-wide prefix over the eight
+// warps' counts places the slabs.
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -88,26 +89,6 @@ __device__ Sum3 block_sum3(unsigned long long a, unsigned long long b, unsigned 
     return s;
 }
 
-// Ordered compaction step: returns the exclusive position of this thread's element
-// among the kept elements of the current chunk and writes the chunk total to *total.
-__device__ __forceinline__ int chunk_prefix(bool keep, int *wtot, int *total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    __syncthreads();
-    if (lane == 0) wtot[warp] = __popc(m);
-    __syncthreads();
-    int before = 0, all = 0;
-#pragma unroll
-    for (int w = 0; w < kSelWarps; ++w) {
-        const int t = wtot[w];
-        before += (w < warp) ? t : 0;
-        all += t;
-    }
-    *total = all;
-    return before + __popc(m & ((1u << lane) - 1u));
-}
-
 __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restrict__ scores,
                                                          int H, int nqb, int nkb, int K,
                                                          uint32_t key0, uint32_t key1,
@@ -116,7 +97,8 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
                                                          float *__restrict__ w,
                                                          double *__restrict__ p_out, int *flag)
 {
-    extern __shared__ uint8_t inS[];  // nkb bytes: 0 = out, 1 = saturated, 2 = joining
+    // nkb bytes (0 = out, 1 = saturated, 2 = joining), then the keep bits of the draws
+    extern __shared__ __align__(16) uint8_t inS[];
     __shared__ unsigned long long red[kSelWarps][3];
     __shared__ int wtot[kSelWarps];
 
@@ -191,20 +173,30 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
         }
     }
 
-    // probabilities, draws, ordered compaction
+    // probabilities and draws, then ordered compaction. Warp w owns the contiguous slab
+    // [w L, (w + 1) L) of the row (L a multiple of 32): it draws its entries 32 at a time,
+    // keeps the keep-bits of each 32-entry chunk in shared memory and counts its kept
+    // entries; one block barrier gives each warp its output offset (the kept entries of
+    // the slabs before it), and a second walk over the slab writes the kept indices and
+    // weights in ascending order. Two block barriers per row instead of two per 256
+    // entries.
     const double Rd = __ull2double_rn(R);
-    int base = 0;
-    for (int j0 = 0; j0 < nkb; j0 += kSelThreads) {
-        const int j = j0 + tid;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int slab = (((nkb + kSelWarps - 1) / kSelWarps) + 31) & ~31;
+    const int j_begin = min(nkb, warp * slab), j_end = min(nkb, j_begin + slab);
+    uint32_t *keep_bits = reinterpret_cast<uint32_t *>(inS + ((nkb + 15) & ~15));  // [nkb / 32]
+    auto prob = [&](int j) -> double {  // p_j of entry j
+        if (inS[j] == 1) return 1.0;
+        if (all_positive_kept) return 0.0;
+        const uint64_t u = fixed50(s[j]);
+        return u > 0 ? __ull2double_rn(k_rest * u) / Rd : 0.0;
+    };
+    int kept_here = 0;
+    for (int j0 = j_begin; j0 < j_end; j0 += 32) {
+        const int j = j0 + lane;
         bool keep = false;
-        double pj = 0.0;
-        if (j < nkb) {
-            if (inS[j] == 1) {
-                pj = 1.0;
-            } else if (!all_positive_kept) {
-                const uint64_t u = fixed50(s[j]);
-                if (u > 0) pj = __ull2double_rn(k_rest * u) / Rd;
-            }
+        if (j < j_end) {
+            const double pj = prob(j);
             if (p_out) p_out[row * nkb + j] = pj;
             const uint4 x = philox_4x32_10(make_uint4((uint32_t)j, (uint32_t)qb, (uint32_t)h,
                                                       (uint32_t)b),
@@ -212,19 +204,35 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
             const uint64_t r53 = ((((uint64_t)x.x) << 32) | x.y) >> 11;
             keep = __ull2double_rn(r53) < pj * 9007199254740992.0;
         }
-        int total;
-        const int pos = chunk_prefix(keep, wtot, &total);
-        if (keep) {
-            idx[row * nkb + base + pos] = j;
-            w[row * nkb + base + pos] = __double2float_rn(1.0 / pj);
-        }
-        base += total;
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) keep_bits[j0 >> 5] = m;
+        kept_here += __popc(m);
     }
-    for (int c = base + tid; c < nkb; c += kSelThreads) {
+    if (lane == 0) wtot[warp] = kept_here;
+    __syncthreads();
+    int base = 0, total = 0;
+#pragma unroll
+    for (int v = 0; v < kSelWarps; ++v) {
+        const int t = wtot[v];
+        base += v < warp ? t : 0;
+        total += t;
+    }
+    __syncwarp();
+    for (int j0 = j_begin; j0 < j_end; j0 += 32) {
+        const unsigned m = keep_bits[j0 >> 5];
+        const int j = j0 + lane;
+        if ((m >> lane) & 1u) {
+            const int pos = base + __popc(m & ((1u << lane) - 1u));
+            idx[row * nkb + pos] = j;
+            w[row * nkb + pos] = __double2float_rn(1.0 / prob(j));
+        }
+        base += __popc(m);
+    }
+    for (int c = total + tid; c < nkb; c += kSelThreads) {
         idx[row * nkb + c] = -1;
         w[row * nkb + c] = 0.f;
     }
-    if (tid == 0) cnt[row] = base;
+    if (tid == 0) cnt[row] = total;
 }
 
 // Score bit patterns (order-preserving for s >= 0, -0 taken as +0): staged in shared
@@ -246,7 +254,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const float *__restri
                                                           int32_t *__restrict__ cnt,
                                                           float *__restrict__ w, int *flag)
 {
-    extern __shared__ uint32_t keys_sh[];  // kSmemKeys: nkb score bit patterns
+    extern __shared__ uint32_t keys_sh[];  // kSmemKeys: nkb score bit patterns; then keep bits
     __shared__ unsigned long long red[kSelWarps][3];
     __shared__ int hist[256];
     __shared__ int wtot[kSelWarps];
@@ -319,30 +327,63 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const float *__restri
         rem = sel_rem;
         __syncthreads();
     }
-    // keep key > T, plus the first `rem` keys equal to T in index order
+    // keep key > T, plus the first `rem` keys equal to T in index order. Warp w owns the
+    // slab [w L, (w + 1) L) (L a multiple of 32): it counts its keys equal to T; a block
+    // barrier gives each warp the number of equal keys before its slab; it decides its
+    // keeps (keep-bits per 32-entry chunk in shared memory) and counts them; a second
+    // barrier gives its output offset; a last walk writes the kept indices in order.
     const uint32_t T = prefix;
-    int base = 0, eq_base = 0;
-    for (int j0 = 0; j0 < nkb; j0 += kSelThreads) {
-        const int j = j0 + tid;
-        const uint32_t key = j < nkb ? keys[j] : 0u;
-        const bool eq = j < nkb && key == T;
-        int eq_total;
-        const int eq_pos = chunk_prefix(eq, wtot, &eq_total);
-        const bool keep = j < nkb && (key > T || (eq && eq_base + eq_pos < rem));
-        eq_base += eq_total;
-        int total;
-        const int pos = chunk_prefix(keep, wtot, &total);
-        if (keep) {
-            idx[row * nkb + base + pos] = j;
-            if (w) w[row * nkb + base + pos] = 1.0f;
-        }
-        base += total;
+    const int slab = (((nkb + kSelWarps - 1) / kSelWarps) + 31) & ~31;
+    const int j_begin = min(nkb, warp * slab), j_end = min(nkb, j_begin + slab);
+    uint32_t *keep_bits = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(keys_sh) +
+                                                       (kSmemKeys ? (size_t)nkb * 4 : 0));
+    const unsigned lt = (1u << lane) - 1u;
+    int eq_here = 0;
+    for (int j0 = j_begin; j0 < j_end; j0 += 32) {
+        const int j = j0 + lane;
+        eq_here += __popc(__ballot_sync(0xffffffffu, j < j_end && keys[j] == T));
     }
-    for (int c = base + tid; c < nkb; c += kSelThreads) {
+    if (lane == 0) wtot[warp] = eq_here;
+    __syncthreads();
+    int eq_run = 0;
+#pragma unroll
+    for (int v = 0; v < kSelWarps; ++v) eq_run += v < warp ? wtot[v] : 0;
+    __syncthreads();
+    int kept_here = 0;
+    for (int j0 = j_begin; j0 < j_end; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t key = j < j_end ? keys[j] : 0u;
+        const bool eq = j < j_end && key == T;
+        const unsigned meq = __ballot_sync(0xffffffffu, eq);
+        const bool keep = j < j_end && (key > T || (eq && eq_run + __popc(meq & lt) < rem));
+        const unsigned mk = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) keep_bits[j0 >> 5] = mk;
+        kept_here += __popc(mk);
+        eq_run += __popc(meq);
+    }
+    if (lane == 0) wtot[warp] = kept_here;
+    __syncthreads();
+    int base = 0, total = 0;
+#pragma unroll
+    for (int v = 0; v < kSelWarps; ++v) {
+        const int t = wtot[v];
+        base += v < warp ? t : 0;
+        total += t;
+    }
+    for (int j0 = j_begin; j0 < j_end; j0 += 32) {
+        const unsigned m = keep_bits[j0 >> 5];
+        if ((m >> lane) & 1u) {
+            const int pos = base + __popc(m & lt);
+            idx[row * nkb + pos] = j0 + lane;
+            if (w) w[row * nkb + pos] = 1.0f;
+        }
+        base += __popc(m);
+    }
+    for (int c = total + tid; c < nkb; c += kSelThreads) {
         idx[row * nkb + c] = -1;
         if (w) w[row * nkb + c] = 0.f;
     }
-    if (tid == 0) cnt[row] = base;
+    if (tid == 0) cnt[row] = total;
 }
 
 // Rows of more than 48 KB of per-row shared memory need the opt-in limit.
@@ -359,7 +400,7 @@ cudaError_t launch_sip(const float *scores, int B, int H, int nqb, int nkb, int 
                        int32_t *idx, int32_t *cnt, float *w, double *p, int *flag, cudaStream_t st)
 {
     const unsigned rows = (unsigned)((size_t)B * H * nqb);
-    const size_t smem = (size_t)nkb;
+    const size_t smem = (size_t)((nkb + 15) & ~15) + (size_t)(nkb + 255) / 256 * 32 + 32;
     cudaError_t e = allow_smem(sip_kernel, smem);
     if (e != cudaSuccess) return e;
     sip_kernel<<<rows, kSelThreads, smem, st>>>(scores, H, nqb, nkb, K, (uint32_t)seed,
@@ -371,13 +412,14 @@ cudaError_t launch_topk(const float *scores, int B, int H, int nqb, int nkb, int
                         int32_t *cnt, float *w, int *flag, cudaStream_t st)
 {
     const unsigned rows = (unsigned)((size_t)B * H * nqb);
+    const size_t bits = (size_t)(nkb + 255) / 256 * 32 + 32;  // keep bits of the compaction
     const size_t smem = (size_t)nkb * sizeof(uint32_t);
     if (smem <= kTopkSmemKeysMax) {
-        cudaError_t e = allow_smem(topk_kernel<true>, smem);
+        cudaError_t e = allow_smem(topk_kernel<true>, smem + bits);
         if (e != cudaSuccess) return e;
-        topk_kernel<true><<<rows, kSelThreads, smem, st>>>(scores, nkb, K, idx, cnt, w, flag);
+        topk_kernel<true><<<rows, kSelThreads, smem + bits, st>>>(scores, nkb, K, idx, cnt, w, flag);
     } else {
-        topk_kernel<false><<<rows, kSelThreads, 0, st>>>(scores, nkb, K, idx, cnt, w, flag);
+        topk_kernel<false><<<rows, kSelThreads, bits, st>>>(scores, nkb, K, idx, cnt, w, flag);
     }
     return cudaGetLastError();
 }
