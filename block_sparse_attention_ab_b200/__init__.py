@@ -83,6 +83,9 @@ def lib():
         L.ab_selftest_bounded_wait.argtypes = [I, I, P, P, P]
         L.ab_selftest_force_counter_slot.argtypes = [I]
         L.ab_selftest_attn_wait_limit.argtypes = [P, P, P, S, I, P, P, P, P, I, P, P, I, P]
+        L.ab_forward_host_workspace_size.argtypes = [S, I, I, I, ctypes.POINTER(ctypes.c_size_t)]
+        L.ab_forward_host.argtypes = [P, P, P, S, I, I, I, I, ctypes.c_uint64, P, I, I, P,
+                                      ctypes.c_size_t, P, P]
         L.ab_check_flag.argtypes = [P, ctypes.POINTER(ctypes.c_int), P]
         L.ab_status_str.argtypes = [I]
         L.ab_status_str.restype = ctypes.c_char_p
@@ -291,3 +294,64 @@ def ab_attention(q, k, v, N: int, budget: int, mode: str = "sip", seed: int = 0,
     if mode == "sip":
         return attn_fwd(q, k, v, N, idx, cnt, w, unit=unit)
     return attn_topk_fwd(q, k, v, N, idx, cnt, unit=unit)
+
+
+def forward_host_workspace_bytes(shape: Shape, n_clusters: int, chunk_heads: int,
+                                 out_dtype=torch.bfloat16) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().ab_forward_host_workspace_size(shape, n_clusters, int(chunk_heads), _out_code(out_dtype),
+                                                ctypes.byref(n)), "ab_forward_host_workspace_size")
+    return int(n.value)
+
+
+def default_chunk_heads(shape, device="cuda") -> int:
+    """Head pairs per ab_forward_host chunk: the fewest that give each chunk's attention
+    launch about four waves of (b, h, query block) items on this GPU. Smaller chunks
+    shorten the first copy-in and last copy-out that nothing overlaps."""
+    B, H, N_pad = shape[:3]
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    nqb = N_pad // BLOCK
+    return max(1, min(B * H, -(-4 * sms // nqb)))
+
+
+def _need_host(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def forward_host(q, k, v, N: int, budget: int, mode: str = "sip", seed: int = 0,
+                 n_clusters: int = 8, iters: int = 5, out: Optional[torch.Tensor] = None,
+                 out_dtype=torch.bfloat16, chunk_heads: Optional[int] = None,
+                 workspace: Optional[torch.Tensor] = None, dev_flag: Optional[torch.Tensor] = None,
+                 device="cuda"):
+    """The whole path for host tensors q, k, v (bf16 [B,H,N_pad,d], pinned for overlap):
+    chunks of head pairs are copied in, scored, selected and attended on the current CUDA
+    stream while the next chunk copies in and the last one's O copies out (ab_forward_host).
+    Returns the host output (pinned unless `out` is given); it is ready when the current
+    stream is. q, k, v (and `out`) must stay alive and unmodified until then: the copies
+    run asynchronously, and a freed pinned buffer may be handed out again at once."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need_host(t, torch.bfloat16, n)
+    B, H = q.shape[:2]
+    ch = int(chunk_heads) if chunk_heads is not None else default_chunk_heads(q.shape, device)
+    shape = make_shape(q, N)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype).pin_memory()
+    else:
+        _need_host(out, out_dtype, "out")
+    need = forward_host_workspace_bytes(shape, n_clusters, ch, out_dtype)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    elif workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    m = {"sip": MODE_SIP, "topk": MODE_TOPK}[mode]
+    _check(lib().ab_forward_host(_ptr(q), _ptr(k), _ptr(v), shape, int(n_clusters), int(iters), m,
+                                 int(budget), ctypes.c_uint64(int(seed) & (2**64 - 1)), _ptr(out),
+                                 _out_code(out_dtype), ch, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _ptr(dev_flag), _stream()),
+           "ab_forward_host")
+    return out

@@ -191,7 +191,7 @@ ab_status ab_select(const float *scores, int B, int H, int nqb, int nkb, int bud
     cudaStream_t cs = (cudaStream_t)stream;
     cudaError_t e;
     if (mode == AB_MODE_SIP)
-        e = ab::launch_sip(scores, B, H, nqb, nkb, K, seed, idx, cnt, w, p, dev_flag, cs);
+        e = ab::launch_sip(scores, B * H, H, 0, nqb, nkb, K, seed, idx, cnt, w, p, dev_flag, cs);
     else
         e = ab::launch_topk(scores, B, H, nqb, nkb, K, idx, cnt, w, dev_flag, cs);
     return cuda_status(e);

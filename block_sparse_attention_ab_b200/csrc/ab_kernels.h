@@ -43,8 +43,10 @@ cudaError_t launch_score(const float *cent, const float *cw, const void *kbar_te
                          cudaStream_t st);
 
 // SIP / top-k selection (select_kernels.cu)
-cudaError_t launch_sip(const float *scores, int B, int H, int nqb, int nkb, int K, uint64_t seed,
-                       int32_t *idx, int32_t *cnt, float *w, double *p, int *flag,
+// SIP over n_bh head pairs starting at global pair bh0 (b = pair / H, h = pair % H key
+// the random numbers)
+cudaError_t launch_sip(const float *scores, int n_bh, int H, int bh0, int nqb, int nkb, int K,
+                       uint64_t seed, int32_t *idx, int32_t *cnt, float *w, double *p, int *flag,
                        cudaStream_t st);
 cudaError_t launch_topk(const float *scores, int B, int H, int nqb, int nkb, int K, int32_t *idx,
                         int32_t *cnt, float *w, int *flag, cudaStream_t st);

@@ -90,7 +90,7 @@ __device__ Sum3 block_sum3(unsigned long long a, unsigned long long b, unsigned 
 }
 
 __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restrict__ scores,
-                                                         int H, int nqb, int nkb, int K,
+                                                         int H, int bh0, int nqb, int nkb, int K,
                                                          uint32_t key0, uint32_t key1,
                                                          int32_t *__restrict__ idx,
                                                          int32_t *__restrict__ cnt,
@@ -102,9 +102,11 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
     __shared__ unsigned long long red[kSelWarps][3];
     __shared__ int wtot[kSelWarps];
 
+    // row of this call; its (b, h) counts from the call's first head pair bh0 (a call on
+    // a range of head pairs draws the same numbers as one on the whole tensor)
     const size_t row = blockIdx.x;
-    const int b = (int)(row / ((size_t)H * nqb));
-    const int h = (int)((row / nqb) % H);
+    const int bh = bh0 + (int)(row / nqb);
+    const int b = bh / H, h = bh % H;
     const int qb = (int)(row % nqb);
     const float *s = scores + row * nkb;
     const int tid = threadIdx.x;
@@ -396,14 +398,15 @@ static cudaError_t allow_smem(Kern kern, size_t bytes)
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-cudaError_t launch_sip(const float *scores, int B, int H, int nqb, int nkb, int K, uint64_t seed,
-                       int32_t *idx, int32_t *cnt, float *w, double *p, int *flag, cudaStream_t st)
+cudaError_t launch_sip(const float *scores, int n_bh, int H, int bh0, int nqb, int nkb, int K,
+                       uint64_t seed, int32_t *idx, int32_t *cnt, float *w, double *p, int *flag,
+                       cudaStream_t st)
 {
-    const unsigned rows = (unsigned)((size_t)B * H * nqb);
+    const unsigned rows = (unsigned)((size_t)n_bh * nqb);
     const size_t smem = (size_t)((nkb + 15) & ~15) + (size_t)(nkb + 255) / 256 * 32 + 32;
     cudaError_t e = allow_smem(sip_kernel, smem);
     if (e != cudaSuccess) return e;
-    sip_kernel<<<rows, kSelThreads, smem, st>>>(scores, H, nqb, nkb, K, (uint32_t)seed,
+    sip_kernel<<<rows, kSelThreads, smem, st>>>(scores, H, bh0, nqb, nkb, K, (uint32_t)seed,
                                                 (uint32_t)(seed >> 32), idx, cnt, w, p, flag);
     return cudaGetLastError();
 }

@@ -13,15 +13,16 @@
  *     of 128 (the block size). Rows t >= N are never read as data (the kernels treat
  *     them as absent) and are written as 0 on output.
  *   - n_qb = n_kb = N_pad / 128 query / key blocks of 128 tokens each.
- *   - Every pointer argument except `stream` is a DEVICE pointer on the current
- *     device, allocated and owned by the caller, 16-byte aligned. The calls allocate
- *     no device memory; the host-side work is argument validation, building TMA tensor
- *     maps and enqueueing kernels (and, for the attention calls, one 16-byte memset).
+ *   - Every pointer argument except `stream` (and the host buffers of ab_forward_host)
+ *     is a DEVICE pointer on the current device, allocated and owned by the caller,
+ *     16-byte aligned. The calls allocate no device memory; the host-side work is
+ *     argument validation, building TMA tensor maps and enqueueing kernels (and, for
+ *     the attention calls, one 16-byte memset; for ab_forward_host, the copies).
  *   - Library-owned device state: two file-scope __device__ arrays exist once on every
  *     GPU that loads the library, from load until process exit: the attention
  *     kernels' 4096 claim slots (16 bytes each; see "Scheduling" at ab_attn_fwd) and
- *     the AB_NOALLOC_SCRATCH_BYTES scratch of ab_score_noalloc. Nothing else persists
- *     between calls.
+ *     the AB_NOALLOC_SCRATCH_BYTES scratch of ab_score_noalloc; and on the host, the
+ *     copy streams and events of ab_forward_host. Nothing else persists between calls.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
  *     enqueues work on it and returns; results are ready when the stream is.
  *   - Argument errors are reported synchronously by the return value and nothing is
@@ -310,6 +311,44 @@ ab_status ab_attn_units_fwd(const void *q, const void *k, const void *v, ab_shap
 ab_status ab_attn_units_topk_fwd(const void *q, const void *k, const void *v, ab_shape s,
                                  int key_unit, const int32_t *idx, const int32_t *cnt, void *out,
                                  ab_dtype out_dtype, float *lse, int *dev_flag, void *stream);
+
+/*
+ * ab_forward_host -- the whole path (ab_score, ab_select, then ab_attn_fwd for SIP or
+ * ab_attn_topk_fwd for top-k) for Q, K, V in HOST memory, with O written back to host
+ * memory: the end-to-end call of an application whose activations live on the host.
+ * The B*H (b, h) head pairs go through in chunks of chunk_heads. The copy of chunk c
+ * to the device overlaps the computation of chunk c - 1 and the copy back of chunk
+ * c - 2's O. Two device slots per tensor are carved from `workspace`, the copies run
+ * on two library-owned streams per GPU, and the computation runs on `stream`. The
+ * result is bit for bit that of the device calls on the whole tensors with the same
+ * seed: every stage works per (b, h), and SIP keys its random numbers by the global
+ * (b, h).
+ * q_host, k_host, v_host : bf16 [B,H,N_pad,d] in host memory. Page-locked memory
+ *          (cudaHostAlloc / cudaHostRegister) lets the copies overlap the computation;
+ *          pageable memory gives the same result with the copies serialised.
+ * o_host : out, [B,H,N_pad,d] in out_dtype (AB_BF16 or AB_F32), host memory.
+ * n_clusters, iters : as ab_score. mode, budget, seed : as ab_select.
+ * chunk_heads : head pairs per chunk, 1 .. B*H. Smaller chunks shorten the first
+ *          copy-in and the last copy-out that nothing overlaps; a few heads per chunk
+ *          keep each attention launch large enough to fill the GPU.
+ * workspace : device memory of ab_forward_host_workspace_size() bytes (16-byte
+ *          aligned). It holds two slots of Q, K, V and O for chunk_heads head pairs,
+ *          plus one chunk's scoring workspace, scores and plan.
+ * Returns once everything is enqueued; O is in host memory when `stream` completes.
+ * The host buffers and the workspace must stay untouched until then. Library-owned
+ * state: two copy streams and seven events per GPU, created on the first call on that
+ * GPU and kept until process exit. Concurrent calls from several host threads are
+ * safe; their copies queue on the same copy streams.
+ * Errors: AB_ERR_NULL, AB_ERR_SHAPE, AB_ERR_DTYPE, AB_ERR_UNSUPPORTED, AB_ERR_RANGE
+ * (iters, budget, chunk_heads), AB_ERR_ALIGN, AB_ERR_WORKSPACE, AB_ERR_CUDA; device-side
+ * problems as the three calls, in dev_flag.
+ */
+ab_status ab_forward_host_workspace_size(ab_shape s, int n_clusters, int chunk_heads,
+                                         ab_dtype out_dtype, size_t *bytes);
+ab_status ab_forward_host(const void *q_host, const void *k_host, const void *v_host, ab_shape s,
+                          int n_clusters, int iters, ab_mode mode, int budget, uint64_t seed,
+                          void *o_host, ab_dtype out_dtype, int chunk_heads, void *workspace,
+                          size_t workspace_bytes, int *dev_flag, void *stream);
 
 /*
  * ab_check_flag -- synchronise `stream`, copy *dev_flag to *host_flag and map it to a

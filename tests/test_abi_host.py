@@ -176,3 +176,33 @@ def test_unit_workspace_size(L):
     assert L.ab_score_units_workspace_size(shape(), 8, 128, ctypes.byref(m)) == 0
     L.ab_score_workspace_size(shape(), 8, ctypes.byref(n))
     assert m.value == n.value
+
+
+def test_forward_host_argument_checks(L):
+    # every rejection comes before any CUDA call: no device is touched
+    s = ab.Shape(1, 4, 1000, 1024, 128, ab.AB_BF16)
+    B16 = ab.AB_BF16
+    n = ctypes.c_size_t(0)
+    assert L.ab_forward_host_workspace_size(s, 8, 2, B16, ctypes.byref(n)) == 0
+    # two slots of Q, K, V (bf16) and O for 2 head pairs, plus one chunk's scoring work
+    assert n.value >= 2 * 4 * 2 * 1024 * 128 * 2
+    assert L.ab_forward_host_workspace_size(s, 8, 0, B16, ctypes.byref(n)) == 5
+    assert L.ab_forward_host_workspace_size(s, 8, 5, B16, ctypes.byref(n)) == 5
+    assert L.ab_forward_host_workspace_size(s, 9, 2, B16, ctypes.byref(n)) == 4
+    assert L.ab_forward_host_workspace_size(s, 8, 2, 7, ctypes.byref(n)) == 3
+    assert L.ab_forward_host_workspace_size(s, 8, 2, B16, None) == 1
+    assert L.ab_forward_host_workspace_size(s, 8, 2, B16, ctypes.byref(n)) == 0
+    need = n.value
+    u = ctypes.c_uint64(1)
+    call = L.ab_forward_host
+    assert call(None, FAKE, FAKE, s, 8, 5, 0, 3, u, FAKE, B16, 2, FAKE, need, None, None) == 1
+    assert call(FAKE, FAKE, FAKE, s, 8, 5, 0, 3, u, None, B16, 2, FAKE, need, None, None) == 1
+    assert call(FAKE, FAKE, FAKE, s, 8, 0, 0, 3, u, FAKE, B16, 2, FAKE, need, None, None) == 5
+    assert call(FAKE, FAKE, FAKE, s, 8, 5, 0, 0, u, FAKE, B16, 2, FAKE, need, None, None) == 5
+    assert call(FAKE, FAKE, FAKE, s, 8, 5, 3, 3, u, FAKE, B16, 2, FAKE, need, None, None) == 4
+    assert call(FAKE, FAKE, FAKE, s, 8, 5, 0, 3, u, FAKE, B16, 9, FAKE, need, None, None) == 5
+    assert call(FAKE, FAKE, FAKE, s, 8, 5, 0, 3, u, FAKE, B16, 2, MISALIGNED, need, None, None) == 9
+    assert call(FAKE, FAKE, FAKE, s, 8, 5, 0, 3, u, FAKE, B16, 2, None, need, None, None) == 10
+    assert call(FAKE, FAKE, FAKE, s, 8, 5, 0, 3, u, FAKE, B16, 2, FAKE, need - 1, None, None) == 10
+    bad = ab.Shape(1, 4, 1000, 1152, 128, ab.AB_BF16)  # N_pad - N >= 128
+    assert call(FAKE, FAKE, FAKE, bad, 8, 5, 0, 3, u, FAKE, B16, 2, FAKE, need, None, None) == 2
