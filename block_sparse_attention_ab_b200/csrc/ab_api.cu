@@ -163,12 +163,13 @@ ab_status ab_score_units(const void *q, const void *k, ab_shape s, int n_cluster
     const int nku_valid = (s.N + key_unit - 1) / key_unit;  // units holding a valid token
     cudaStream_t cs = (cudaStream_t)stream;
     void *kt = ws + L.kbar_terms;
-    cudaError_t e = ab::launch_meankey_units(k, kb, kt, BH, s.N, s.N_pad, s.d, key_unit, cs);
+    float *ks = reinterpret_cast<float *>(ws + L.kscale);
+    cudaError_t e = ab::launch_meankey_units(k, kb, kt, ks, BH, s.N, s.N_pad, s.d, key_unit, cs);
     if (e == cudaSuccess)
         e = ab::launch_kmeans(q, ce, cw, assign, BH, s.N, s.N_pad, s.d, n_clusters, iters,
                               dev_flag, cs);
     if (e == cudaSuccess)
-        e = ab::launch_score(ce, cw, kt, scores, BH, nqb, nku, nku_valid, s.d, n_clusters,
+        e = ab::launch_score(ce, cw, kt, ks, scores, BH, nqb, nku, nku_valid, s.d, n_clusters,
                              dev_flag, cs);
     return cuda_status(e);
 }

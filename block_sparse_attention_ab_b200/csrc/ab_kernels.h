@@ -14,11 +14,14 @@ ab_status status_of(cudaError_t e);
 // IBCS scoring (score_kernels.cu)
 // Device scratch of the scoring pass, each region 256-byte aligned: mean keys fp32
 // [BH][n_ku][d], centroids fp32 [BH][n_qb][C][d], cluster weights fp32 [BH][n_qb][C],
-// and the three bf16 terms of the mean keys [3][BH][n_ku][d]; n_ku = key units per head
-// (n_qb for 128-token key blocks).
+// the two fp16 terms of the scaled mean keys [2][BH][n_ku][d], and each mean key's
+// unscale factor fp32 [BH][n_ku_pad] (n_ku_pad = n_ku rounded up to 256); n_ku = key
+// units per head (n_qb for 128-token key blocks).
 struct ScoreLayout {
-    size_t kbar, cent, cw, kbar_terms, total;
+    size_t kbar, cent, cw, kbar_terms, kscale, total;
 };
+
+inline size_t kscale_stride(size_t nku) { return (nku + 255) / 256 * 256; }
 
 inline ScoreLayout score_layout(size_t BH, size_t nqb, size_t nku, size_t d, size_t C)
 {
@@ -28,19 +31,20 @@ inline ScoreLayout score_layout(size_t BH, size_t nqb, size_t nku, size_t d, siz
     L.cent = up(L.kbar + BH * nku * d * sizeof(float));
     L.cw = up(L.cent + BH * nqb * C * d * sizeof(float));
     L.kbar_terms = up(L.cw + BH * nqb * C * sizeof(float));
-    L.total = up(L.kbar_terms + 3 * BH * nku * d * 2);
+    L.kscale = up(L.kbar_terms + 2 * BH * nku * d * 2);
+    L.total = up(L.kscale + BH * kscale_stride(nku) * sizeof(float));
     return L;
 }
 
-cudaError_t launch_meankey(const void *k, float *kbar, void *kbar_terms, int BH, int N, int N_pad,
-                           int d, cudaStream_t st);
-cudaError_t launch_meankey_units(const void *k, float *kbar, void *kbar_terms, int BH, int N,
-                                 int N_pad, int d, int unit, cudaStream_t st);
+cudaError_t launch_meankey(const void *k, float *kbar, void *kbar_terms, float *kscale, int BH,
+                           int N, int N_pad, int d, cudaStream_t st);
+cudaError_t launch_meankey_units(const void *k, float *kbar, void *kbar_terms, float *kscale,
+                                 int BH, int N, int N_pad, int d, int unit, cudaStream_t st);
 cudaError_t launch_kmeans(const void *q, float *cent, float *cw, uint8_t *assign, int BH, int N,
                           int N_pad, int d, int C, int T, int *flag, cudaStream_t st);
-cudaError_t launch_score(const float *cent, const float *cw, const void *kbar_terms, float *scores,
-                         int BH, int nqb, int nkb, int nkb_valid, int d, int C, int *flag,
-                         cudaStream_t st);
+cudaError_t launch_score(const float *cent, const float *cw, const void *kbar_terms,
+                         const float *kscale, float *scores, int BH, int nqb, int nkb,
+                         int nkb_valid, int d, int C, int *flag, cudaStream_t st);
 
 // SIP / top-k selection (select_kernels.cu)
 // SIP over n_bh head pairs starting at global pair bh0 (b = pair / H, h = pair % H key

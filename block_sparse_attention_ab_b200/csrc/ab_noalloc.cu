@@ -75,14 +75,15 @@ ab_status score_noalloc(const void *q, const void *k, ab_shape s, int n_clusters
     float *ce = reinterpret_cast<float *>(ws + L.cent);
     float *cw = reinterpret_cast<float *>(ws + L.cw);
     void *kt = ws + L.kbar_terms;
+    float *ks = reinterpret_cast<float *>(ws + L.kscale);
     const int BH = s.B * s.H, nb = s.N_pad / AB_BLOCK;
     cudaStream_t cs = (cudaStream_t)stream;
-    cudaError_t e = ab::launch_meankey(k, kb, kt, BH, s.N, s.N_pad, s.d, cs);
+    cudaError_t e = ab::launch_meankey(k, kb, kt, ks, BH, s.N, s.N_pad, s.d, cs);
     if (e == cudaSuccess)
         e = ab::launch_kmeans(q, ce, cw, nullptr, BH, s.N, s.N_pad, s.d, n_clusters, iters,
                               dev_flag, cs);
     if (e == cudaSuccess)
-        e = ab::launch_score(ce, cw, kt, scores, BH, nb, nb, nb, s.d, n_clusters, dev_flag, cs);
+        e = ab::launch_score(ce, cw, kt, ks, scores, BH, nb, nb, nb, s.d, n_clusters, dev_flag, cs);
     return ab::status_of(e);
 }
 

@@ -4,6 +4,7 @@
 // s_j = sum_c w_c softmax_j(cent_c . kbar_j / sqrt(d)).
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "ab_device.cuh"
@@ -15,19 +16,6 @@ namespace ab {
 __device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 
-// Exact three-term bf16 split of fp32 values: x = hi + mid + lo with every term a bf16
-// (each subtraction is exact: the remainder of rounding to 8 significant bits has at
-// most 16, then at most 8). Products of two such splits with the terms of total
-// order <= 4 reproduce an fp32 product to about 2^-24 relative.
-__device__ __forceinline__ void split3(float x, __nv_bfloat16 &a, __nv_bfloat16 &b,
-                                       __nv_bfloat16 &c)
-{
-    a = __float2bfloat16_rn(x);
-    const float r = x - __bfloat162float(a);
-    b = __float2bfloat16_rn(r);
-    c = __float2bfloat16_rn(r - __bfloat162float(b));
-}
-
 // Round-to-nearest-even of a finite fp32 value to bf16 precision on its bit pattern:
 // add 0x7FFF plus the lowest kept bit, then clear the 16 dropped bits (integer pipe,
 // no conversion unit). The result is an fp32 bit pattern whose upper half is the bf16.
@@ -37,7 +25,11 @@ __device__ __forceinline__ uint32_t rne_bf16_bits(float x)
     return (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
 }
 
-// split3 on the integer pipe: the three terms as fp32 bit patterns (bf16 in the upper half).
+// Exact three-term bf16 split of an fp32 value on the integer pipe, x = hi + mid + lo
+// with every term a bf16 (each subtraction is exact: the remainder of rounding to 8
+// significant bits has at most 16, then at most 8); the terms come back as fp32 bit
+// patterns (bf16 in the upper half). Products of two such splits with the terms of total
+// order <= 4 reproduce an fp32 product to about 2^-24 relative.
 __device__ __forceinline__ void split3_bits(float x, uint32_t &a, uint32_t &b, uint32_t &c)
 {
     a = rne_bf16_bits(x);
@@ -62,21 +54,36 @@ __device__ __forceinline__ float rcp_approx(float n)
     return r;
 }
 
-// The same for 8 consecutive values, packed as three 16-byte rows (hi, mid, lo).
-__device__ __forceinline__ void split3x8(const float (&x)[8], uint4 (&t)[3])
+// Power-of-two scaling for the two-term fp16 split of the block-score operands: the
+// exponent e with amax * 2^e in [2^14, 2^15) for a vector whose largest magnitude is amax
+// (0 for a zero vector; clamped to [-126, 126]). The scaled components stay below the
+// fp16 maximum, and the low term of a component within 2^10 of amax is a normal fp16.
+__device__ __forceinline__ int scale_exponent(float amax)
 {
-    uint32_t a[4], b[4], c[4];
+    if (!(amax > 0.f)) return 0;
+    const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127;  // floor(log2 amax)
+    return min(126, max(-126, 14 - ex));
+}
+
+// 2^e as a float, e in [-126, 127]
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// Two-term fp16 split of y (|y| < 2^15): y = hi + lo + r with hi, lo fp16 and |r| at most
+// half an fp16 ulp of lo; y - hi is exact in fp32 (hi keeps the leading 11 bits of y).
+__device__ __forceinline__ uint32_t half2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+
+__device__ __forceinline__ void split2h_x8(const float (&y)[8], uint4 (&t)[2])
+{
+    uint32_t a[4], b[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const float x0 = x[2 * e], x1 = x[2 * e + 1];
-        a[e] = pack_bf16x2(x0, x1);
-        const float r0 = x0 - bf16_lo(a[e]), r1 = x1 - bf16_hi(a[e]);
-        b[e] = pack_bf16x2(r0, r1);
-        c[e] = pack_bf16x2(r0 - bf16_lo(b[e]), r1 - bf16_hi(b[e]));
+        const __half2 h = __floats2half2_rn(y[2 * e], y[2 * e + 1]);
+        const float2 hf = __half22float2(h);
+        a[e] = half2_bits(h);
+        b[e] = half2_bits(__floats2half2_rn(y[2 * e] - hf.x, y[2 * e + 1] - hf.y));
     }
     t[0] = make_uint4(a[0], a[1], a[2], a[3]);
     t[1] = make_uint4(b[0], b[1], b[2], b[3]);
-    t[2] = make_uint4(c[0], c[1], c[2], c[3]);
 }
 
 // Byte offset of the 16-byte chunk holding element (row, col) of a K-major tile stored
@@ -90,19 +97,22 @@ __device__ __forceinline__ int sw128_chunk(int row, int col, int panel_bytes)
 // ---------------------------------------------------------------------------------
 // Mean key: one CTA of 256 threads per (b, h, key block); 16-byte coalesced loads,
 // fp32 sums in a fixed order, divided by the block's valid-key count. Also writes the
-// three bf16 terms of each mean key (split3) for the tensor-core block score:
-// kbs[t][bh][j][i], t = 0 (hi), 1 (mid), 2 (lo).
+// mean key for the tensor-core block score: scaled by 2^e (scale_exponent of its largest
+// component) and split into two fp16 terms, kbs[t][bh][j][i] (t = 0 high, 1 low), with
+// the unscale factor 2^-e in kscale[bh][j] (row stride ks_stride).
 // ---------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) meankey_kernel(const __nv_bfloat16 *__restrict__ k,
                                                       float *__restrict__ kbar,
-                                                      __nv_bfloat16 *__restrict__ kbs, int N,
-                                                      int N_pad, int nkb)
+                                                      __half *__restrict__ kbs,
+                                                      float *__restrict__ kscale, int N,
+                                                      int N_pad, int nkb, int ks_stride)
 {
     constexpr int VEC = D / 8;         // 16-byte vectors per row
     constexpr int GROUPS = 256 / VEC;  // row groups
     constexpr int RPT = 128 / GROUPS;  // rows per thread
     __shared__ __align__(16) float part[GROUPS][D];
+    __shared__ float wmax[D / 32];
 
     const int blk = blockIdx.x;
     const int bh = blk / nkb, j = blk % nkb;
@@ -129,33 +139,50 @@ __global__ void __launch_bounds__(256) meankey_kernel(const __nv_bfloat16 *__res
     dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     __syncthreads();
+    // thread col < D owns column col (D <= 128 < 256 threads)
     const float inv = 1.0f / (float)nv;
-    const size_t term = (size_t)gridDim.x * D;
-    for (int col = tid; col < D; col += 256) {
-        float s = 0.f;
+    float m = 0.f;
+    if (tid < D) {
+        float sum = 0.f;
 #pragma unroll 8
-        for (int g = 0; g < GROUPS; ++g) s += part[g][col];
-        const float m = s * inv;
-        kbar[(size_t)blk * D + col] = m;
-        __nv_bfloat16 a, b, c;
-        split3(m, a, b, c);
-        kbs[(size_t)blk * D + col] = a;
-        kbs[term + (size_t)blk * D + col] = b;
-        kbs[2 * term + (size_t)blk * D + col] = c;
+        for (int g = 0; g < GROUPS; ++g) sum += part[g][tid];
+        m = sum * inv;
+        kbar[(size_t)blk * D + tid] = m;
+    }
+    // the mean key's largest |component|: warp maxima, then over the D / 32 warps
+    float amax = fabsf(m);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if (tid < D && (tid & 31) == 0) wmax[tid >> 5] = amax;
+    __syncthreads();
+    if (tid < D) {
+        amax = wmax[0];
+#pragma unroll
+        for (int w = 1; w < D / 32; ++w) amax = fmaxf(amax, wmax[w]);
+        const int e = scale_exponent(amax);
+        const float y = m * pow2f(e);
+        const __half hi = __float2half_rn(y);
+        const size_t term = (size_t)gridDim.x * D;
+        kbs[(size_t)blk * D + tid] = hi;
+        kbs[term + (size_t)blk * D + tid] = __float2half_rn(y - __half2float(hi));
+        if (tid == 0) kscale[(size_t)bh * ks_stride + j] = pow2f(-e);
     }
 }
 
 // ---------------------------------------------------------------------------------
 // Mean key of 4-token key units (the page's fine-grained selection unit): one CTA of
-// 256 threads per (b, h, 128-token span) = 32 units; thread (unit pair, 16-byte column
-// chunk) sums the unit's valid rows (fixed order) and writes the fp32 mean and its
-// three bf16 terms. A unit with no valid token gets 0.
+// 256 threads per (b, h, 128-token span) = 32 units; thread (unit, 16-byte column chunk)
+// sums the unit's valid rows (fixed order) and writes the fp32 mean, its two scaled fp16
+// terms and (for chunk 0) the unit's unscale factor, as meankey_kernel. The D / 8 threads
+// of a unit are adjacent lanes of one warp and share its largest |component| by shuffles.
+// A unit with no valid token gets 0 (factor 1).
 // ---------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) meankey4_kernel(const __nv_bfloat16 *__restrict__ k,
                                                        float *__restrict__ kbar,
-                                                       __nv_bfloat16 *__restrict__ kbs, int N,
-                                                       int N_pad, int nspan)
+                                                       __half *__restrict__ kbs,
+                                                       float *__restrict__ kscale, int N,
+                                                       int N_pad, int nspan, int ks_stride)
 {
     constexpr int CH = D / 8;                // 16-byte chunks per row
     constexpr int PER = 32 * CH / 256;       // (unit, chunk) pairs per thread
@@ -183,16 +210,27 @@ __global__ void __launch_bounds__(256) meankey4_kernel(const __nv_bfloat16 *__re
         }
         const float inv = nv > 0 ? 1.0f / (float)nv : 0.f;
         float m[8];
+        float amax = 0.f;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) m[c] = acc[c] * inv;
+        for (int c = 0; c < 8; ++c) {
+            m[c] = acc[c] * inv;
+            amax = fmaxf(amax, fabsf(m[c]));
+        }
+#pragma unroll
+        for (int o = CH / 2; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const int ex = scale_exponent(amax);
+        const float sc = pow2f(ex);
         const size_t o = ((size_t)bh * nku + u) * D + ch * 8;
         float4 *dst = reinterpret_cast<float4 *>(kbar + o);
         dst[0] = make_float4(m[0], m[1], m[2], m[3]);
         dst[1] = make_float4(m[4], m[5], m[6], m[7]);
-        uint4 t[3];
-        split3x8(m, t);
 #pragma unroll
-        for (int s3 = 0; s3 < 3; ++s3) *reinterpret_cast<uint4 *>(kbs + s3 * term + o) = t[s3];
+        for (int c = 0; c < 8; ++c) m[c] *= sc;
+        uint4 t[2];
+        split2h_x8(m, t);
+        *reinterpret_cast<uint4 *>(kbs + o) = t[0];
+        *reinterpret_cast<uint4 *>(kbs + term + o) = t[1];
+        if (ch == 0) kscale[(size_t)bh * ks_stride + u] = pow2f(-ex);
     }
 }
 
@@ -202,7 +240,7 @@ __global__ void __launch_bounds__(256) meankey4_kernel(const __nv_bfloat16 *__re
 // N read as zero) and stay in shared memory for all T iterations. Each iteration runs
 // two single-CTA tcgen05 GEMMs with fp32 accumulators in TMEM:
 //   assign: G = Q B^T (M = 128 queries, N = 32, K = d): rows 8t + c of B hold term t
-//           (split3) of fp32 centroid c, rows 24..31 are zero, so q . c =
+//           (split3_bits) of fp32 centroid c, rows 24..31 are zero, so q . c =
 //           G[q][c] + G[q][8 + c] + G[q][16 + c] is the bf16 query times the fp32
 //           centroid; distance |c|^2 - 2 q.c (|q|^2 is common), argmin with ties to
 //           the lowest cluster; thread t reads TMEM lane t = query t;
@@ -499,11 +537,14 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
 // blocks); its 128 TMEM lanes are the centroid rows r = 8 * (query block) + c
 // (clusters c >= C and query blocks past the end are zero rows with weight 0).
 // Logits L[r][j] = cent_r . kbar_j are computed as 128 x 64 x d tcgen05 GEMMs over
-// tiles of 64 key blocks, with both fp32 operands split exactly into three bf16 terms
-// (split3) and the six term products of total order <= 4 accumulated in fp32: the
-// omitted terms are below 2^-24 relative, so the logits carry fp32 accuracy. The
-// centroid terms are built once in shared memory by all threads; the key terms are
-// written by the mean-key kernel and arrive by TMA.
+// tiles of 64 key blocks. Both fp32 operands are scaled by powers of two (each centroid
+// row and each mean key so that its largest component lies in [2^14, 2^15)) and split
+// into two fp16 terms, hi + lo, which hold 22 significant bits; the three products
+// hi.hi + hi.lo + lo.hi accumulate in fp32, the omitted lo.lo and the split's remainder
+// lie near 2^-22 of each product, and the exact power-of-two unscaling enters the
+// epilogue's per-row and per-column factors. The centroid terms are built once in shared
+// memory by all threads; the key terms and factors are written by the mean-key kernel,
+// the terms arrive by TMA.
 // Key blocks are processed in chunks of 256 (one TMEM buffer of 256 columns; two
 // buffers). With n_kb <= 256 one pass suffices: each row's softmax max and sum and
 // then the scores come from the logits held in TMEM. With more chunks, a first pass
@@ -522,28 +563,29 @@ struct ScSmem {
     static constexpr int kPanels = D / 64;
     static constexpr int kATerm = kPanels * 16384;           // one term of the 128 centroid rows
     static constexpr int kBTerm = kPanels * 8192;            // one term of 64 mean keys
-    static constexpr int kStageBytes = 3 * kBTerm;
-    static constexpr int kStages = D == 128 ? 2 : 4;
+    static constexpr int kStageBytes = 2 * kBTerm;
+    static constexpr int kStages = D == 128 ? 4 : 8;
     static constexpr int kA = 0;
-    static constexpr int kB = kA + 3 * kATerm;
+    static constexpr int kB = kA + 2 * kATerm;
     static constexpr int kBar = kB + kStages * kStageBytes;
     // barriers: full[S], empty[S], tfull[2], tempty[2], drain
     static constexpr int kNumBars = 2 * kStages + 5;
-    static constexpr int kMisc = kBar + kNumBars * 8;       // TMEM base, abort flag
+    static constexpr int kRows = kBar + kNumBars * 8;  // float [2][128]: 2^e, 2^-e per row
+    static constexpr int kMisc = kRows + 2 * 128 * 4;  // TMEM base, abort flag
     static constexpr int kBytes = kMisc + 8;
     static constexpr int kAlloc = kBytes + 1024;
 };
 
-// the six term products (a, b) of total order <= 4, terms numbered 0 (hi), 1, 2 (lo):
-// (0,0) (0,1) (1,0) (0,2) (1,1) (2,0)
-__host__ __device__ constexpr int prod_term_a(int pr) { return pr == 2 || pr == 4 ? 1 : (pr == 5 ? 2 : 0); }
-__host__ __device__ constexpr int prod_term_b(int pr) { return pr == 1 || pr == 4 ? 1 : (pr == 3 ? 2 : 0); }
+// the three term products (a, b), terms numbered 0 (hi), 1 (lo): (0,0) (0,1) (1,0)
+__host__ __device__ constexpr int prod_term_a(int pr) { return pr == 2 ? 1 : 0; }
+__host__ __device__ constexpr int prod_term_b(int pr) { return pr == 1 ? 1 : 0; }
 
 template <int D>
 __global__ void __launch_bounds__(kScThreads, 1)
     score_kernel(const __grid_constant__ CUtensorMap tmKB, const float *__restrict__ cent,
-                 const float *__restrict__ cw, int BH, int nqb, int nkb, int nkb_valid, int C,
-                 float scale_log2, float *__restrict__ scores, int *flag)
+                 const float *__restrict__ cw, const float *__restrict__ kscale, int ks_stride,
+                 int BH, int nqb, int nkb, int nkb_valid, int C, float scale_log2,
+                 float *__restrict__ scores, int *flag)
 {
     using L = ScSmem<D>;
     extern __shared__ uint8_t sc_raw[];
@@ -559,6 +601,25 @@ __global__ void __launch_bounds__(kScThreads, 1)
     const int g = blockIdx.x, bh = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+    // each centroid row's scale 2^e and unscale 2^-e (zero rows: 1)
+    float *row_mul = reinterpret_cast<float *>(smem + L::kRows);
+    float *row_unscale = row_mul + 128;
+    if (tid < 128) {
+        const int qb = g * 16 + (tid >> 3), c = tid & 7;
+        float amax = 0.f;
+        if (qb < nqb && c < C) {
+            const float4 *src = reinterpret_cast<const float4 *>(cent + (((size_t)bh * nqb + qb) * C + c) * D);
+#pragma unroll 8
+            for (int i = 0; i < D / 4; ++i) {
+                const float4 u = __ldg(src + i);
+                amax = fmaxf(fmaxf(amax, fmaxf(fabsf(u.x), fabsf(u.y))), fmaxf(fabsf(u.z), fabsf(u.w)));
+            }
+        }
+        const int e = scale_exponent(amax);
+        row_mul[tid] = pow2f(e);
+        row_unscale[tid] = pow2f(-e);
+    }
+    __syncthreads();
     // centroid terms (A operand), all threads
     {
         constexpr int CH = D / 8;
@@ -570,16 +631,17 @@ __global__ void __launch_bounds__(kScThreads, 1)
                 const float4 *src = reinterpret_cast<const float4 *>(
                     cent + (((size_t)bh * nqb + qb) * C + c) * D + k0);
                 const float4 u = __ldg(src), v = __ldg(src + 1);
-                x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-                x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+                const float sc = row_mul[row];
+                x[0] = u.x * sc; x[1] = u.y * sc; x[2] = u.z * sc; x[3] = u.w * sc;
+                x[4] = v.x * sc; x[5] = v.y * sc; x[6] = v.z * sc; x[7] = v.w * sc;
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) x[e] = 0.f;
             }
-            uint4 t[3];
-            split3x8(x, t);
+            uint4 t[2];
+            split2h_x8(x, t);
 #pragma unroll
-            for (int s = 0; s < 3; ++s)
+            for (int s = 0; s < 2; ++s)
                 *reinterpret_cast<uint4 *>(smem + L::kA + s * L::kATerm + sw128_chunk(row, k0, 16384)) = t[s];
         }
     }
@@ -631,7 +693,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
                     uint8_t *dst = smem + L::kB + s * L::kStageBytes;
                     mbar_arrive_expect_tx(&full[s], L::kStageBytes);
 #pragma unroll
-                    for (int t = 0; t < 3; ++t)
+                    for (int t = 0; t < 2; ++t)
 #pragma unroll
                         for (int h = 0; h < L::kPanels; ++h)
                             tma_load_3d(dst + t * L::kBTerm + h * 8192, &tmKB, &full[s], h * 64,
@@ -653,7 +715,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
         // ------------------------------- MMA issuer -------------------------------
         const uint64_t a0 = smem_desc_sw128(smem_u32(smem + L::kA), 16, 1024);
         const uint64_t b0 = smem_desc_sw128(smem_u32(smem + L::kB), 16, 1024);
-        constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
+        constexpr uint32_t idesc = idesc_f16_f32(128, 64, 0, 0);
         int pos = 0;
         bool ok = true;
         for (int j = 0; j < njobs && ok; ++j) {
@@ -676,7 +738,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
                 const uint64_t bs = b0 + (uint64_t)((s * L::kStageBytes) >> 4);
                 if (elect_one()) {
 #pragma unroll
-                    for (int pr = 0; pr < 6; ++pr) {
+                    for (int pr = 0; pr < 3; ++pr) {
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const int ta = prod_term_a(pr), tb = prod_term_b(pr);
@@ -711,6 +773,23 @@ __global__ void __launch_bounds__(kScThreads, 1)
         const float wr = (row_ok && c < C) ? __ldg(cw + ((size_t)bh * nqb + qb) * C + c) : 0.f;
         float *dst = scores + ((size_t)bh * nqb + (row_ok ? qb : 0)) * nkb;
         const uint32_t t_lane = tmem + ((uint32_t)(qd * 32) << 16);
+        // x = L * 2^-(e_row + e_j) * log2(e) / sqrt(d): the logit in log2 units from the
+        // scaled product, with the 32 column factors of a TMEM slice loaded together
+        // (every lane reads the same addresses; the factor rows are padded to a multiple
+        // of the chunk, so a slice never reads past them)
+        const float rs = row_unscale[row] * scale_log2;
+        const float *ks_row = kscale + (size_t)bh * ks_stride;
+        auto factors = [&](int col0, float (&f)[32]) {
+            const float4 *src = reinterpret_cast<const float4 *>(ks_row + col0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 u = __ldg(src + q);
+                f[4 * q + 0] = u.x * rs;
+                f[4 * q + 1] = u.y * rs;
+                f[4 * q + 2] = u.z * rs;
+                f[4 * q + 3] = u.w * rs;
+            }
+        };
         const int r8 = lane & 7;
         const bool b4 = (r8 & 4) != 0, b2 = (r8 & 2) != 0, b1 = (r8 & 1) != 0;
         float m = -INFINITY, z = 0.f, coef = 0.f;
@@ -731,22 +810,26 @@ __global__ void __launch_bounds__(kScThreads, 1)
                 float mx = m;
                 for (int sl = 0; sl < nvsl; ++sl) {
                     uint32_t v[32];
+                    float f[32];
                     tmem_ld32(tb + sl * 32, v);
+                    factors(c0 + sl * 32, f);
                     tmem_wait_ld();
                     const int lim = nvcols - sl * 32;
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        if (i < lim) mx = fmaxf(mx, __uint_as_float(v[i]) * scale_log2);
+                        if (i < lim) mx = fmaxf(mx, __uint_as_float(v[i]) * f[i]);
                 }
                 float zz = m == -INFINITY ? 0.f : z * fast_exp2(m - mx);
                 for (int sl = 0; sl < nvsl; ++sl) {
                     uint32_t v[32];
+                    float f[32];
                     tmem_ld32(tb + sl * 32, v);
+                    factors(c0 + sl * 32, f);
                     tmem_wait_ld();
                     const int lim = nvcols - sl * 32;
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        if (i < lim) zz += fast_exp2(fmaf(__uint_as_float(v[i]), scale_log2, -mx));
+                        if (i < lim) zz += fast_exp2(fmaf(__uint_as_float(v[i]), f[i], -mx));
                 }
                 m = mx;
                 z = zz;
@@ -755,7 +838,9 @@ __global__ void __launch_bounds__(kScThreads, 1)
             if (nch == 1 || j >= nch) {
                 for (int sl = 0; sl < nsl; ++sl) {
                     uint32_t v[32];
+                    float f[32];
                     tmem_ld32(tb + sl * 32, v);
+                    factors(c0 + sl * 32, f);
                     tmem_wait_ld();
 #pragma unroll
                     for (int q8 = 0; q8 < 4; ++q8) {
@@ -763,7 +848,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             e[i] = c0 + sl * 32 + q8 * 8 + i < nkb_valid
-                                       ? coef * fast_exp2(fmaf(__uint_as_float(v[q8 * 8 + i]), scale_log2, -m))
+                                       ? coef * fast_exp2(fmaf(__uint_as_float(v[q8 * 8 + i]), f[q8 * 8 + i], -m))
                                        : 0.f;
                         // sum over the 8 rows (lanes) of this query block; lane r8 ends
                         // with column q8 * 8 + r8
@@ -805,30 +890,36 @@ __global__ void __launch_bounds__(kScThreads, 1)
 // ---------------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------------
-cudaError_t launch_meankey_units(const void *k, float *kbar, void *kbar_terms, int BH, int N,
-                                 int N_pad, int d, int unit, cudaStream_t st)
+cudaError_t launch_meankey_units(const void *k, float *kbar, void *kbar_terms, float *kscale,
+                                 int BH, int N, int N_pad, int d, int unit, cudaStream_t st)
 {
-    if (unit != 4) return launch_meankey(k, kbar, kbar_terms, BH, N, N_pad, d, st);
+    if (unit != 4) return launch_meankey(k, kbar, kbar_terms, kscale, BH, N, N_pad, d, st);
     const int nspan = N_pad / 128;
+    const int ks_stride = (int)kscale_stride((size_t)N_pad / 4);
     const dim3 grid((unsigned)(BH * nspan));
-    __nv_bfloat16 *kbs = static_cast<__nv_bfloat16 *>(kbar_terms);
+    __half *kbs = static_cast<__half *>(kbar_terms);
     if (d == 128)
-        meankey4_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, N, N_pad, nspan);
+        meankey4_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, kscale, N, N_pad,
+                                                   nspan, ks_stride);
     else
-        meankey4_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, N, N_pad, nspan);
+        meankey4_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, kscale, N, N_pad,
+                                                  nspan, ks_stride);
     return cudaGetLastError();
 }
 
-cudaError_t launch_meankey(const void *k, float *kbar, void *kbar_terms, int BH, int N, int N_pad,
-                           int d, cudaStream_t st)
+cudaError_t launch_meankey(const void *k, float *kbar, void *kbar_terms, float *kscale, int BH,
+                           int N, int N_pad, int d, cudaStream_t st)
 {
     const int nkb = N_pad / 128;
+    const int ks_stride = (int)kscale_stride((size_t)nkb);
     const dim3 grid((unsigned)(BH * nkb));
-    __nv_bfloat16 *kbs = static_cast<__nv_bfloat16 *>(kbar_terms);
+    __half *kbs = static_cast<__half *>(kbar_terms);
     if (d == 128)
-        meankey_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, N, N_pad, nkb);
+        meankey_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, kscale, N, N_pad,
+                                                  nkb, ks_stride);
     else
-        meankey_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, N, N_pad, nkb);
+        meankey_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, kscale, N, N_pad,
+                                                 nkb, ks_stride);
     return cudaGetLastError();
 }
 
@@ -859,11 +950,13 @@ cudaError_t launch_kmeans(const void *q, float *cent, float *cw, uint8_t *assign
 
 template <int D>
 static cudaError_t launch_score_t(const float *cent, const float *cw, const void *kbar_terms,
-                                  float *scores, int BH, int nqb, int nkb, int nkb_valid, int C,
-                                  int *flag, cudaStream_t st)
+                                  const float *kscale, float *scores, int BH, int nqb, int nkb,
+                                  int nkb_valid, int C, int *flag, cudaStream_t st)
 {
     CUtensorMap tm;
-    if (!make_tmap_bf16_3d(&tm, kbar_terms, D, (uint64_t)nkb, (uint64_t)3 * BH, (uint64_t)D * 2,
+    // the fp16 terms travel as 2-byte elements (the map's type only sets the element size
+    // and the zero fill)
+    if (!make_tmap_bf16_3d(&tm, kbar_terms, D, (uint64_t)nkb, (uint64_t)2 * BH, (uint64_t)D * 2,
                            (uint64_t)nkb * D * 2, 64, 64))
         return cudaErrorInvalidValue;
     const int smem = ScSmem<D>::kAlloc;
@@ -872,19 +965,19 @@ static cudaError_t launch_score_t(const float *cent, const float *cw, const void
     if (e != cudaSuccess) return e;
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     const dim3 grid((unsigned)((nqb + 15) / 16), (unsigned)BH);
-    score_kernel<D><<<grid, kScThreads, smem, st>>>(tm, cent, cw, BH, nqb, nkb, nkb_valid, C,
-                                                    scale_log2, scores, flag);
+    score_kernel<D><<<grid, kScThreads, smem, st>>>(tm, cent, cw, kscale, (int)kscale_stride((size_t)nkb), BH,
+                                                    nqb, nkb, nkb_valid, C, scale_log2, scores, flag);
     return cudaGetLastError();
 }
 
-cudaError_t launch_score(const float *cent, const float *cw, const void *kbar_terms, float *scores,
-                         int BH, int nqb, int nkb, int nkb_valid, int d, int C, int *flag,
-                         cudaStream_t st)
+cudaError_t launch_score(const float *cent, const float *cw, const void *kbar_terms,
+                         const float *kscale, float *scores, int BH, int nqb, int nkb,
+                         int nkb_valid, int d, int C, int *flag, cudaStream_t st)
 {
-    return d == 128 ? launch_score_t<128>(cent, cw, kbar_terms, scores, BH, nqb, nkb, nkb_valid, C,
-                                          flag, st)
-                    : launch_score_t<64>(cent, cw, kbar_terms, scores, BH, nqb, nkb, nkb_valid, C,
-                                         flag, st);
+    return d == 128 ? launch_score_t<128>(cent, cw, kbar_terms, kscale, scores, BH, nqb, nkb,
+                                          nkb_valid, C, flag, st)
+                    : launch_score_t<64>(cent, cw, kbar_terms, kscale, scores, BH, nqb, nkb,
+                                         nkb_valid, C, flag, st);
 }
 
 }  // namespace ab

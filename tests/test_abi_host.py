@@ -51,9 +51,10 @@ def test_workspace_size(L):
     n = ctypes.c_size_t(0)
     assert L.ab_score_workspace_size(shape(), 8, ctypes.byref(n)) == 0
     nb = 8
-    # mean keys, centroids, cluster weights (fp32) and the three bf16 terms of the mean keys
-    need = 2 * nb * 64 * 4 + 2 * nb * 8 * 64 * 4 + 2 * nb * 8 * 4 + 3 * 2 * nb * 64 * 2
-    assert need <= n.value <= need + 4 * 256
+    # mean keys, centroids, cluster weights (fp32), the two fp16 terms of the scaled mean
+    # keys and their unscale factors (fp32 rows padded to 256 entries)
+    need = 2 * nb * 64 * 4 + 2 * nb * 8 * 64 * 4 + 2 * nb * 8 * 4 + 2 * 2 * nb * 64 * 2 + 2 * 256 * 4
+    assert need <= n.value <= need + 5 * 256
     assert L.ab_score_workspace_size(shape(), 9, ctypes.byref(n)) == 4
     assert n.value == 0
     assert L.ab_score_workspace_size(shape(N=1024, N_pad=1000), 8, ctypes.byref(n)) == 2
@@ -169,9 +170,10 @@ def test_unit_workspace_size(L):
     n = ctypes.c_size_t(0)
     assert L.ab_score_units_workspace_size(shape(), 8, 4, ctypes.byref(n)) == 0
     nqb, nku = 8, 256
-    # mean keys [2, nku, 64] fp32, centroids and weights per query block, bf16 key terms
-    need = 2 * nku * 64 * 4 + 2 * nqb * 8 * 64 * 4 + 2 * nqb * 8 * 4 + 3 * 2 * nku * 64 * 2
-    assert need <= n.value <= need + 4 * 256
+    # mean keys [2, nku, 64] fp32, centroids and weights per query block, fp16 key terms,
+    # unscale factors
+    need = 2 * nku * 64 * 4 + 2 * nqb * 8 * 64 * 4 + 2 * nqb * 8 * 4 + 2 * 2 * nku * 64 * 2 + 2 * 256 * 4
+    assert need <= n.value <= need + 5 * 256
     m = ctypes.c_size_t(0)
     assert L.ab_score_units_workspace_size(shape(), 8, 128, ctypes.byref(m)) == 0
     L.ab_score_workspace_size(shape(), 8, ctypes.byref(n))
