@@ -40,7 +40,7 @@ __device__ __forceinline__ uint4 philox_4x32_10(uint4 c, uint32_t k0, uint32_t k
 
 __device__ __forceinline__ bool score_ok(float v) { return v >= 0.f && v <= 2.f; }
 
-// exact: v in [0, 2] -> floor(v * 2^50) < 2^52
+// exact: v in [0, 2] -> floor(v * 2^50) < 2^52 (the product is exact in double)
 __device__ __forceinline__ uint64_t fixed50(float v)
 {
     return __double2ull_rz((double)v * 1125899906842624.0);
@@ -50,6 +50,20 @@ __device__ __forceinline__ uint64_t fixed50(float v)
 __device__ __forceinline__ bool mul_ge(uint64_t k, uint64_t u, uint64_t R)
 {
     return __umul64hi(k, u) != 0ull || k * u >= R;
+}
+
+// The least u with k u >= R (k >= 1), so that the test k u_j >= R of a pass becomes
+// u_j >= thr: a double quotient (within a few units of the exact one: R / k < 2^64
+// carries a relative error near 2^-52) corrected by the exact 128-bit test. k = 0: 0
+// when R = 0, else no u qualifies.
+__device__ __forceinline__ uint64_t ceil_div_threshold(uint64_t R, uint64_t k)
+{
+    if (k == 0) return R == 0 ? 0ull : ~0ull;
+    const double qd = __ull2double_rn(R) / __ull2double_rn(k);
+    uint64_t q = qd >= 18446744073709549568.0 ? ~0ull : __double2ull_rz(qd);
+    while (q > 0 && mul_ge(k, q - 1, R)) --q;
+    while (!mul_ge(k, q, R)) ++q;
+    return q;
 }
 
 template <typename T>
@@ -89,6 +103,11 @@ __device__ Sum3 block_sum3(unsigned long long a, unsigned long long b, unsigned 
     return s;
 }
 
+// kCacheU: the row's u_j stay in shared memory after pass 0 (rows of up to
+// kSipCacheMax entries); otherwise each pass recomputes them from the scores.
+constexpr int kSipCacheMax = 8192;
+
+template <bool kCacheU>
 __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restrict__ scores,
                                                          int H, int bh0, int nqb, int nkb, int K,
                                                          uint32_t key0, uint32_t key1,
@@ -97,8 +116,11 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
                                                          float *__restrict__ w,
                                                          double *__restrict__ p_out, int *flag)
 {
-    // nkb bytes (0 = out, 1 = saturated, 2 = joining), then the keep bits of the draws
-    extern __shared__ __align__(16) uint8_t inS[];
+    // kCacheU: u_j as uint64 [nkb]; then nkb bytes (0 = out, 1 = saturated, 2 = joining),
+    // then the keep bits of the draws
+    extern __shared__ __align__(16) uint8_t sip_sh[];
+    uint64_t *u_sh = reinterpret_cast<uint64_t *>(sip_sh);
+    uint8_t *inS = sip_sh + (kCacheU ? (size_t)nkb * 8 : 0);
     __shared__ unsigned long long red[kSelWarps][3];
     __shared__ int wtot[kSelWarps];
 
@@ -110,6 +132,7 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
     const int qb = (int)(row % nqb);
     const float *s = scores + row * nkb;
     const int tid = threadIdx.x;
+    auto u_of = [&](int j) -> uint64_t { return kCacheU ? u_sh[j] : fixed50(s[j]); };
 
     // pass 0: validate, U = sum u_j, number of positive u_j. U is summed exactly as
     // U_hi = sum (u_j >> 12) and U_lo = sum (u_j & 0xfff) (neither can overflow), and a row
@@ -123,6 +146,7 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
             continue;
         }
         const uint64_t u = fixed50(v);
+        if (kCacheU) u_sh[j] = u;
         u_hi += u >> 12;
         u_lo += u & 0xfffull;
         counts += u > 0;
@@ -148,18 +172,20 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
     const bool all_positive_kept = npos <= (unsigned long long)K;
     uint64_t k_rest = 0, R = 0;
     if (all_positive_kept) {
-        for (int j = tid; j < nkb; j += kSelThreads) inS[j] = fixed50(s[j]) > 0 ? 1 : 0;
+        for (int j = tid; j < nkb; j += kSelThreads) inS[j] = u_of(j) > 0 ? 1 : 0;
         __syncthreads();
     } else {
         unsigned long long sizeS = 0, sumS = 0;
         for (;;) {
             k_rest = (uint64_t)K - sizeS;
             R = U - sumS;
+            // (K - |S|) u_j >= R  <=>  u_j >= ceil(R / (K - |S|))
+            const uint64_t thr = ceil_div_threshold(R, k_rest);
             unsigned long long add_n = 0, add_u = 0;
             for (int j = tid; j < nkb; j += kSelThreads) {
                 if (inS[j]) continue;
-                const uint64_t u = fixed50(s[j]);
-                if (mul_ge(k_rest, u, R)) {
+                const uint64_t u = u_of(j);
+                if (u >= thr) {
                     inS[j] = 2;
                     ++add_n;
                     add_u += u;
@@ -190,7 +216,7 @@ __global__ void __launch_bounds__(kSelThreads) sip_kernel(const float *__restric
     auto prob = [&](int j) -> double {  // p_j of entry j
         if (inS[j] == 1) return 1.0;
         if (all_positive_kept) return 0.0;
-        const uint64_t u = fixed50(s[j]);
+        const uint64_t u = u_of(j);
         return u > 0 ? __ull2double_rn(k_rest * u) / Rd : 0.0;
     };
     int kept_here = 0;
@@ -403,11 +429,21 @@ cudaError_t launch_sip(const float *scores, int n_bh, int H, int bh0, int nqb, i
                        cudaStream_t st)
 {
     const unsigned rows = (unsigned)((size_t)n_bh * nqb);
-    const size_t smem = (size_t)((nkb + 15) & ~15) + (size_t)(nkb + 255) / 256 * 32 + 32;
-    cudaError_t e = allow_smem(sip_kernel, smem);
-    if (e != cudaSuccess) return e;
-    sip_kernel<<<rows, kSelThreads, smem, st>>>(scores, H, bh0, nqb, nkb, K, (uint32_t)seed,
-                                                (uint32_t)(seed >> 32), idx, cnt, w, p, flag);
+    const size_t flags = (size_t)((nkb + 15) & ~15) + (size_t)(nkb + 255) / 256 * 32 + 32;
+    const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    cudaError_t e;
+    if (nkb <= kSipCacheMax) {
+        const size_t smem = (size_t)nkb * 8 + flags;
+        e = allow_smem(sip_kernel<true>, smem);
+        if (e != cudaSuccess) return e;
+        sip_kernel<true><<<rows, kSelThreads, smem, st>>>(scores, H, bh0, nqb, nkb, K, k0, k1, idx,
+                                                          cnt, w, p, flag);
+    } else {
+        e = allow_smem(sip_kernel<false>, flags);
+        if (e != cudaSuccess) return e;
+        sip_kernel<false><<<rows, kSelThreads, flags, st>>>(scores, H, bh0, nqb, nkb, K, k0, k1, idx,
+                                                            cnt, w, p, flag);
+    }
     return cudaGetLastError();
 }
 
