@@ -571,7 +571,10 @@ struct ScSmem {
     // barriers: full[S], empty[S], tfull[2], tempty[2], drain
     static constexpr int kNumBars = 2 * kStages + 5;
     static constexpr int kRows = kBar + kNumBars * 8;  // float [2][128]: 2^e, 2^-e per row
-    static constexpr int kMisc = kRows + 2 * 128 * 4;  // TMEM base, abort flag
+    // float [4 warps][2 jobs][256]: column factors, read as float4 (16-byte aligned)
+    static constexpr int kFac = (kRows + 2 * 128 * 4 + 15) & ~15;
+    static constexpr int kMisc = kFac + 4 * 2 * 256 * 4;  // TMEM base, abort flag
+    static_assert(kFac % 16 == 0 && kB % 1024 == 0, "shared-memory layout alignment");
     static constexpr int kBytes = kMisc + 8;
     static constexpr int kAlloc = kBytes + 1024;
 };
@@ -774,16 +777,25 @@ __global__ void __launch_bounds__(kScThreads, 1)
         float *dst = scores + ((size_t)bh * nqb + (row_ok ? qb : 0)) * nkb;
         const uint32_t t_lane = tmem + ((uint32_t)(qd * 32) << 16);
         // x = L * 2^-(e_row + e_j) * log2(e) / sqrt(d): the logit in log2 units from the
-        // scaled product, with the 32 column factors of a TMEM slice loaded together
-        // (every lane reads the same addresses; the factor rows are padded to a multiple
-        // of the chunk, so a slice never reads past them)
+        // scaled product. Each warp copies a job's 256 column factors into its own shared
+        // buffer (one per job parity) before it waits for the job's logits, and every
+        // lane then reads the 32 factors of a TMEM slice from there (broadcast reads; the
+        // factor rows are padded to a multiple of the chunk, so no read passes them).
         const float rs = row_unscale[row] * scale_log2;
         const float *ks_row = kscale + (size_t)bh * ks_stride;
-        auto factors = [&](int col0, float (&f)[32]) {
+        float *fac_w = reinterpret_cast<float *>(smem + L::kFac) + qd * 2 * 256;
+        auto stage_factors = [&](int job, int col0) {
             const float4 *src = reinterpret_cast<const float4 *>(ks_row + col0);
+            float4 *dst = reinterpret_cast<float4 *>(fac_w + (job & 1) * 256);
+            dst[lane] = __ldg(src + lane);
+            dst[32 + lane] = __ldg(src + 32 + lane);
+            __syncwarp();
+        };
+        auto factors = [&](int job, int sl, float (&f)[32]) {
+            const float4 *src = reinterpret_cast<const float4 *>(fac_w + (job & 1) * 256 + sl * 32);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const float4 u = __ldg(src + q);
+                const float4 u = src[q];
                 f[4 * q + 0] = u.x * rs;
                 f[4 * q + 1] = u.y * rs;
                 f[4 * q + 2] = u.z * rs;
@@ -796,6 +808,8 @@ __global__ void __launch_bounds__(kScThreads, 1)
         for (int j = 0; j < njobs; ++j) {
             const int buf = j & 1;
             const int ch = j < nch ? j : j - nch;
+            // this warp read the buffer of parity j & 1 for job j - 2, which it has finished
+            stage_factors(j, ch * kScChunk);
             if (!wait(&tfull[buf], (j >> 1) & 1)) break;
             tc_fence_after();
             const int c0 = ch * kScChunk;
@@ -812,7 +826,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
                     uint32_t v[32];
                     float f[32];
                     tmem_ld32(tb + sl * 32, v);
-                    factors(c0 + sl * 32, f);
+                    factors(j, sl, f);
                     tmem_wait_ld();
                     const int lim = nvcols - sl * 32;
 #pragma unroll
@@ -824,7 +838,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
                     uint32_t v[32];
                     float f[32];
                     tmem_ld32(tb + sl * 32, v);
-                    factors(c0 + sl * 32, f);
+                    factors(j, sl, f);
                     tmem_wait_ld();
                     const int lim = nvcols - sl * 32;
 #pragma unroll
@@ -840,7 +854,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
                     uint32_t v[32];
                     float f[32];
                     tmem_ld32(tb + sl * 32, v);
-                    factors(c0 + sl * 32, f);
+                    factors(j, sl, f);
                     tmem_wait_ld();
 #pragma unroll
                     for (int q8 = 0; q8 < 4; ++q8) {
