@@ -551,10 +551,13 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
 // accumulates each row's max and sum online and a second pass recomputes the logits
 // and writes s_j = sum_c (w_c / Z_c) 2^(L'_cj - m_c) (L' in log2 units), the sum over
 // a query block's 8 centroid rows taken across 8 lanes (butterfly reduce-scatter).
-// Warp 0: TMA producer; warp 1: TMEM owner and MMA issuer; warps 2..5: epilogue
-// (warp w reads TMEM lanes 32 (w mod 4) .. +31).
+// Warp 0: TMA producer; warp 1: TMEM owner and MMA issuer; warps 2..9: epilogue, two
+// per TMEM lane group (warp w reads lanes 32 (w mod 4) .. +31 and takes every other 32-
+// column slice of a chunk, starting at slice (w - 2) / 4). Each keeps its own row max and
+// sum over its slices through the statistics pass; the two of a lane group merge them
+// once, where the output pass begins.
 // ---------------------------------------------------------------------------------
-constexpr int kScThreads = 192;
+constexpr int kScThreads = 320;
 constexpr int kScChunk = 256;
 constexpr int kScTmemCols = 512;
 
@@ -571,9 +574,10 @@ struct ScSmem {
     // barriers: full[S], empty[S], tfull[2], tempty[2], drain
     static constexpr int kNumBars = 2 * kStages + 5;
     static constexpr int kRows = kBar + kNumBars * 8;  // float [2][128]: 2^e, 2^-e per row
-    // float [4 warps][2 jobs][256]: column factors, read as float4 (16-byte aligned)
+    // float [8 warps][2 jobs][256]: column factors, read as float4 (16-byte aligned)
     static constexpr int kFac = (kRows + 2 * 128 * 4 + 15) & ~15;
-    static constexpr int kMisc = kFac + 4 * 2 * 256 * 4;  // TMEM base, abort flag
+    static constexpr int kXch = kFac + 8 * 2 * 256 * 4;  // float [2][2][128]: (m, z) per half
+    static constexpr int kMisc = kXch + 2 * 2 * 128 * 4;  // TMEM base, abort flag
     static_assert(kFac % 16 == 0 && kB % 1024 == 0, "shared-memory layout alignment");
     static constexpr int kBytes = kMisc + 8;
     static constexpr int kAlloc = kBytes + 1024;
@@ -655,7 +659,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 128);
+            mbar_init(&tempty[b], 256);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -770,6 +774,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
     } else {
         // -------------------------------- epilogue --------------------------------
         const int qd = warp & 3;
+        const int half = (warp - 2) >> 2;  // slices half, half + 2, .. of each chunk
         const int row = qd * 32 + lane;
         const int qb = g * 16 + (row >> 3), c = row & 7;
         const bool row_ok = qb < nqb;
@@ -783,12 +788,12 @@ __global__ void __launch_bounds__(kScThreads, 1)
         // factor rows are padded to a multiple of the chunk, so no read passes them).
         const float rs = row_unscale[row] * scale_log2;
         const float *ks_row = kscale + (size_t)bh * ks_stride;
-        float *fac_w = reinterpret_cast<float *>(smem + L::kFac) + qd * 2 * 256;
+        float *fac_w = reinterpret_cast<float *>(smem + L::kFac) + (warp - 2) * 2 * 256;
         auto stage_factors = [&](int job, int col0) {
             const float4 *src = reinterpret_cast<const float4 *>(ks_row + col0);
-            float4 *dst = reinterpret_cast<float4 *>(fac_w + (job & 1) * 256);
-            dst[lane] = __ldg(src + lane);
-            dst[32 + lane] = __ldg(src + 32 + lane);
+            float4 *fdst = reinterpret_cast<float4 *>(fac_w + (job & 1) * 256);
+            fdst[lane] = __ldg(src + lane);
+            fdst[32 + lane] = __ldg(src + 32 + lane);
             __syncwarp();
         };
         auto factors = [&](int job, int sl, float (&f)[32]) {
@@ -802,16 +807,20 @@ __global__ void __launch_bounds__(kScThreads, 1)
                 f[4 * q + 3] = u.w * rs;
             }
         };
+        float *xm = reinterpret_cast<float *>(smem + L::kXch);  // [2 halves][128]
+        float *xz = xm + 2 * 128;                                // [2 halves][128]
         const int r8 = lane & 7;
         const bool b4 = (r8 & 4) != 0, b2 = (r8 & 2) != 0, b1 = (r8 & 1) != 0;
         float m = -INFINITY, z = 0.f, coef = 0.f;
+        // After a failed wait a warp skips the remaining waits and work but still walks
+        // every job, so both warps of a lane group always meet at the merge's barrier.
+        bool ok = true;
         for (int j = 0; j < njobs; ++j) {
             const int buf = j & 1;
             const int ch = j < nch ? j : j - nch;
             // this warp read the buffer of parity j & 1 for job j - 2, which it has finished
             stage_factors(j, ch * kScChunk);
-            if (!wait(&tfull[buf], (j >> 1) & 1)) break;
-            tc_fence_after();
+            ok = ok && wait(&tfull[buf], (j >> 1) & 1);
             const int c0 = ch * kScChunk;
             const int ncols = min(kScChunk, nkb - c0);
             const int nsl = (ncols + 31) >> 5;
@@ -819,10 +828,12 @@ __global__ void __launch_bounds__(kScThreads, 1)
             const int nvcols = max(0, min(ncols, nkb_valid - c0));
             const int nvsl = (nvcols + 31) >> 5;
             const uint32_t tb = t_lane + buf * kScChunk;
-            if (j < nch) {
-                // row statistics in log2 units: max, then the sum of 2^(x - max)
+            if (ok) tc_fence_after();
+            if (ok && j < nch) {
+                // row statistics of this warp's slices in log2 units: max, then the sum of
+                // 2^(x - max)
                 float mx = m;
-                for (int sl = 0; sl < nvsl; ++sl) {
+                for (int sl = half; sl < nvsl; sl += 2) {
                     uint32_t v[32];
                     float f[32];
                     tmem_ld32(tb + sl * 32, v);
@@ -834,7 +845,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
                         if (i < lim) mx = fmaxf(mx, __uint_as_float(v[i]) * f[i]);
                 }
                 float zz = m == -INFINITY ? 0.f : z * fast_exp2(m - mx);
-                for (int sl = 0; sl < nvsl; ++sl) {
+                for (int sl = half; sl < nvsl; sl += 2) {
                     uint32_t v[32];
                     float f[32];
                     tmem_ld32(tb + sl * 32, v);
@@ -847,10 +858,21 @@ __global__ void __launch_bounds__(kScThreads, 1)
                 }
                 m = mx;
                 z = zz;
-                if (j == nch - 1) coef = z > 0.f ? wr / z : 0.f;
             }
-            if (nch == 1 || j >= nch) {
-                for (int sl = 0; sl < nsl; ++sl) {
+            if (j == nch - 1) {
+                // merge the two warps' (max, sum) of each row: named barrier 1 + qd
+                xm[half * 128 + row] = m;
+                xz[half * 128 + row] = z;
+                asm volatile("bar.sync %0, 64;" ::"r"(1 + qd) : "memory");
+                const float m_o = xm[(half ^ 1) * 128 + row], z_o = xz[(half ^ 1) * 128 + row];
+                const float mt = fmaxf(m, m_o);
+                z = (m == -INFINITY ? 0.f : z * fast_exp2(m - mt)) +
+                    (m_o == -INFINITY ? 0.f : z_o * fast_exp2(m_o - mt));
+                m = mt;
+                coef = z > 0.f ? wr / z : 0.f;
+            }
+            if (ok && (nch == 1 || j >= nch)) {
+                for (int sl = half; sl < nsl; sl += 2) {
                     uint32_t v[32];
                     float f[32];
                     tmem_ld32(tb + sl * 32, v);
@@ -888,8 +910,10 @@ __global__ void __launch_bounds__(kScThreads, 1)
                     }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&tempty[buf]);
+            if (ok) {
+                tc_fence_before();
+                mbar_arrive(&tempty[buf]);
+            }
         }
     }
 
