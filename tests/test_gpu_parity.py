@@ -124,6 +124,60 @@ def test_sip_bit_exact(orc, nkb, budget):
         np.testing.assert_array_equal(p.cpu().numpy().view(np.uint64), p_r.view(np.uint64))
 
 
+def _boundary_row(orc, s, K, seed, h, qb, j0):
+    """Move score j0 of row (h, qb) until its SIP probability times 2^53 lands on its own
+    Philox draw R53 (the oracle's p and Philox), so that keeping j0 is decided by the last
+    bits of p_j0."""
+    key = np.array([seed & 0xFFFFFFFF, seed >> 32], dtype=np.uint32)
+    x = orc.philox4x32_10(np.array([j0, qb, h, 0], dtype=np.uint32), key)
+    target = ((((int(x[0]) << 32) | int(x[1])) >> 11) / 2.0**53)
+    for _ in range(40):
+        p = orc.sip(s.reshape(1, 1, 1, -1), K, seed)[3][0, 0, 0, j0]
+        if not 0.0 < p < 1.0 or p == target:
+            break
+        v = np.float32(s[j0] * (target / p))
+        if v == s[j0]:
+            break
+        s[j0] = v
+    return s
+
+
+@pytest.mark.parametrize("nkb,budget", [(200, 20), (9000, 900)])
+def test_sip_draws_at_the_boundary(orc, nkb, budget):
+    """Rows whose draw for one entry falls within a few float steps of p 2^53, on both
+    sides: the kernel's fast fp32 pre-decision must hand these to the exact test, so the
+    plan still equals the oracle's bit for bit (rows of up to 8192 entries and longer)."""
+    seed = 11
+    rng = np.random.default_rng(nkb)
+    H, nqb = 2, 7  # row r = (h, qb): step -3 .. +3 float steps away from the boundary
+    s = (rng.random((1, H, nqb, nkb)) * 0.01).astype(np.float32)
+    for h in range(H):
+        j0 = int(rng.integers(nkb))
+        base = _boundary_row(orc, s[0, h, 0].copy(), budget, seed, h, 0, j0)
+        for qb in range(nqb):
+            row = _boundary_row(orc, base.copy(), budget, seed, h, qb, j0)
+            v = row[j0]
+            step = qb - 3
+            for _ in range(abs(step)):
+                v = np.nextafter(v, np.float32(np.inf) if step > 0 else np.float32(0))
+            row[j0] = v
+            s[0, h, qb] = row
+    idx_r, cnt_r, w_r, p_r, bad = orc.sip(s, budget, seed)
+    assert not bad.any()
+    for want_p in (False, True):
+        flag = _flag()
+        res = ab.select(torch.from_numpy(s).cuda(), budget, "sip", seed, want_p=want_p,
+                        dev_flag=flag)
+        idx, cnt, w = res[:3]
+        torch.cuda.synchronize()
+        assert ab.check_flag(flag) == 0
+        np.testing.assert_array_equal(cnt.cpu().numpy(), cnt_r)
+        np.testing.assert_array_equal(idx.cpu().numpy(), idx_r)
+        np.testing.assert_array_equal(w.cpu().numpy().view(np.uint32), w_r.view(np.uint32))
+        if want_p:
+            np.testing.assert_array_equal(res[3].cpu().numpy().view(np.uint64), p_r.view(np.uint64))
+
+
 @pytest.mark.parametrize("nkb,budget", [(8, 3), (300, 30), (2048, 614), (929, 93), (5, 9)])
 def test_topk_bit_exact(orc, nkb, budget):
     s = _random_scores(2, 2, 3, nkb, seed=7 * nkb, kind="lognormal")
