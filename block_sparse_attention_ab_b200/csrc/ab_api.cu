@@ -1,8 +1,10 @@
 // ab_api.cu -- the C ABI declared in include/ab_attn.h: host-side argument checks,
 // workspace carving, and kernel launches on the caller's stream. No device memory is
-// allocated here and no state is kept between calls.
+// allocated here; the only state kept between calls is one side stream and two events
+// per device for ab_score's concurrent mean-key pass.
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
@@ -61,6 +63,62 @@ ab_status check_unit(const ab_shape &s, int unit)
 }
 
 ab_status cuda_status(cudaError_t e) { return ab::status_of(e); }
+
+// ab_score's mean keys (an HBM-bound read of K) and k-means (a latency-bound chain over Q)
+// are independent: the mean keys run on a side stream forked from the caller's stream by
+// an event and joined back by another before the block score. One side stream and two
+// events per device, created on the device's first ab_score call and kept until exit; the
+// mutex makes a call's record-wait-launch sequence atomic across host threads.
+constexpr int kMaxSideDevices = 64;
+
+struct SideStream {
+    std::mutex mu;
+    bool ready = false;
+    cudaStream_t st = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+SideStream g_side[kMaxSideDevices];
+
+cudaError_t side_init(SideStream &ss)
+{
+    if (ss.ready) return cudaSuccess;
+    cudaError_t e = cudaStreamCreateWithFlags(&ss.st, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
+    if (e == cudaSuccess) ss.ready = true;
+    return e;
+}
+
+// Mean keys and k-means of one ab_score call: concurrently through the device's side
+// stream, or in sequence on the caller's stream while that stream is being captured
+// into a graph (or on a device past the side-stream table).
+template <typename MeanKey, typename KMeans>
+cudaError_t meankey_and_kmeans(cudaStream_t cs, MeanKey meankey, KMeans kmeans)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(cs, &cap);
+    if (e != cudaSuccess || cap != cudaStreamCaptureStatusNone || dev < 0 || dev >= kMaxSideDevices) {
+        (void)cudaGetLastError();  // a capture-status query refused on the legacy stream
+        e = meankey(cs);
+        return e == cudaSuccess ? kmeans(cs) : e;
+    }
+    // k-means is enqueued first so that its CTAs take the SMs and the mean-key CTAs fill
+    // the resources they leave (one per SM)
+    SideStream &ss = g_side[dev];
+    std::lock_guard<std::mutex> lock(ss.mu);
+    e = side_init(ss);
+    if (e == cudaSuccess) e = cudaEventRecord(ss.fork, cs);
+    if (e == cudaSuccess) e = kmeans(cs);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.st, ss.fork, 0);
+    if (e == cudaSuccess) e = meankey(ss.st);
+    if (e == cudaSuccess) e = cudaEventRecord(ss.join, ss.st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cs, ss.join, 0);
+    return e;
+}
 
 ab_status attn_common(const void *q, const void *k, const void *v, ab_shape s, int unit,
                       const int32_t *idx, const int32_t *cnt, const float *w, void *out,
@@ -164,10 +222,15 @@ ab_status ab_score_units(const void *q, const void *k, ab_shape s, int n_cluster
     cudaStream_t cs = (cudaStream_t)stream;
     void *kt = ws + L.kbar_terms;
     float *ks = reinterpret_cast<float *>(ws + L.kscale);
-    cudaError_t e = ab::launch_meankey_units(k, kb, kt, ks, BH, s.N, s.N_pad, s.d, key_unit, cs);
-    if (e == cudaSuccess)
-        e = ab::launch_kmeans(q, ce, cw, assign, BH, s.N, s.N_pad, s.d, n_clusters, iters,
-                              dev_flag, cs);
+    cudaError_t e = meankey_and_kmeans(
+        cs,
+        [&](cudaStream_t st) {
+            return ab::launch_meankey_units(k, kb, kt, ks, BH, s.N, s.N_pad, s.d, key_unit, st);
+        },
+        [&](cudaStream_t st) {
+            return ab::launch_kmeans(q, ce, cw, assign, BH, s.N, s.N_pad, s.d, n_clusters, iters,
+                                     dev_flag, st);
+        });
     if (e == cudaSuccess)
         e = ab::launch_score(ce, cw, kt, ks, scores, BH, nqb, nku, nku_valid, s.d, n_clusters,
                              dev_flag, cs);

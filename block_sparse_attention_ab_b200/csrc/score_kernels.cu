@@ -101,8 +101,10 @@ __device__ __forceinline__ int sw128_chunk(int row, int col, int panel_bytes)
 // component) and split into two fp16 terms, kbs[t][bh][j][i] (t = 0 high, 1 low), with
 // the unscale factor 2^-e in kscale[bh][j] (row stride ks_stride).
 // ---------------------------------------------------------------------------------
+// At most 32 registers per thread (8 CTAs' worth of the register file), so that one CTA
+// fits beside the four k-means CTAs of an SM when the two kernels run concurrently.
 template <int D>
-__global__ void __launch_bounds__(256) meankey_kernel(const __nv_bfloat16 *__restrict__ k,
+__global__ void __launch_bounds__(256, 8) meankey_kernel(const __nv_bfloat16 *__restrict__ k,
                                                       float *__restrict__ kbar,
                                                       __half *__restrict__ kbs,
                                                       float *__restrict__ kscale, int N,
@@ -252,6 +254,9 @@ __global__ void __launch_bounds__(256) meankey4_kernel(const __nv_bfloat16 *__re
 // Thread i keeps feature i of the 8 centroids in registers: after each update it
 // writes column i of the next assignment's B operand and its share of the squared
 // norms (reduced across the warp, then across the 4 warps through shared memory).
+// A round whose assignments equal the previous round's ends the iteration there: the
+// update would give the same centroids bit for bit, so the remaining rounds change
+// nothing (the outputs equal those of all T rounds).
 // One elected thread of warp 0 issues the MMAs. Every wait is bounded; a timed-out
 // CTA drains its in-flight work and exits.
 // ---------------------------------------------------------------------------------
@@ -323,6 +328,7 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
     __shared__ __align__(16) float normw[CMAX][4];  // squared-norm partials per warp
     __shared__ __align__(16) int wcount[CMAX][4];   // member counts per warp
     __shared__ uint8_t lab[128];
+    __shared__ int wchanged[4];                     // per warp: an assignment changed
     uint64_t *q_full = reinterpret_cast<uint64_t *>(smem + L::kBar);
     uint64_t *mma_done = q_full + 1;
     uint64_t *drain = q_full + 2;
@@ -444,7 +450,10 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
                 }
             }
             const int a = tid < nv ? arg : 255;
+            const bool changed = it == 0 || lab[tid] != (uint8_t)a;  // lab: previous round
             lab[tid] = (uint8_t)a;
+            const unsigned chg = __ballot_sync(0xffffffffu, changed);
+            if (lane == 0) wchanged[warp] = chg != 0u;
             // (2) one-hot column of this query (B of the update GEMM) and member counts
             __nv_bfloat16 *oh = reinterpret_cast<__nv_bfloat16 *>(smem + L::kBU);
 #pragma unroll
@@ -459,6 +468,10 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
         tc_fence_before();
         ok = __syncthreads_and(good);
         if (!ok) break;
+        // Converged: this round reproduced the previous assignments, so the update would
+        // reproduce the current centroids bit for bit (same members, same sums) and every
+        // later round this one. The outputs of all T rounds are the current ones.
+        if (it > 0 && (wchanged[0] | wchanged[1] | wchanged[2] | wchanged[3]) == 0) break;
         tc_fence_after();
 
         // (3) update GEMM
@@ -571,11 +584,11 @@ struct ScSmem {
     static constexpr int kA = 0;
     static constexpr int kB = kA + 2 * kATerm;
     static constexpr int kBar = kB + kStages * kStageBytes;
-    // barriers: full[S], empty[S], tfull[2], tempty[2], drain
-    static constexpr int kNumBars = 2 * kStages + 5;
-    static constexpr int kRows = kBar + kNumBars * 8;  // float [2][128]: 2^e, 2^-e per row
+    // barriers: full[S], empty[S], tfull[2], tempty[2], drain, a_ready
+    static constexpr int kNumBars = 2 * kStages + 6;
+    static constexpr int kRows = kBar + kNumBars * 8;  // float [128]: 2^-e per centroid row
     // float [8 warps][2 jobs][256]: column factors, read as float4 (16-byte aligned)
-    static constexpr int kFac = (kRows + 2 * 128 * 4 + 15) & ~15;
+    static constexpr int kFac = (kRows + 128 * 4 + 15) & ~15;
     static constexpr int kXch = kFac + 8 * 2 * 256 * 4;  // float [2][2][128]: (m, z) per half
     static constexpr int kMisc = kXch + 2 * 2 * 128 * 4;  // TMEM base, abort flag
     static_assert(kFac % 16 == 0 && kB % 1024 == 0, "shared-memory layout alignment");
@@ -608,50 +621,8 @@ __global__ void __launch_bounds__(kScThreads, 1)
     const int g = blockIdx.x, bh = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // each centroid row's scale 2^e and unscale 2^-e (zero rows: 1)
-    float *row_mul = reinterpret_cast<float *>(smem + L::kRows);
-    float *row_unscale = row_mul + 128;
-    if (tid < 128) {
-        const int qb = g * 16 + (tid >> 3), c = tid & 7;
-        float amax = 0.f;
-        if (qb < nqb && c < C) {
-            const float4 *src = reinterpret_cast<const float4 *>(cent + (((size_t)bh * nqb + qb) * C + c) * D);
-#pragma unroll 8
-            for (int i = 0; i < D / 4; ++i) {
-                const float4 u = __ldg(src + i);
-                amax = fmaxf(fmaxf(amax, fmaxf(fabsf(u.x), fabsf(u.y))), fmaxf(fabsf(u.z), fabsf(u.w)));
-            }
-        }
-        const int e = scale_exponent(amax);
-        row_mul[tid] = pow2f(e);
-        row_unscale[tid] = pow2f(-e);
-    }
-    __syncthreads();
-    // centroid terms (A operand), all threads
-    {
-        constexpr int CH = D / 8;
-        for (int pi = tid; pi < 128 * CH; pi += kScThreads) {
-            const int row = pi / CH, k0 = (pi % CH) * 8;
-            const int qb = g * 16 + (row >> 3), c = row & 7;
-            float x[8];
-            if (qb < nqb && c < C) {
-                const float4 *src = reinterpret_cast<const float4 *>(
-                    cent + (((size_t)bh * nqb + qb) * C + c) * D + k0);
-                const float4 u = __ldg(src), v = __ldg(src + 1);
-                const float sc = row_mul[row];
-                x[0] = u.x * sc; x[1] = u.y * sc; x[2] = u.z * sc; x[3] = u.w * sc;
-                x[4] = v.x * sc; x[5] = v.y * sc; x[6] = v.z * sc; x[7] = v.w * sc;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = 0.f;
-            }
-            uint4 t[2];
-            split2h_x8(x, t);
-#pragma unroll
-            for (int s = 0; s < 2; ++s)
-                *reinterpret_cast<uint4 *>(smem + L::kA + s * L::kATerm + sw128_chunk(row, k0, 16384)) = t[s];
-        }
-    }
+    uint64_t *a_ready = drain + 1;  // the centroid terms and row factors are in place
+    float *row_unscale = reinterpret_cast<float *>(smem + L::kRows);  // 2^-e per centroid row
     if (tid == 0) {
         for (int s = 0; s < L::kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -662,6 +633,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
             mbar_init(&tempty[b], 256);
         }
         mbar_init(drain, 1);
+        mbar_init(a_ready, 8);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -669,11 +641,54 @@ __global__ void __launch_bounds__(kScThreads, 1)
         tmem_alloc(tmem_slot, kScTmemCols);
         tmem_relinquish();
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+
+    if (warp >= 2) {
+        // Centroid terms (A operand), built by the eight epilogue warps while the producer
+        // already streams mean-key tiles: warp w takes rows 16 (w - 2) .. + 15, each row
+        // read once (a row spans 128 / D warp passes' lanes: D / 4 lanes of one float4
+        // each), its scale exponent from a shuffle max, then scaled, split and stored.
+        constexpr int LPR = D / 4;        // lanes per row
+        constexpr int RPP = 32 / LPR;     // rows per warp pass
+        constexpr int PASSES = 16 / RPP;  // passes for the warp's 16 rows
+        const int sub = lane / LPR, li = lane % LPR;
+        float4 u[PASSES];
+#pragma unroll
+        for (int ps = 0; ps < PASSES; ++ps) {
+            const int row = (warp - 2) * 16 + ps * RPP + sub;
+            const int qb = g * 16 + (row >> 3), c = row & 7;
+            u[ps] = (qb < nqb && c < C)
+                        ? __ldg(reinterpret_cast<const float4 *>(cent + (((size_t)bh * nqb + qb) * C + c) * D) + li)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int ps = 0; ps < PASSES; ++ps) {
+            const int row = (warp - 2) * 16 + ps * RPP + sub;
+            float amax = fmaxf(fmaxf(fabsf(u[ps].x), fabsf(u[ps].y)), fmaxf(fabsf(u[ps].z), fabsf(u[ps].w)));
+#pragma unroll
+            for (int o = LPR / 2; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const int e = scale_exponent(amax);
+            const float sc = pow2f(e);
+            if (li == 0) row_unscale[row] = pow2f(-e);
+            const float2 y01 = make_float2(u[ps].x * sc, u[ps].y * sc);
+            const float2 y23 = make_float2(u[ps].z * sc, u[ps].w * sc);
+            const __half2 h01 = __floats2half2_rn(y01.x, y01.y), h23 = __floats2half2_rn(y23.x, y23.y);
+            const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+            const __half2 l01 = __floats2half2_rn(y01.x - f01.x, y01.y - f01.y);
+            const __half2 l23 = __floats2half2_rn(y23.x - f23.x, y23.y - f23.y);
+            const int k0 = 4 * li;  // four elements: half of a 16-byte chunk
+            const int off = sw128_chunk(row, k0 & ~7, 16384) + (k0 & 7) * 2;
+            *reinterpret_cast<uint2 *>(smem + L::kA + off) = make_uint2(half2_bits(h01), half2_bits(h23));
+            *reinterpret_cast<uint2 *>(smem + L::kA + L::kATerm + off) =
+                make_uint2(half2_bits(l01), half2_bits(l23));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(a_ready);
+    }
 
     const int nch = (nkb + kScChunk - 1) / kScChunk;
     const int njobs = nch == 1 ? 1 : 2 * nch;
@@ -724,7 +739,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
         const uint64_t b0 = smem_desc_sw128(smem_u32(smem + L::kB), 16, 1024);
         constexpr uint32_t idesc = idesc_f16_f32(128, 64, 0, 0);
         int pos = 0;
-        bool ok = true;
+        bool ok = wait(a_ready, 0);
         for (int j = 0; j < njobs && ok; ++j) {
             const int buf = j & 1;
             const int ch = j < nch ? j : j - nch;
@@ -781,12 +796,14 @@ __global__ void __launch_bounds__(kScThreads, 1)
         const float wr = (row_ok && c < C) ? __ldg(cw + ((size_t)bh * nqb + qb) * C + c) : 0.f;
         float *dst = scores + ((size_t)bh * nqb + (row_ok ? qb : 0)) * nkb;
         const uint32_t t_lane = tmem + ((uint32_t)(qd * 32) << 16);
+        // the row factors are written by the other epilogue warps' operand build
+        const bool ok_a = wait(a_ready, 0);
+        const float rs = row_unscale[row] * scale_log2;
         // x = L * 2^-(e_row + e_j) * log2(e) / sqrt(d): the logit in log2 units from the
         // scaled product. Each warp copies a job's 256 column factors into its own shared
         // buffer (one per job parity) before it waits for the job's logits, and every
         // lane then reads the 32 factors of a TMEM slice from there (broadcast reads; the
         // factor rows are padded to a multiple of the chunk, so no read passes them).
-        const float rs = row_unscale[row] * scale_log2;
         const float *ks_row = kscale + (size_t)bh * ks_stride;
         float *fac_w = reinterpret_cast<float *>(smem + L::kFac) + (warp - 2) * 2 * 256;
         auto stage_factors = [&](int job, int col0) {
@@ -814,7 +831,7 @@ __global__ void __launch_bounds__(kScThreads, 1)
         float m = -INFINITY, z = 0.f, coef = 0.f;
         // After a failed wait a warp skips the remaining waits and work but still walks
         // every job, so both warps of a lane group always meet at the merge's barrier.
-        bool ok = true;
+        bool ok = ok_a;
         for (int j = 0; j < njobs; ++j) {
             const int buf = j & 1;
             const int ch = j < nch ? j : j - nch;
@@ -830,9 +847,9 @@ __global__ void __launch_bounds__(kScThreads, 1)
             const uint32_t tb = t_lane + buf * kScChunk;
             if (ok) tc_fence_after();
             if (ok && j < nch) {
-                // row statistics of this warp's slices in log2 units: max, then the sum of
-                // 2^(x - max)
-                float mx = m;
+                // row statistics of this warp's slices in log2 units, online per slice: the
+                // slice max (a tree of three-way maxima), then the running sum rescaled to
+                // the new max plus the slice's 2^(x - max) in four partial sums
                 for (int sl = half; sl < nvsl; sl += 2) {
                     uint32_t v[32];
                     float f[32];
@@ -840,24 +857,23 @@ __global__ void __launch_bounds__(kScThreads, 1)
                     factors(j, sl, f);
                     tmem_wait_ld();
                     const int lim = nvcols - sl * 32;
+                    float x[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = i < lim ? __uint_as_float(v[i]) * f[i] : -INFINITY;
+                    float t[11];
+#pragma unroll
+                    for (int i = 0; i < 10; ++i) t[i] = fmax3(x[3 * i], x[3 * i + 1], x[3 * i + 2]);
+                    t[10] = fmaxf(x[30], x[31]);
+                    const float smax = fmax3(fmax3(t[0], t[1], t[2]), fmax3(t[3], t[4], t[5]),
+                                             fmax3(fmax3(t[6], t[7], t[8]), t[9], t[10]));
+                    const float mx = fmaxf(m, smax);
+                    float zp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        if (i < lim) mx = fmaxf(mx, __uint_as_float(v[i]) * f[i]);
+                        if (i < lim) zp[i & 3] += fast_exp2(x[i] - mx);
+                    z = (m == -INFINITY ? 0.f : z * fast_exp2(m - mx)) + ((zp[0] + zp[1]) + (zp[2] + zp[3]));
+                    m = mx;
                 }
-                float zz = m == -INFINITY ? 0.f : z * fast_exp2(m - mx);
-                for (int sl = half; sl < nvsl; sl += 2) {
-                    uint32_t v[32];
-                    float f[32];
-                    tmem_ld32(tb + sl * 32, v);
-                    factors(j, sl, f);
-                    tmem_wait_ld();
-                    const int lim = nvcols - sl * 32;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i < lim) zz += fast_exp2(fmaf(__uint_as_float(v[i]), f[i], -mx));
-                }
-                m = mx;
-                z = zz;
             }
             if (j == nch - 1) {
                 // merge the two warps' (max, sum) of each row: named barrier 1 + qd
@@ -952,6 +968,11 @@ cudaError_t launch_meankey(const void *k, float *kbar, void *kbar_terms, float *
     const int ks_stride = (int)kscale_stride((size_t)nkb);
     const dim3 grid((unsigned)(BH * nkb));
     __half *kbs = static_cast<__half *>(kbar_terms);
+    cudaError_t e = cudaFuncSetAttribute(d == 128 ? (const void *)meankey_kernel<128>
+                                                  : (const void *)meankey_kernel<64>,
+                                         cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     if (d == 128)
         meankey_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, kscale, N, N_pad,
                                                   nkb, ks_stride);
@@ -973,6 +994,11 @@ static cudaError_t launch_kmeans_t(const void *q, float *cent, float *cw, uint8_
     const int smem = KmSmem<D>::kAlloc;
     cudaError_t e =
         cudaFuncSetAttribute(kmeans_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // the whole unified L1 as shared memory: four k-means CTAs then leave room for a
+    // concurrent mean-key CTA (a carveout sized to the four alone would not)
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kmeans_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     kmeans_kernel<D><<<(unsigned)(BH * nqb), 128, smem, st>>>(tm, N, N_pad, nqb, C, T, cent, cw,
                                                                 assign, flag);
