@@ -22,7 +22,9 @@
  *     GPU that loads the library, from load until process exit: the attention
  *     kernels' 4096 claim slots (16 bytes each; see "Scheduling" at ab_attn_fwd) and
  *     the AB_NOALLOC_SCRATCH_BYTES scratch of ab_score_noalloc; and on the host, the
- *     copy streams and events of ab_forward_host. Nothing else persists between calls.
+ *     copy streams and events of ab_forward_host and one side stream and two events
+ *     per device for ab_score (created on first use). Nothing else persists between
+ *     calls.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
  *     enqueues work on it and returns; results are ready when the stream is.
  *   - Argument errors are reported synchronously by the return value and nothing is
@@ -90,8 +92,9 @@ typedef struct {
 /*
  * ab_score_workspace_size -- bytes of device scratch ab_score() needs for shape `s`
  * and `n_clusters`: the mean keys [B,H,n_kb,d] fp32, the centroids [B,H,n_qb,C,d] fp32,
- * the cluster weights [B,H,n_qb,C] fp32 and the mean keys' exact three-term bf16 split
- * [3,B,H,n_kb,d] (operands of the tensor-core block score), each region 256-byte aligned.
+ * the cluster weights [B,H,n_qb,C] fp32, the two fp16 terms of each mean key scaled by a
+ * power of two [2,B,H,n_kb,d] (operands of the tensor-core block score) and each mean
+ * key's unscale factor fp32 [B,H,n_kb rounded up to 256], each region 256-byte aligned.
  * Returns AB_ERR_* for an invalid shape; *bytes is then 0.
  */
 ab_status ab_score_workspace_size(ab_shape s, int n_clusters, size_t *bytes);
