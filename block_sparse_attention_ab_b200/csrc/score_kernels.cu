@@ -101,8 +101,9 @@ __device__ __forceinline__ int sw128_chunk(int row, int col, int panel_bytes)
 // component) and split into two fp16 terms, kbs[t][bh][j][i] (t = 0 high, 1 low), with
 // the unscale factor 2^-e in kscale[bh][j] (row stride ks_stride).
 // ---------------------------------------------------------------------------------
-// At most 32 registers per thread (8 CTAs' worth of the register file), so that one CTA
-// fits beside the four k-means CTAs of an SM when the two kernels run concurrently.
+// At most 32 registers per thread (8 CTAs' worth of the register file): a CTA then fits
+// beside four k-means CTAs, so the mean keys can start on SMs that still run the last
+// k-means wave (ab_score launches them on a side stream).
 template <int D>
 __global__ void __launch_bounds__(256, 8) meankey_kernel(const __nv_bfloat16 *__restrict__ k,
                                                       float *__restrict__ kbar,
@@ -968,11 +969,6 @@ cudaError_t launch_meankey(const void *k, float *kbar, void *kbar_terms, float *
     const int ks_stride = (int)kscale_stride((size_t)nkb);
     const dim3 grid((unsigned)(BH * nkb));
     __half *kbs = static_cast<__half *>(kbar_terms);
-    cudaError_t e = cudaFuncSetAttribute(d == 128 ? (const void *)meankey_kernel<128>
-                                                  : (const void *)meankey_kernel<64>,
-                                         cudaFuncAttributePreferredSharedMemoryCarveout,
-                                         (int)cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
     if (d == 128)
         meankey_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, kbs, kscale, N, N_pad,
                                                   nkb, ks_stride);
@@ -994,11 +990,6 @@ static cudaError_t launch_kmeans_t(const void *q, float *cent, float *cw, uint8_
     const int smem = KmSmem<D>::kAlloc;
     cudaError_t e =
         cudaFuncSetAttribute(kmeans_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    // the whole unified L1 as shared memory: four k-means CTAs then leave room for a
-    // concurrent mean-key CTA (a carveout sized to the four alone would not)
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(kmeans_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     kmeans_kernel<D><<<(unsigned)(BH * nqb), 128, smem, st>>>(tm, N, N_pad, nqb, C, T, cent, cw,
                                                                 assign, flag);
