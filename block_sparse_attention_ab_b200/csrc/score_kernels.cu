@@ -276,7 +276,9 @@ constexpr int kKmTmemCols = 64;  // G in columns 0..31, S in columns 32..47
 
 // Write feature k of the 8 centroids as column k of the assignment GEMM's B operand
 // (three bf16 terms each) and the warp's partial squared norms to normw[c][warp].
-template <int D>
+// kFirst: the initial centroids are bf16 queries, whose middle and low terms are exactly
+// zero; those rows were zeroed at the start, so only the high terms are written.
+template <int D, bool kFirst = false>
 __device__ __forceinline__ void km_publish(uint8_t *smem, const float (&cur)[8], int k,
                                            bool has_k, int warp, int lane, float (*normw)[4])
 {
@@ -286,13 +288,17 @@ __device__ __forceinline__ void km_publish(uint8_t *smem, const float (&cur)[8],
     for (int c = 0; c < 8; ++c) {
         sq[c] = cur[c] * cur[c];
         if (has_k) {
-            uint32_t t0, t1, t2;
-            split3_bits(cur[c], t0, t1, t2);
             // rows c, 8 + c, 16 + c share the swizzle phase (row mod 8 = c)
             const int o = (sw128_chunk(c, k, 4096) >> 1) + (k & 7);
-            ba[o] = (uint16_t)(t0 >> 16);
-            ba[o + 8 * 64] = (uint16_t)(t1 >> 16);
-            ba[o + 16 * 64] = (uint16_t)(t2 >> 16);
+            if (kFirst) {
+                ba[o] = (uint16_t)(__float_as_uint(cur[c]) >> 16);
+            } else {
+                uint32_t t0, t1, t2;
+                split3_bits(cur[c], t0, t1, t2);
+                ba[o] = (uint16_t)(t0 >> 16);
+                ba[o + 8 * 64] = (uint16_t)(t1 >> 16);
+                ba[o + 16 * 64] = (uint16_t)(t2 >> 16);
+            }
         }
     }
     // reduce-scatter across the warp: lane L ends with cluster (L >> 2) & 7
@@ -349,14 +355,21 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
+        // the query tile's load goes out first and overlaps the rest of the set-up
+        prefetch_tmap(&tmQ);
+        mbar_arrive_expect_tx(q_full, (D / 64) * 16384);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+            tma_load_3d(smem + L::kQ + h * 16384, &tmQ, q_full, h * 64, t0, bh);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kKmTmemCols);
         tmem_relinquish();
     }
-    // constant zero rows: centroid-term rows 24..31, one-hot rows 8..15
-    for (int e = tid; e < (D / 64) * 64; e += 128)
-        *reinterpret_cast<uint4 *>(smem + L::kBA + (e >> 6) * 4096 + (24 + ((e >> 3) & 7)) * 128 +
+    // zero rows: centroid-term rows 8..31 (the initial centroids' middle and low terms,
+    // then the constant padding rows 24..31), one-hot rows 8..15
+    for (int e = tid; e < (D / 64) * 192; e += 128)
+        *reinterpret_cast<uint4 *>(smem + L::kBA + (e / 192) * 4096 + (8 + (e % 192) / 8) * 128 +
                                    (e & 7) * 16) = make_uint4(0, 0, 0, 0);
     *reinterpret_cast<uint4 *>(smem + L::kBU + (tid >> 6) * 2048 + (8 + ((tid >> 3) & 7)) * 128 +
                                (tid & 7) * 16) = make_uint4(0, 0, 0, 0);
@@ -365,16 +378,6 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
-        if (elect_one()) {
-            prefetch_tmap(&tmQ);
-            mbar_arrive_expect_tx(q_full, (D / 64) * 16384);
-#pragma unroll
-            for (int h = 0; h < D / 64; ++h)
-                tma_load_3d(smem + L::kQ + h * 16384, &tmQ, q_full, h * 64, t0, bh);
-        }
-        __syncwarp();
-    }
     bool ok = mbar_wait(q_full, 0, abort_flag, flag);
 
     // initial centroid c: the query at block-local index c*floor(nv/C) (min(c, nv-1)
@@ -391,7 +394,7 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
                          : 0.f;
         }
     }
-    km_publish<D>(smem, cur, tid, has_k, warp, lane, normw);
+    km_publish<D, true>(smem, cur, tid, has_k, warp, lane, normw);
     fence_proxy_async_smem();
     tc_fence_before();
     ok = __syncthreads_and(ok);

@@ -250,6 +250,28 @@ def test_score_parity(orc, N, d, H, C):
     np.testing.assert_allclose(sg.sum(-1), 1.0, rtol=1e-5)
 
 
+@pytest.mark.parametrize("T", [1, 2, 30])
+def test_kmeans_rounds_past_convergence(orc, T):
+    """k-means stops once a round reproduces the previous round's assignments; with T = 30
+    most blocks converge long before the last round, and the GPU's outputs must still be
+    those of all T rounds (the oracle runs every round). T = 1 and 2 leave no room for an
+    early stop."""
+    N, d, H, C = 5 * 128 + 77, 128, 2, 8
+    q, k, _ = _inputs(N, H=H, d=d, seed=T + 11)
+    _, _, cent, cw, assign = ab.score(*_cuda(q, k), N, C, T, intermediates=True)
+    torch.cuda.synchronize()
+    cent_r, wts_r, assign_r, gap, inertia = orc.kmeans(q, N, C, T)
+    if T == 30:  # the early stop is exercised: most blocks settle by round 15
+        assert np.mean(inertia[..., -1] == inertia[..., 14]) > 0.5
+    B, H_, N_pad, _ = q.shape
+    nb = N_pad // 128
+    mism = (assign.cpu().numpy() != assign_r).reshape(B, H_, nb, 128).any(-1)
+    assert not np.any(mism & ~(gap < TIE_GAP)), "assignment mismatch outside a near tie"
+    ok = ~mism
+    np.testing.assert_array_equal(cw.cpu().numpy()[ok], wts_r[ok].astype(np.float32))
+    np.testing.assert_allclose(cent.cpu().numpy()[ok], cent_r[ok], rtol=1e-5, atol=1e-5)
+
+
 def test_score_tiny_workload_end_to_end(orc):
     w = synth.WORKLOADS["tiny"]
     q, k, v = synth.make_qkv(w)
