@@ -211,6 +211,24 @@ def score_bytes(w) -> float:
     return 2.0 * w.B * w.H * w.N_pad * w.d * 2 + 4.0 * w.B * w.H * w.n_blocks ** 2
 
 
+def score_floor(w, peaks, score_ms: float) -> dict:
+    """Serial floor of one scoring pass: Q and K read once at the measured HBM rate (the
+    mean keys and k-means), then the block score, bound by the larger of its tensor work
+    (C centroid rows x n_kb key blocks x d per query block, three fp16 products per logit
+    and pass; two passes when n_kb > 256) at the measured dense bf16 burst rate (fp16
+    runs at the same rate) and its score writes."""
+    hbm = peaks["hbm_gbs"] * 1e9
+    qk = 2.0 * w.B * w.H * w.N_pad * w.d * 2
+    sw = 4.0 * w.B * w.H * w.n_blocks ** 2
+    passes = 1 if w.n_blocks <= 256 else 2
+    flop = 2.0 * w.n_clusters * w.d * w.n_blocks ** 2 * w.B * w.H * 3 * passes
+    gemm_ms = flop / (peaks["bf16_tflops"] * 1e12) * 1e3
+    floor_ms = qk / hbm * 1e3 + max(gemm_ms, sw / hbm * 1e3)
+    return {"ms": round(floor_ms, 4), "qk_read_ms": round(qk / hbm * 1e3, 4),
+            "score_gemm_tflop": round(flop / 1e12, 4), "score_gemm_ms": round(gemm_ms, 4),
+            "frac": round(floor_ms / score_ms, 4)}
+
+
 def stats(ts):
     return {"median": round(statistics.median(ts), 4), "min": round(min(ts), 4),
             "mean": round(float(np.mean(ts)), 4)}
@@ -515,7 +533,8 @@ def run_ours(args, rank, world, local_rank):
         "score_roofline": {"bound": "hbm", "bytes": sbytes,
                            "achieved": round(sbytes / (score_med * 1e-3) / 1e9, 1),
                            "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": round(sbytes / (score_med * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+                           "frac": round(sbytes / (score_med * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                           "floor": score_floor(w, peaks, score_med)},
         "plan_reuse": {"every": args.reuse,
                        "ms_per_step": round(reuse_ms, 4),
                        "value": round(world * dense / (reuse_ms * 1e-3) / 1e12, 2),
@@ -654,7 +673,8 @@ def other_workloads(ab, dev, args, peaks, calls):
                                  "achieved": round(sbytes / (s0["score_ms"]["median"] * 1e-3) / 1e9, 1),
                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                  "frac": round(sbytes / (s0["score_ms"]["median"] * 1e-3) / 1e9 /
-                                               peaks["hbm_gbs"], 4)}
+                                               peaks["hbm_gbs"], 4),
+                                 "floor": score_floor(w, peaks, s0["score_ms"]["median"])}
         a_tf = s0["attn_selected_tflops"]
         rec["attn_roofline"] = {"bound": "tensor", "achieved": a_tf, "peak": peaks["bf16_tflops"],
                                 "unit": "TFLOP/s", "frac": round(a_tf / peaks["bf16_tflops"], 4)}

@@ -101,8 +101,13 @@ cudaError_t meankey_and_kmeans(cudaStream_t cs, MeanKey meankey, KMeans kmeans)
     if (e != cudaSuccess) return e;
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     e = cudaStreamIsCapturing(cs, &cap);
-    if (e != cudaSuccess || cap != cudaStreamCaptureStatusNone || dev < 0 || dev >= kMaxSideDevices) {
-        (void)cudaGetLastError();  // a capture-status query refused on the legacy stream
+    if (e != cudaSuccess) {
+        // the query is refused for the legacy stream while another stream captures in
+        // global mode: clear that error (only it) and launch in order
+        (void)cudaGetLastError();
+        cap = cudaStreamCaptureStatusActive;
+    }
+    if (cap != cudaStreamCaptureStatusNone || dev < 0 || dev >= kMaxSideDevices) {
         e = meankey(cs);
         return e == cudaSuccess ? kmeans(cs) : e;
     }
