@@ -36,6 +36,8 @@ median and min; "cold" = a 256 MB buffer written before each call to flush L2):
                  extrapolated to a whole step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Profiling runs: --config NAME --heads H --headline-only (the headline step only) or
+--units-only (the 4-token unit step only), both without the CPU leg (--no-cpu-baseline).
 For N > 1 run under torchrun: every rank runs the headline workload on its own data
 (weak scaling over independent batches, no data-path collective); the step time is the
 max over ranks.
@@ -345,6 +347,13 @@ def run_ours(args, rank, world, local_rank):
     frac = args.budget if args.budget is not None else (
         HEADLINE[1] if args.config == HEADLINE[0] else w.budgets[0])
     K = w.budget_blocks(frac)
+    if args.units_only:
+        # only the 4-token unit step of this workload (profiling and unit comparisons)
+        r = Runner(ab, w, dev)
+        return {"metric": "4-token unit step (unit scores, SIP over units, unit attention)",
+                "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} (N_pad={w.N_pad}) "
+                                       f"d={w.d}, {32 * K} units per query block"},
+                "units4": units4(r, K, max(3, args.calls))}
     r = Runner(ab, w, dev, keep_host=True)
     q, d, nb = r.q, r.d, r.nb
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -833,6 +842,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the extra cases and workloads (profiling runs)")
+    ap.add_argument("--units-only", action="store_true",
+                    help="run only the 4-token unit step of --config (profiling runs)")
     ap.add_argument("--reuse", type=int, default=4,
                     help="plan reuse period for the amortised-step measurement")
     ap.add_argument("--traffic", type=float, default=None,
