@@ -242,8 +242,10 @@ __global__ void __launch_bounds__(256) meankey4_kernel(const __nv_bfloat16 *__re
 // (b, h, query block). The block's queries arrive by TMA (128-byte swizzle; rows past
 // N read as zero) and stay in shared memory for all T iterations. Each iteration runs
 // two single-CTA tcgen05 GEMMs with fp32 accumulators in TMEM:
-//   assign: G = Q B^T (M = 128 queries, N = 32, K = d): rows 8t + c of B hold term t
-//           (split3_bits) of fp32 centroid c, rows 24..31 are zero, so q . c =
+//   assign: G = Q B^T (M = 128 queries, N = 32, K = d): columns 8t + c of B hold term
+//           t (split3_bits) of fp32 centroid c, columns 24..31 are zero (B is stored
+//           MN-major, so each thread writes its feature's 24 terms as three 16-byte
+//           chunks), so q . c =
 //           G[q][c] + G[q][8 + c] + G[q][16 + c] is the bf16 query times the fp32
 //           centroid; distance |c|^2 - 2 q.c (|q|^2 is common), argmin with ties to
 //           the lowest cluster; thread t reads TMEM lane t = query t;
@@ -264,8 +266,8 @@ __global__ void __launch_bounds__(256) meankey4_kernel(const __nv_bfloat16 *__re
 template <int D>
 struct KmSmem {
     static constexpr int kQ = 0;                        // queries: 2 panels [128][64] bf16
-    static constexpr int kBA = kQ + 2 * 16384;          // centroid terms: (D/64) x [32][64]
-    static constexpr int kBU = kBA + (D / 64) * 4096;   // one-hot: 2 panels [16][64]
+    static constexpr int kBA = kQ + 2 * 16384;          // centroid terms: [D][64], MN-major
+    static constexpr int kBU = kBA + D * 128;           // one-hot: 2 panels [16][64]
     static constexpr int kBar = kBU + 2 * 2048;         // q_full, mma_done, drain
     static constexpr int kMisc = kBar + 3 * 8;          // TMEM base, abort flag
     static constexpr int kBytes = kMisc + 8;
@@ -282,23 +284,32 @@ template <int D, bool kFirst = false>
 __device__ __forceinline__ void km_publish(uint8_t *smem, const float (&cur)[8], int k,
                                            bool has_k, int warp, int lane, float (*normw)[4])
 {
-    uint16_t *ba = reinterpret_cast<uint16_t *>(smem + KmSmem<D>::kBA);
+    // The assignment GEMM's B operand is stored MN-major (the 8 clusters of a term are
+    // contiguous): row k of the 128-byte-swizzled tile holds feature k, its 16-byte chunk
+    // t the bf16 term t of the 8 centroids (chunk 3, the zero rows 24..31, stays zero).
     float sq[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        sq[c] = cur[c] * cur[c];
-        if (has_k) {
-            // rows c, 8 + c, 16 + c share the swizzle phase (row mod 8 = c)
-            const int o = (sw128_chunk(c, k, 4096) >> 1) + (k & 7);
+    for (int c = 0; c < 8; ++c) sq[c] = cur[c] * cur[c];
+    if (has_k) {
+        uint32_t t[3][8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
             if (kFirst) {
-                ba[o] = (uint16_t)(__float_as_uint(cur[c]) >> 16);
+                t[0][c] = __float_as_uint(cur[c]);
+                t[1][c] = t[2][c] = 0u;
             } else {
-                uint32_t t0, t1, t2;
-                split3_bits(cur[c], t0, t1, t2);
-                ba[o] = (uint16_t)(t0 >> 16);
-                ba[o + 8 * 64] = (uint16_t)(t1 >> 16);
-                ba[o + 16 * 64] = (uint16_t)(t2 >> 16);
+                split3_bits(cur[c], t[0][c], t[1][c], t[2][c]);
             }
+        }
+        uint8_t *row = smem + KmSmem<D>::kBA + k * 128;
+#pragma unroll
+        for (int tt = 0; tt < 3; ++tt) {
+            // two bf16 per 32-bit word: the upper halves of the fp32 patterns of c, c + 1
+            const uint4 v = make_uint4(__byte_perm(t[tt][0], t[tt][1], 0x7632),
+                                       __byte_perm(t[tt][2], t[tt][3], 0x7632),
+                                       __byte_perm(t[tt][4], t[tt][5], 0x7632),
+                                       __byte_perm(t[tt][6], t[tt][7], 0x7632));
+            *reinterpret_cast<uint4 *>(row + ((tt ^ (k & 7)) << 4)) = v;
         }
     }
     // reduce-scatter across the warp: lane L ends with cluster (L >> 2) & 7
@@ -366,11 +377,11 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
         tmem_alloc(tmem_slot, kKmTmemCols);
         tmem_relinquish();
     }
-    // zero rows: centroid-term rows 8..31 (the initial centroids' middle and low terms,
-    // then the constant padding rows 24..31), one-hot rows 8..15
-    for (int e = tid; e < (D / 64) * 192; e += 128)
-        *reinterpret_cast<uint4 *>(smem + L::kBA + (e / 192) * 4096 + (8 + (e % 192) / 8) * 128 +
-                                   (e & 7) * 16) = make_uint4(0, 0, 0, 0);
+    // zero: the constant padding clusters 24..31 of the centroid terms (chunk 3 of every
+    // feature row), one-hot rows 8..15
+    if (tid < D)
+        *reinterpret_cast<uint4 *>(smem + L::kBA + tid * 128 + ((3 ^ (tid & 7)) << 4)) =
+            make_uint4(0, 0, 0, 0);
     *reinterpret_cast<uint4 *>(smem + L::kBU + (tid >> 6) * 2048 + (8 + ((tid >> 3) & 7)) * 128 +
                                (tid & 7) * 16) = make_uint4(0, 0, 0, 0);
     tc_fence_before();
@@ -401,10 +412,10 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
 
     const uint32_t q_addr = smem_u32(smem + L::kQ);
     const uint64_t a_asg = smem_desc_sw128(q_addr, 16, 1024);
-    const uint64_t b_asg = smem_desc_sw128(smem_u32(smem + L::kBA), 16, 1024);
+    const uint64_t b_asg = smem_desc_sw128(smem_u32(smem + L::kBA), 16384, 1024);  // MN-major
     const uint64_t a_upd = smem_desc_sw128(q_addr, 16384, 1024);  // feature-major view of Q
     const uint64_t b_upd = smem_desc_sw128(smem_u32(smem + L::kBU), 16, 1024);
-    constexpr uint32_t idesc_asg = idesc_bf16_f32(128, 32, 0, 0);
+    constexpr uint32_t idesc_asg = idesc_bf16_f32(128, 32, 0, 1);
     constexpr uint32_t idesc_upd = idesc_bf16_f32(128, 16, 1, 0);
     const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
     uint32_t phase = 0;
@@ -417,7 +428,7 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem, a_asg + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                           b_asg + (uint64_t)(((kk >> 2) * 4096 + (kk & 3) * 32) >> 4), idesc_asg,
+                           b_asg + (uint64_t)((kk * 2048) >> 4), idesc_asg,
                            kk > 0 ? 1u : 0u);
                 mma_commit(mma_done);
             }
