@@ -267,7 +267,7 @@ template <int D>
 struct KmSmem {
     static constexpr int kQ = 0;                        // queries: 2 panels [128][64] bf16
     static constexpr int kBA = kQ + 2 * 16384;          // centroid terms: [D][64], MN-major
-    static constexpr int kBU = kBA + D * 128;           // one-hot: 2 panels [16][64]
+    static constexpr int kBU = kBA + D * 128;           // one-hot: [128 queries][16], MN-major
     static constexpr int kBar = kBU + 2 * 2048;         // q_full, mma_done, drain
     static constexpr int kMisc = kBar + 3 * 8;          // TMEM base, abort flag
     static constexpr int kBytes = kMisc + 8;
@@ -382,8 +382,8 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
     if (tid < D)
         *reinterpret_cast<uint4 *>(smem + L::kBA + tid * 128 + ((3 ^ (tid & 7)) << 4)) =
             make_uint4(0, 0, 0, 0);
-    *reinterpret_cast<uint4 *>(smem + L::kBU + (tid >> 6) * 2048 + (8 + ((tid >> 3) & 7)) * 128 +
-                               (tid & 7) * 16) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4 *>(smem + L::kBU + tid * 32 + ((1 ^ ((tid >> 2) & 1)) << 4)) =
+        make_uint4(0, 0, 0, 0);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -414,9 +414,11 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
     const uint64_t a_asg = smem_desc_sw128(q_addr, 16, 1024);
     const uint64_t b_asg = smem_desc_sw128(smem_u32(smem + L::kBA), 16384, 1024);  // MN-major
     const uint64_t a_upd = smem_desc_sw128(q_addr, 16384, 1024);  // feature-major view of Q
-    const uint64_t b_upd = smem_desc_sw128(smem_u32(smem + L::kBU), 16, 1024);
+    // MN-major, 32-byte swizzle: 8-row groups of 256 bytes
+    const uint64_t b_upd = (smem_desc_sw128(smem_u32(smem + L::kBU), 16, 256) & ~(7ull << 61)) |
+                           (6ull << 61);
     constexpr uint32_t idesc_asg = idesc_bf16_f32(128, 32, 0, 1);
-    constexpr uint32_t idesc_upd = idesc_bf16_f32(128, 16, 1, 0);
+    constexpr uint32_t idesc_upd = idesc_bf16_f32(128, 16, 1, 1);
     const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
     uint32_t phase = 0;
 
@@ -469,12 +471,18 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
             lab[tid] = (uint8_t)a;
             const unsigned chg = __ballot_sync(0xffffffffu, changed);
             if (lane == 0) wchanged[warp] = chg != 0u;
-            // (2) one-hot column of this query (B of the update GEMM) and member counts
-            __nv_bfloat16 *oh = reinterpret_cast<__nv_bfloat16 *>(smem + L::kBU);
+            // (2) one-hot row of this query (B of the update GEMM, MN-major with the 32-byte
+            // swizzle: row tid holds clusters 0..7 in its first 16-byte chunk, 8..15 zero in
+            // the other) and member counts
+            {
+                const uint32_t one = a < 8 ? 0x3F80u << (16 * (a & 1)) : 0u;
+                const int wsel = a >> 1;
+                *reinterpret_cast<uint4 *>(smem + L::kBU + tid * 32 + (((tid >> 2) & 1) << 4)) =
+                    make_uint4(wsel == 0 ? one : 0u, wsel == 1 ? one : 0u, wsel == 2 ? one : 0u,
+                               wsel == 3 ? one : 0u);
+            }
 #pragma unroll
             for (int c = 0; c < CMAX; ++c) {
-                oh[(sw128_chunk(c, tid, 2048) >> 1) + (tid & 7)] =
-                    __ushort_as_bfloat16(a == c ? (unsigned short)0x3F80u : (unsigned short)0u);
                 const unsigned m = __ballot_sync(0xffffffffu, a == c);
                 if (lane == 0) wcount[c][warp] = __popc(m);
             }
@@ -495,7 +503,7 @@ __global__ void __launch_bounds__(128, 4) kmeans_kernel(const __grid_constant__ 
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tmem + 32, a_upd + (uint64_t)((kk * 2048) >> 4),
-                           b_upd + (uint64_t)(((kk >> 2) * 2048 + (kk & 3) * 32) >> 4), idesc_upd,
+                           b_upd + (uint64_t)((kk * 512) >> 4), idesc_upd,
                            kk > 0 ? 1u : 0u);
                 mma_commit(mma_done);
             }
