@@ -53,10 +53,11 @@ def lib():
         L.orc_attn_rows.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P, i64, P, P, P, P,
                                     P]
         L.orc_dense_attn.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P]
+        L.orc_attn_bwd.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P]
         L.orc_num_threads.argtypes = []
         for name in ("orc_mean_key", "orc_kmeans", "orc_score", "orc_sip", "orc_topk",
                      "orc_attn_rows", "orc_dense_attn", "orc_num_threads", "orc_mean_key_u",
-                     "orc_score_u", "orc_attn_rows_u"):
+                     "orc_score_u", "orc_attn_rows_u", "orc_attn_bwd"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -201,6 +202,24 @@ def attn_rows(q, k, v, N: int, idx, cnt, w=None, rows=None, want_num_den: bool =
     if rc:
         raise ValueError(f"orc_attn_rows rc={rc}")
     return out, lse, num, den
+
+
+def attn_bwd(q, k, v, do, N: int, idx, cnt, w=None):
+    """Gradients (dQ, dK, dV), fp64 [B,H,N_pad,d], of the block-sparse HT attention over
+    key blocks for the upstream gradient `do` (bf16) of its output; w None = top-k."""
+    qb_, kb_, vb_, gb_ = _bits(q), _bits(k), _bits(v), _bits(do)
+    B, H, N_pad, d = qb_.shape
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    cnt = np.ascontiguousarray(cnt, dtype=np.int32)
+    wv = None if w is None else np.ascontiguousarray(w, dtype=np.float32)
+    dq = np.zeros((B, H, N_pad, d), dtype=np.float64)
+    dk = np.zeros_like(dq)
+    dv = np.zeros_like(dq)
+    rc = lib().orc_attn_bwd(_ptr(qb_), _ptr(kb_), _ptr(vb_), _ptr(gb_), B, H, N, N_pad, d,
+                            _ptr(idx), _ptr(cnt), _ptr(wv), _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc:
+        raise ValueError(f"orc_attn_bwd rc={rc}")
+    return dq, dk, dv
 
 
 def dense_attn(q, k, v, N: int):

@@ -29,7 +29,8 @@
  * closed forms (sum of scores = 1, sum of p = K, p = 1/4 -> w = 4); torch SDPA in fp64
  * for the all-blocks case, top-k case and integer-weight duplication case; exact
  * rational water-filling; Monte Carlo unbiasedness; Philox against an independent
- * implementation.
+ * implementation; torch autograd in fp64 of the masked, log-weight-shifted softmax
+ * attention for the gradients, and the softmax's shift invariance (sum_t dK_t = 0).
  */
 #include <math.h>
 #include <stdint.h>
@@ -658,6 +659,126 @@ int orc_dense_attn(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int 
             if (lse) lse[r] = m + log(z);
         }
         free(row);
+    }
+    return rc;
+}
+
+/* ------------------------------------------------------------------------------
+ * Gradient of the block-sparse HT attention above (key blocks of 128 tokens) with
+ * respect to Q, K and V, for an upstream gradient dO of the output. The weights and
+ * the selection are constants (the selection is a sample, not a differentiable
+ * function of Q or K). With the loss L = sum_i dO_i . O_i, per valid query row i of
+ * query block qb and every valid key t of its kept blocks j:
+ *   P_it  = w_j e^{q_i.k_t/sqrt(d)} / sum_{j',t'} w_j' e^{q_i.k_t'/sqrt(d)}  (O_i = sum_t P_it v_t)
+ *   dV_t += P_it dO_i
+ *   dP_it = dO_i . v_t,   D_i = dO_i . O_i = sum_t P_it dP_it
+ *   dS_it = P_it (dP_it - D_i)          (derivative through the softmax)
+ *   dQ_i += dS_it k_t / sqrt(d),   dK_t += dS_it q_i / sqrt(d)
+ * Rows i >= N and rows with an empty selection contribute nothing and get dQ_i = 0;
+ * keys t >= N get dK_t = dV_t = 0. dO is bf16 bits like Q, K, V; dQ, dK, dV are fp64
+ * [B,H,N_pad,d]. w = NULL means all weights 1 (top-k). Work is split over the (b, h)
+ * pairs, each pair's rows taken in order, so the sums over query rows into dK and dV
+ * run in a fixed order.
+ * ------------------------------------------------------------------------------ */
+int orc_attn_bwd(const uint16_t *Q, const uint16_t *K, const uint16_t *V, const uint16_t *dO,
+                 int B, int H, int N, int N_pad, int d, const int32_t *idx, const int32_t *cnt,
+                 const float *w, double *dQ, double *dK, double *dV)
+{
+    if (!Q || !K || !V || !dO || !idx || !cnt || !dQ || !dK || !dV ||
+        check_shape(B, H, N, N_pad, d))
+        return -1;
+    const int64_t nb = n_blocks_of(N_pad);
+    const int64_t BH = (int64_t)B * H;
+    for (int64_t r = 0; r < BH * nb; ++r) {
+        if (cnt[r] < 0 || cnt[r] > nb) return -1;
+        for (int32_t c = 0; c < cnt[r]; ++c) {
+            if (idx[r * nb + c] < 0 || idx[r * nb + c] >= nb) return -1;
+            if (w && !(w[r * nb + c] > 0.0f && isfinite(w[r * nb + c]))) return -1;
+        }
+    }
+    const int64_t total = BH * N_pad * d;
+    for (int64_t e = 0; e < total; ++e) dQ[e] = dK[e] = dV[e] = 0.0;
+    const double scale = 1.0 / sqrt((double)d);
+    int rc = 0;
+#pragma omp parallel
+    {
+        const int64_t max_keys = nb * ORC_BLOCK;
+        double *pr = (double *)malloc(sizeof(double) * max_keys);
+        int64_t *key = (int64_t *)malloc(sizeof(int64_t) * max_keys);
+        double *qv = (double *)malloc(sizeof(double) * d);
+        double *gv = (double *)malloc(sizeof(double) * d);
+        double *ov = (double *)malloc(sizeof(double) * d);
+        if (!pr || !key || !qv || !gv || !ov) {
+#pragma omp atomic write
+            rc = -2;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < BH; ++bh) {
+            if (rc) continue;
+            const uint16_t *Qh = Q + bh * N_pad * d, *Kh = K + bh * N_pad * d;
+            const uint16_t *Vh = V + bh * N_pad * d, *Gh = dO + bh * N_pad * d;
+            double *dQh = dQ + bh * N_pad * d, *dKh = dK + bh * N_pad * d;
+            double *dVh = dV + bh * N_pad * d;
+            for (int64_t qb = 0; qb < nb; ++qb) {
+                const int64_t r = bh * nb + qb;
+                for (int i = 0; i < ORC_BLOCK; ++i) {
+                    const int64_t tq = qb * ORC_BLOCK + i;
+                    if (tq >= N) continue;
+                    for (int e = 0; e < d; ++e) {
+                        qv[e] = bf16_val(Qh[tq * d + e]);
+                        gv[e] = bf16_val(Gh[tq * d + e]);
+                    }
+                    /* logits (with ln w_j) of the valid keys of the kept blocks */
+                    int64_t nk = 0;
+                    double m = -INFINITY;
+                    for (int32_t c = 0; c < cnt[r]; ++c) {
+                        const int64_t j = idx[r * nb + c];
+                        const double lw = w ? log((double)w[r * nb + c]) : 0.0;
+                        for (int t = 0; t < ORC_BLOCK; ++t) {
+                            const int64_t tk = j * ORC_BLOCK + t;
+                            if (tk >= N) break;
+                            double dot = 0.0;
+                            for (int e = 0; e < d; ++e) dot += qv[e] * bf16_val(Kh[tk * d + e]);
+                            pr[nk] = dot * scale + lw;
+                            key[nk] = tk;
+                            if (pr[nk] > m) m = pr[nk];
+                            ++nk;
+                        }
+                    }
+                    if (nk == 0) continue;
+                    /* softmax probabilities and the output row */
+                    double z = 0.0;
+                    for (int64_t a = 0; a < nk; ++a) {
+                        pr[a] = exp(pr[a] - m);
+                        z += pr[a];
+                    }
+                    for (int e = 0; e < d; ++e) ov[e] = 0.0;
+                    for (int64_t a = 0; a < nk; ++a) {
+                        pr[a] /= z;
+                        for (int e = 0; e < d; ++e) ov[e] += pr[a] * bf16_val(Vh[key[a] * d + e]);
+                    }
+                    double Di = 0.0;
+                    for (int e = 0; e < d; ++e) Di += gv[e] * ov[e];
+                    /* gradients */
+                    for (int64_t a = 0; a < nk; ++a) {
+                        const int64_t tk = key[a];
+                        double dp = 0.0;
+                        for (int e = 0; e < d; ++e) dp += gv[e] * bf16_val(Vh[tk * d + e]);
+                        const double ds = pr[a] * (dp - Di);
+                        for (int e = 0; e < d; ++e) {
+                            dVh[tk * d + e] += pr[a] * gv[e];
+                            dQh[tq * d + e] += ds * bf16_val(Kh[tk * d + e]) * scale;
+                            dKh[tk * d + e] += ds * qv[e] * scale;
+                        }
+                    }
+                }
+            }
+        }
+        free(pr);
+        free(key);
+        free(qv);
+        free(gv);
+        free(ov);
     }
     return rc;
 }
