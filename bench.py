@@ -30,14 +30,17 @@ median and min; "cold" = a 256 MB buffer written before each call to flush L2):
                  refreshed every 4 steps;
   dense_attn     the attention kernel with every key block kept;
   units4         the pages' 4-token key units at the same tile budget;
+  backward       (HunyuanVideo-720p and Wan2.1-1.3B) the gradient of the attention with
+                 respect to Q, K, V for the SIP plan;
   e2e            the headline step through the public API with host buffers (pinned
                  H2D of Q, K, V and D2H of O inside the timed region);
   cpu_baseline   the CPU oracle on a bounded sample of the headline workload,
                  extrapolated to a whole step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-Profiling runs: --config NAME --heads H --headline-only (the headline step only) or
---units-only (the 4-token unit step only), both without the CPU leg (--no-cpu-baseline).
+Profiling runs: --config NAME --heads H --headline-only (the headline step only),
+--units-only (the 4-token unit step only) or --bwd-only (the attention backward only),
+each without the CPU leg (--no-cpu-baseline).
 For N > 1 run under torchrun: every rank runs the headline workload on its own data
 (weak scaling over independent batches, no data-path collective); the step time is the
 max over ranks.
@@ -354,6 +357,13 @@ def run_ours(args, rank, world, local_rank):
                 "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} (N_pad={w.N_pad}) "
                                        f"d={w.d}, {32 * K} units per query block"},
                 "units4": units4(r, K, max(3, args.calls))}
+    if args.bwd_only:
+        # only the attention backward of this workload (profiling)
+        r = Runner(ab, w, dev)
+        return {"metric": "attention backward (dQ, dK, dV) for the SIP plan",
+                "config": {"workload": f"{w.name}: B={w.B} H={w.H} N={w.N} (N_pad={w.N_pad}) "
+                                       f"d={w.d}, {K} of {w.n_blocks} key blocks"},
+                "backward": backward(r, K, peaks, max(3, args.calls))}
     r = Runner(ab, w, dev, keep_host=True)
     q, d, nb = r.q, r.d, r.nb
     flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -620,6 +630,40 @@ def dense_attn(r, peaks, calls):
             "note": "same kernel, every key block kept (budget n_kb, weights 1)"}
 
 
+def backward(r, K, peaks, calls):
+    """The attention backward (dQ, dK, dV) for the SIP plan at budget K: the forward once
+    for O and lse, a seeded upstream gradient dO, then per-call events of ab_attn_bwd.
+    Algorithmic work per kept pair: the five 128 x 128 x d products of the gradient
+    (S and dP recomputed, dV, dK, dQ) = 10 * 128 * 128 * d FLOP; the kernels run seven
+    (S and dP in both the query-major and the key-major pass)."""
+    ab, w, dev = r.ab, r.w, r.dev
+    r.score()
+    r.select(K, "sip")
+    out, lse = ab.attn_fwd(r.q, r.k, r.v, w.N, r.idx, r.cnt, r.wt, want_lse=True, dev_flag=r.flag)
+    g = torch.Generator(device=dev).manual_seed(11)
+    dout = torch.randn(r.q.shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    dout[:, :, w.N:] = 0
+    ws = torch.empty(ab.attn_bwd_workspace_bytes(ab.make_shape(r.q, w.N)), device=dev, dtype=torch.uint8)
+
+    def bwd():
+        return ab.attn_bwd(r.q, r.k, r.v, w.N, r.idx, r.cnt, r.wt, out, lse, dout,
+                           dev_flag=r.flag, workspace=ws)
+
+    bwd()
+    torch.cuda.synchronize()
+    t = stats(time_calls(bwd, calls))
+    t_fwd = stats(time_calls(lambda: r.attn("sip"), calls))
+    r.check("backward")
+    pairs = r.sum_cnt()
+    flop = 2.5 * selected_flops(pairs, r.d)
+    tf = flop / (t["median"] * 1e-3) / 1e12
+    return {"budget": K, "sum_cnt": pairs, "bwd_ms": t, "fwd_ms": t_fwd,
+            "bwd_over_fwd": round(t["median"] / t_fwd["median"], 3),
+            "bwd_tflops": round(tf, 2), "frac": round(tf / peaks["bf16_tflops"], 4),
+            "note": "gradients of Q, K, V (fp32) for the SIP plan; TFLOP/s on the five "
+                    "products per kept pair, against the burst bf16 peak"}
+
+
 def units4(r, K, calls):
     """The pages' 4-token key units at the same tile budget (32 units per 128-key tile):
     unit scores -> SIP over units -> attention over the gathered units."""
@@ -689,6 +733,7 @@ def other_workloads(ab, dev, args, peaks, calls):
                                 "unit": "TFLOP/s", "frac": round(a_tf / peaks["bf16_tflops"], 4)}
         if name in ("wan13b", "hunyuan720"):
             rec["dense_attn"] = dense_attn(r, peaks, calls=max(1, min(3, calls)))
+            rec["backward"] = backward(r, w.budget_blocks(w.budgets[0]), peaks, calls)
         if w.N_pad // 4 <= ab.MAX_UNITS:
             try:
                 rec["units4"] = units4(r, w.budget_blocks(w.budgets[0]), calls)
@@ -844,6 +889,8 @@ def main():
                     help="skip the extra cases and workloads (profiling runs)")
     ap.add_argument("--units-only", action="store_true",
                     help="run only the 4-token unit step of --config (profiling runs)")
+    ap.add_argument("--bwd-only", action="store_true",
+                    help="run only the attention backward of --config (profiling runs)")
     ap.add_argument("--reuse", type=int, default=4,
                     help="plan reuse period for the amortised-step measurement")
     ap.add_argument("--traffic", type=float, default=None,

@@ -76,6 +76,9 @@ def lib():
         L.ab_select.argtypes = [P, I, I, I, I, I, I, ctypes.c_uint64, P, P, P, P, P, P]
         L.ab_attn_fwd.argtypes = [P, P, P, S, P, P, P, P, I, P, P, P]
         L.ab_attn_topk_fwd.argtypes = [P, P, P, S, P, P, P, I, P, P, P]
+        L.ab_attn_bwd_workspace_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
+        L.ab_attn_bwd.argtypes = [P, P, P, S, P, P, P, P, I, P, P, P, P, P, P, ctypes.c_size_t,
+                                  P, P]
         L.ab_score_units_workspace_size.argtypes = [S, I, I, ctypes.POINTER(ctypes.c_size_t)]
         L.ab_score_units.argtypes = [P, P, S, I, I, I, P, P, P, P, P, P, ctypes.c_size_t, P, P]
         L.ab_attn_units_fwd.argtypes = [P, P, P, S, I, P, P, P, P, I, P, P, P]
@@ -263,6 +266,37 @@ def attn_topk_fwd(q, k, v, N: int, idx, cnt, want_lse: bool = False,
                                             _ptr(lse), _ptr(dev_flag), _stream()),
                "ab_attn_units_topk_fwd")
     return (o, lse) if want_lse else o
+
+
+def attn_bwd_workspace_bytes(shape: Shape) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().ab_attn_bwd_workspace_size(shape, ctypes.byref(n)), "ab_attn_bwd_workspace_size")
+    return n.value
+
+
+def attn_bwd(q, k, v, N: int, idx, cnt, w, out, lse, dout,
+             dev_flag: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+    """Gradients (dq, dk, dv), fp32 [B,H,N_pad,d], of attn_fwd (w given) or attn_topk_fwd
+    (w None) over key blocks, for the upstream gradient `dout` (bf16) of the output
+    `out` (bf16 or fp32) whose lse the forward returned."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _need(t, torch.bfloat16, n)
+    _need(idx, torch.int32, "idx")
+    _need(cnt, torch.int32, "cnt")
+    if w is not None:
+        _need(w, torch.float32, "w")
+    _need(out, out.dtype, "out")
+    _need(lse, torch.float32, "lse")
+    shape = make_shape(q, N)
+    need = attn_bwd_workspace_bytes(shape)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq, dk, dv = (torch.empty(q.shape, device=q.device, dtype=torch.float32) for _ in range(3))
+    _check(lib().ab_attn_bwd(_ptr(q), _ptr(k), _ptr(v), shape, _ptr(idx), _ptr(cnt), _ptr(w),
+                             _ptr(out), _out_code(out.dtype), _ptr(lse), _ptr(dout), _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(),
+                             _ptr(dev_flag), _stream()), "ab_attn_bwd")
+    return dq, dk, dv
 
 
 def selftest_bounded_wait(limit_us: int, complete: bool, device="cuda"):

@@ -11,7 +11,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libab_attn.so")
 SOURCES = ["ab_api.cu", "score_kernels.cu", "select_kernels.cu", "attn_kernel.cu", "ab_noalloc.cu",
-           "ab_selftest.cu", "ab_host.cu"]
+           "ab_selftest.cu", "ab_host.cu", "attn_bwd_kernel.cu"]
 HEADERS = ["ab_device.cuh", "ab_kernels.h", os.path.join("..", "..", "include", "ab_attn.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

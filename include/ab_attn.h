@@ -294,6 +294,45 @@ ab_status ab_attn_topk_fwd(const void *q, const void *k, const void *v, ab_shape
                            float *lse, int *dev_flag, void *stream);
 
 /*
+ * ab_attn_bwd_workspace_size -- bytes of device scratch ab_attn_bwd() needs for shape s:
+ * two fp32 values per query row and a uint16 table of n_qb x n_kb entries per head,
+ * each region 256-byte aligned. Errors: AB_ERR_NULL and the shape errors of ab_attn_fwd.
+ */
+ab_status ab_attn_bwd_workspace_size(ab_shape s, size_t *bytes);
+
+/*
+ * ab_attn_bwd -- gradient of ab_attn_fwd (w != NULL) or ab_attn_topk_fwd (w == NULL)
+ * with respect to Q, K and V, for an upstream gradient dO of the output. The plan and
+ * the weights are constants (the selection is a sample, page section «Три приёма
+ * AB-Attention»); the gradient is that of the softmax attention with logits
+ * q_i.k_t/sqrt(d) + ln w_j over the kept blocks: with P_it the attention probabilities
+ * and D_i = dO_i . O_i,
+ *   dV_t = sum_i P_it dO_i,  dS_it = P_it (dO_i . v_t - D_i),
+ *   dQ_i = sum_t dS_it k_t / sqrt(d),  dK_t = sum_i dS_it q_i / sqrt(d).
+ * q, k, v   : bf16 [B,H,N_pad,d] as given to the forward call; d in {64, 128}.
+ * idx, cnt, w : the plan given to the forward call (key blocks of 128 tokens); the
+ *             blocks of a row must be distinct (as ab_select makes them).
+ * out, out_dtype, lse : the forward call's output (AB_BF16 or AB_F32) and its lse.
+ * dout      : bf16 [B,H,N_pad,d], the upstream gradient; rows t >= N are ignored.
+ * dq, dk, dv: out, fp32 [B,H,N_pad,d]; rows t >= N, the rows of a query block with an
+ *             empty selection (dq) and the rows of a key block no query block kept
+ *             (dk, dv) are 0.
+ * workspace : device scratch of ab_attn_bwd_workspace_size() bytes, owned by the
+ *             caller, contents need not be initialised; the call clears its table with
+ *             one memset on `stream`.
+ * Every sum runs in a fixed order: the result is the same on every run.
+ * Device-side: an idx/cnt outside range or a block twice in one row sets
+ * AB_FLAG_BAD_INDEX, a bad weight AB_FLAG_BAD_WEIGHT, a bounded wait that gave up
+ * AB_FLAG_TIMEOUT (the output is then undefined).
+ * Errors: AB_ERR_NULL, AB_ERR_SHAPE, AB_ERR_DTYPE, AB_ERR_UNSUPPORTED, AB_ERR_RANGE,
+ * AB_ERR_ALIGN, AB_ERR_WORKSPACE, AB_ERR_CUDA.
+ */
+ab_status ab_attn_bwd(const void *q, const void *k, const void *v, ab_shape s, const int32_t *idx,
+                      const int32_t *cnt, const float *w, const void *out, ab_dtype out_dtype,
+                      const float *lse, const void *dout, float *dq, float *dk, float *dv,
+                      void *workspace, size_t workspace_bytes, int *dev_flag, void *stream);
+
+/*
  * ab_attn_units_fwd, ab_attn_units_topk_fwd -- the attention of ab_attn_fwd /
  * ab_attn_topk_fwd over selected key units of key_unit tokens (AB_BLOCK, or AB_UNIT4:
  * the page's 4-token units, third technique). idx / cnt / w come from ab_select run on

@@ -208,3 +208,42 @@ def test_forward_host_argument_checks(L):
     assert call(FAKE, FAKE, FAKE, s, 8, 5, 0, 3, u, FAKE, B16, 2, FAKE, need - 1, None, None) == 10
     bad = ab.Shape(1, 4, 1000, 1152, 128, ab.AB_BF16)  # N_pad - N >= 128
     assert call(FAKE, FAKE, FAKE, bad, 8, 5, 0, 3, u, FAKE, B16, 2, FAKE, need, None, None) == 2
+
+
+def test_attn_bwd_argument_checks(L):
+    # every rejection comes before any CUDA call: no device is touched
+    s = ab.Shape(1, 2, 1000, 1024, 128, ab.AB_BF16)
+    n = ctypes.c_size_t(0)
+    assert L.ab_attn_bwd_workspace_size(s, ctypes.byref(n)) == 0
+    # D_i and lse_i log2e per query row (fp32) and the n_kb x n_qb uint16 mark table per head
+    need = 2 * 2 * 1024 * 4 + 2 * 8 * 8 * 2
+    assert need <= n.value <= need + 3 * 256
+    assert L.ab_attn_bwd_workspace_size(s, None) == 1
+    assert L.ab_attn_bwd_workspace_size(ab.Shape(1, 2, 1000, 1024, 96, ab.AB_BF16), ctypes.byref(n)) == 4
+    assert n.value == 0
+    assert L.ab_attn_bwd_workspace_size(s, ctypes.byref(n)) == 0
+    need = n.value
+    B16 = ab.AB_BF16
+    call = L.ab_attn_bwd
+    args = [FAKE, FAKE, FAKE, s, FAKE, FAKE, FAKE, FAKE, B16, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+            need, None, None]
+
+    def with_(**kw):
+        a = list(args)
+        pos = dict(q=0, k=1, v=2, s=3, idx=4, cnt=5, w=6, out=7, odt=8, lse=9, do=10, dq=11,
+                   dk=12, dv=13, ws=14, wsb=15)
+        for key, val in kw.items():
+            a[pos[key]] = val
+        return call(*a)
+
+    for key in ("q", "k", "v", "idx", "cnt", "out", "lse", "do", "dq", "dk", "dv"):
+        assert with_(**{key: None}) == 1, key
+    assert with_(odt=7) == 3
+    assert with_(s=ab.Shape(1, 2, 1000, 1024, 128, 0)) == 3
+    assert with_(s=ab.Shape(1, 2, 1000, 1152, 128, B16)) == 2
+    assert with_(s=ab.Shape(1, 2, 1000, 1024, 256, B16)) == 4
+    for key in ("q", "dq", "do", "lse", "w", "ws"):
+        assert with_(**{key: MISALIGNED}) == 9, key
+    assert with_(ws=None) == 10
+    assert with_(wsb=need - 1) == 10
+    assert "ab_attn_bwd" in declared_functions()
