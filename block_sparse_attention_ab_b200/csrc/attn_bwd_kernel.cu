@@ -14,22 +14,23 @@
 //   1. row statistics: D_i and lse_i log2e per query row (+inf on rows that take no part:
 //      padding rows and rows of an empty selection, so that their P is 0);
 //   2. the plan transposed into a mark table [bh][key block][query block] holding c + 1
-//      for the plan entry c that keeps the pair (zeroed just before; a second mark of the
-//      same pair is a duplicate block in a row and raises AB_FLAG_BAD_INDEX);
+//      for the plan entry c that keeps the pair, and a count per key block (zeroed just
+//      before; a second mark of the same pair is a duplicate block in a row and raises
+//      AB_FLAG_BAD_INDEX);
 //   3. dQ: one CTA per (b, h, query block), over its kept key blocks in plan order:
 //      S = Q K_j^T and dP = dO V_j^T into TMEM (SS MMAs, both operands K-major), dS packed
-//      to bf16 over S, dQ += dS K_j (TS MMA: dS from TMEM, K_j as an MN-major operand);
+//      to bf16 over dP, dQ += dS K_j (TS MMA: dS from TMEM, K_j as an MN-major operand);
 //   4. dK, dV: one CTA per (b, h, key block), over the query blocks that kept it in
 //      ascending order (read from the mark table): S^T = K Q^T and dP^T = V dO^T, then
 //      dV += P^T dO and dK += dS^T Q (TS MMAs, dO and Q as MN-major operands).
 // Every sum runs in a fixed order, so the result does not depend on scheduling. The two
-// gradient kernels share one structure: 8 warps; warp w reads TMEM lanes 32 (w mod 4) ..
-// +31 (its rows) and half w / 4 of the columns; thread 0 issues the TMA copies and the
-// MMAs; the K/V (dQ kernel) or Q/dO (dK/dV kernel) tiles of the next pair load while the
-// current one is computed (two stages). Tiles arrive by TMA in 64-column boxes with the
-// 128-byte swizzle, as in the forward kernel. Every wait is bounded; a wait that gives up
-// raises AB_FLAG_TIMEOUT, and the CTA lets its copies and MMAs land and frees its tensor
-// memory before it returns. The C entry points ab_attn_bwd and ab_attn_bwd_workspace_size
+// gradient kernels share one structure: warps 0-7 do the elementwise work, warp w on
+// TMEM lanes 32 (w mod 4) .. +31 (its rows) and half w / 4 of the columns; warp 8 issues
+// every TMA copy and MMA. The two hand over through mbarriers (S read, dS stored), so the
+// tensor core runs the next pair's products while the warps work on the current one.
+// Tiles arrive by TMA in 64-column boxes with the 128-byte swizzle, as in the forward
+// kernel. Every wait is bounded; a wait that gives up raises AB_FLAG_TIMEOUT, and the
+// CTA lets its copies and MMAs land and frees its tensor memory before it returns. The C entry points ab_attn_bwd and ab_attn_bwd_workspace_size
 // are at the end of this file.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -49,9 +50,10 @@ namespace ab {
 namespace {
 
 // Workspace regions, each 256-byte aligned: per query row D_i = dO_i . O_i and
-// lse_i log2e (fp32 [BH][N_pad] each), and the plan's mark table uint16 [BH][n_kb][n_qb].
+// lse_i log2e (fp32 [BH][N_pad] each), the plan's mark table uint16 [BH][n_kb][n_qb] and
+// the number of query blocks keeping each key block, uint32 [BH][n_kb].
 struct AttnBwdLayout {
-    size_t rowD, rowL2, mark, total;
+    size_t rowD, rowL2, mark, kcount, total;
 };
 
 AttnBwdLayout attn_bwd_layout(size_t BH, size_t N_pad)
@@ -62,7 +64,8 @@ AttnBwdLayout attn_bwd_layout(size_t BH, size_t N_pad)
     L.rowD = 0;
     L.rowL2 = up(BH * N_pad * sizeof(float));
     L.mark = up(L.rowL2 + BH * N_pad * sizeof(float));
-    L.total = up(L.mark + BH * nb * nb * sizeof(uint16_t));
+    L.kcount = up(L.mark + BH * nb * nb * sizeof(uint16_t));
+    L.total = up(L.kcount + BH * nb * sizeof(uint32_t));
     return L;
 }
 
@@ -80,16 +83,20 @@ struct AttnBwdLaunch {
     int B, H, N, N_pad, d;
 };
 
-constexpr int kBwdThreads = 256;
+constexpr int kBwdThreads = 288;  // 8 compute warps + 1 issuer warp
 constexpr int kBwdTmemCols = 512;
-constexpr int kTileMax = 128 * 128 * 2;     // one 128 x 128 bf16 tile
-constexpr int kBwdSmem = 6 * kTileMax + 1024;  // six tile slots + alignment slack: 1 CTA / SM
+constexpr int kTileMax = 128 * 128 * 2;  // one 128 x 128 bf16 tile
+// dynamic shared memory (+ 1024 bytes of alignment slack), one CTA per SM:
+// dQ: Q, dO and rings of 3 (K) and 2 (V) tiles; dK/dV: K, V and two rings of 2 (Q, dO)
+constexpr int kDqSmem = 7 * kTileMax + 1024;
+constexpr int kDkdvSmem = 6 * kTileMax + 1024;
 
 struct BwdParams {
     const int32_t *idx, *cnt;
     const float *w;  // nullptr: every weight 1 (top-k)
     const float *rowD, *rowL2;
     const uint16_t *mark;
+    const uint32_t *kcount;
     float *dq, *dk, *dv;
     int *flag;
     int N, N_pad, nqb, nkb;
@@ -132,13 +139,21 @@ __device__ __forceinline__ void tma_tile(uint8_t *dst, const CUtensorMap *tm, ui
     for (int x = 0; x < D / 64; ++x) tma_load_3d(dst + x * 16384, tm, bar, x * 64, row_block * 128, bh);
 }
 
-__device__ __forceinline__ float lw2_of(const float *w, int *flag, bool report)
+__device__ __forceinline__ float lw2_val(float wj, int *flag, bool report)
 {
-    if (!w) return 0.f;
-    const float wj = __ldg(w);
     if (wj > 0.f && wj < INFINITY) return fast_log2(wj);
     if (report) raise_flag(flag, AB_FLAG_BAD_WEIGHT);
     return 0.f;
+}
+
+// 2^x for a pair: on the MUFU unit, or (soft) on the FMA pipe by the forward kernel's
+// polynomial (max relative error 7.5e-5); the P step gives every fifth pair to the FMA
+// pipe so that the two units share the exponentials.
+__device__ __forceinline__ float2 exp2_pair(uint64_t x2, bool soft)
+{
+    if (soft) return soft_exp2_pair(x2);
+    const float2 x = f2_unpack(x2);
+    return make_float2(fast_exp2(x.x), fast_exp2(x.y));
 }
 
 // Rows [row0, row0 + 128) of a [.., D] fp32 tensor set to 0 by the whole CTA.
@@ -224,11 +239,11 @@ __global__ void __launch_bounds__(256) attn_bwd_rowstats_kernel(const void *o, c
 
 // ---------------------------------------------------------------------------------
 // 2. Mark table: mark[bh][j][qb] = c + 1 for plan entry c of row (bh, qb) keeping block
-//    j (one warp per plan row).
+//    j, and kcount[bh][j] = the number of query blocks keeping j (one warp per plan row).
 // ---------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) attn_bwd_mark_kernel(const int32_t *idx, const int32_t *cnt,
-                                                            uint16_t *mark, size_t n_rows, int nqb,
-                                                            int nkb, int *flag)
+                                                            uint16_t *mark, uint32_t *kcount,
+                                                            size_t n_rows, int nqb, int nkb, int *flag)
 {
     const size_t r = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -249,26 +264,63 @@ __global__ void __launch_bounds__(256) attn_bwd_mark_kernel(const int32_t *idx, 
         unsigned short *m = reinterpret_cast<unsigned short *>(mark + (bh * nkb + j) * nqb + qb);
         if (atomicCAS(m, (unsigned short)0, (unsigned short)(c + 1)) != 0)
             raise_flag(flag, AB_FLAG_BAD_INDEX);  // block j twice in one row
+        else
+            atomicAdd(kcount + bh * nkb + j, 1u);
     }
 }
 
 // ---------------------------------------------------------------------------------
-// Shared pieces of the two gradient kernels.
+// Shared pieces of the two gradient kernels: warps 0-7 compute (elementwise work on TMEM
+// rows), warp 8 issues every TMA copy and MMA. Barrier slots:
+//   0: the CTA's fixed tiles   1-3: ring A (3 slots in the dQ kernel, 2 in the dK/dV
+//   kernel)   4-5: ring B (2 slots)   6: S (or S^T) done   7: dP (or dP^T) done
+//   8: S read (and P^T stored) (256 arrivals)   9: dS stored, dP read (256 arrivals)
+//   10: a pair's accumulating MMAs done (dK/dV kernel)   11: all MMAs done
+//   12: drain after a failed wait
 // ---------------------------------------------------------------------------------
-struct BwdCta {
-    uint64_t *bars;  // 0: first tiles, 1-2: stage tiles, 3: S/dP done, 4: accumulate done, 5: drain
-    volatile int *abort;
-    int *flag;
+constexpr int kIssuerWarp = 8;
+constexpr int kBars = 13;
+
+// 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16), counted on bar.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(smem_dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// The issuer warp's bounded wait (all lanes agree).
+__device__ __forceinline__ bool issuer_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *flag)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, flag));
+}
+
+// Copies of the issuer still in flight after a failed wait: let them land before the CTA
+// releases its memory. Loads of each ring were issued and waited in order.
+struct Inflight {
+    int issued[3] = {0, 0, 0}, waited[3] = {0, 0, 0};  // 0: fixed tiles, 1: ring A, 2: ring B
 };
 
-// Thread 0's bounded wait.
-__device__ __forceinline__ bool bwd_wait(const BwdCta &c, uint64_t *bar, uint32_t parity)
+__device__ __forceinline__ void drain_issuer(uint64_t *bars, const Inflight &f, int ring_a)
 {
-    return mbar_wait(bar, parity, c.abort, c.flag);
+    if (elect_one()) mma_commit(&bars[12]);
+    __syncwarp();
+    drain_wait(&bars[12], 0);
+    for (int k = f.waited[0]; k < f.issued[0]; ++k) drain_wait(&bars[0], 0);
+    for (int k = f.waited[1]; k < f.issued[1]; ++k) drain_wait(&bars[1 + k % ring_a], (k / ring_a) & 1);
+    for (int k = f.waited[2]; k < f.issued[2]; ++k) drain_wait(&bars[4 + (k & 1)], (k >> 1) & 1);
 }
 
 // ---------------------------------------------------------------------------------
-// 3. dQ: one CTA per (b, h, query block).
+// 3. dQ: one CTA per (b, h, query block). Pipeline per kept block c (K_c in slot c mod 3
+//    of the three-slot ring, V_c in slot c mod 2 of the two-slot ring):
+//      issuer: S(0), dP(0); then for each c: [S(c) read] S(c+1); [dS(c) stored]
+//              dQ += dS(c) K_c, dP(c+1); loads of K, V for c + 2;
+//      compute: [S(c)] P in registers, arrive; [dP(c)] dS packed to bf16 over dP, arrive.
+//    dS sits in the dP columns, so S(c+1) overlaps the dS step and dQ(c), dP(c+1) overlap
+//    the next P step. (Issuing dP(c+1) ahead of dQ(c), with dS in two buffers of the spare
+//    TMEM columns, measured 10% slower.)
 // ---------------------------------------------------------------------------------
 template <int D, bool kW>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -292,16 +344,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem_1024(smem_raw);
     uint8_t *sQ = smem, *sG = smem + kTileMax;
-    __shared__ __align__(8) uint64_t bars[6];
+    auto sK = [&](int slot) { return smem + (2 + slot) * kTileMax; };
+    auto sV = [&](int slot) { return smem + (5 + slot) * kTileMax; };
+    __shared__ __align__(8) uint64_t bars[kBars];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_s;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int b = 0; b < 6; ++b) mbar_init(&bars[b], 1);
+        for (int b = 0; b < kBars; ++b) mbar_init(&bars[b], (b == 8 || b == 9) ? 256 : 1);
         abort_s = 0;
         fence_barrier_init();
     }
-    if (warp == 0) {
+    if (warp == kIssuerWarp) {
         tmem_alloc(&tmem_slot, kBwdTmemCols);
         tmem_relinquish();
     }
@@ -309,126 +363,200 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
-    const uint32_t tS = tmem, tP = tmem + 128, tAcc = tmem + 256;  // S then dS, dP, dQ
-    const BwdCta cta{bars, &abort_s, p.flag};
-    const int grp = warp & 3, half = warp >> 2;
-    const uint32_t lane_off = (uint32_t)(32 * grp) << 16;
-    const int row = 32 * grp + lane;  // query row of the block (TMEM lane)
-    const float L2r = p.rowL2[row0 + row];
-    const float Dr = p.rowD[row0 + row];
+    const uint32_t tS = tmem, tP = tmem + 128, tAcc = tmem + 256;  // S, dP then dS, dQ
     const int32_t *idx = p.idx + (size_t)item * p.nkb;
     const float *wrow = kW ? p.w + (size_t)item * p.nkb : nullptr;
-    auto block_of = [&](int c) {
-        const int j = __ldg(idx + c);
-        if (j >= 0 && j < p.nkb) return j;
-        if (threadIdx.x == 0) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
-        return j < 0 ? 0 : p.nkb - 1;
-    };
-    auto sK = [&](int s) { return smem + (2 + 2 * s) * kTileMax; };
-    auto sV = [&](int s) { return smem + (3 + 2 * s) * kTileMax; };
-    const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-    const uint64_t g_desc = smem_desc_sw128(smem_u32(sG), 16, 1024);
+    auto clamp_j = [&](int j) { return j < 0 ? 0 : (j >= p.nkb ? p.nkb - 1 : j); };
 
-    // thread 0's bookkeeping of copies in flight (for the drain after a failed wait)
-    bool first_done = false;
-    int kv_issued = 0, kv_done = 0;
-    auto issue_kv = [&](int c) {
-        const int j = block_of(c);
-        const int s = c & 1;
-        mbar_arrive_expect_tx(&bars[1 + s], 2 * kTileBytes);
-        tma_tile<D>(sK(s), &tmK, &bars[1 + s], j, bh);
-        tma_tile<D>(sV(s), &tmV, &bars[1 + s], j, bh);
-        ++kv_issued;
-    };
-    bool ok0 = true;  // thread 0: every wait so far succeeded
-    if (threadIdx.x == 0) {
-        prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
-        prefetch_tmap(&tmG);
-        mbar_arrive_expect_tx(&bars[0], 2 * kTileBytes);
-        tma_tile<D>(sQ, &tmQ, &bars[0], qb, bh);
-        tma_tile<D>(sG, &tmG, &bars[0], qb, bh);
-        issue_kv(0);
-    }
-    bool failed = false;
-    for (int c = 0; c < n; ++c) {
-        const int s = c & 1;
-        const int j = block_of(c);
-        const float lw2 = kW ? lw2_of(wrow + c, p.flag, threadIdx.x == 0) : 0.f;
-        if (warp == 0) {
-            if (lane == 0) {
-                if (c == 0) ok0 = first_done = bwd_wait(cta, &bars[0], 0);
-                if (ok0) ok0 = bwd_wait(cta, &bars[1 + s], (c >> 1) & 1);
-                if (ok0) {
-                    ++kv_done;
-                    tc_fence_after();
-                    mma_rows<D>(tS, q_desc, smem_desc_sw128(smem_u32(sK(s)), 16, 1024));
-                    mma_rows<D>(tP, g_desc, smem_desc_sw128(smem_u32(sV(s)), 16, 1024));
-                    mma_commit(&bars[3]);
-                }
-                // the other stage is free once dQ of pair c - 1 is done: load pair c + 1
-                if (ok0 && c >= 1) ok0 = bwd_wait(cta, &bars[4], (c - 1) & 1);
-                if (ok0 && c + 1 < n) issue_kv(c + 1);
+    if (warp == kIssuerWarp) {
+        // ------------------------------ issuer warp ------------------------------
+        Inflight f;
+        auto block_of = [&](int c) {
+            const int j = __ldg(idx + c);
+            if ((j < 0 || j >= p.nkb) && lane == 0) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
+            return clamp_j(j);
+        };
+        auto load_k = [&](int c, int j) {
+            const int slot = c % 3;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&bars[1 + slot], kTileBytes);
+                tma_tile<D>(sK(slot), &tmK, &bars[1 + slot], j, bh);
+            }
+            __syncwarp();
+            ++f.issued[1];
+        };
+        auto load_v = [&](int c, int j) {
+            const int slot = c & 1;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&bars[4 + slot], kTileBytes);
+                tma_tile<D>(sV(slot), &tmV, &bars[4 + slot], j, bh);
+            }
+            __syncwarp();
+            ++f.issued[2];
+        };
+        auto kd = [&](int slot) { return smem_desc_sw128(smem_u32(sK(slot)), 16, 1024); };
+        auto kd_mn = [&](int slot) { return smem_desc_sw128(smem_u32(sK(slot)), 16384, 1024); };
+        auto vd = [&](int slot) { return smem_desc_sw128(smem_u32(sV(slot)), 16, 1024); };
+        const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+        const uint64_t g_desc = smem_desc_sw128(smem_u32(sG), 16, 1024);
+        volatile int *ab = &abort_s;
+        if (elect_one()) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            prefetch_tmap(&tmG);
+            mbar_arrive_expect_tx(&bars[0], 2 * kTileBytes);
+            tma_tile<D>(sQ, &tmQ, &bars[0], qb, bh);
+            tma_tile<D>(sG, &tmG, &bars[0], qb, bh);
+        }
+        __syncwarp();
+        f.issued[0] = 1;
+        {
+            const int j0 = block_of(0);
+            load_k(0, j0);
+            load_v(0, j0);
+        }
+        if (n > 1) {
+            const int j1 = block_of(1);
+            load_k(1, j1);
+            load_v(1, j1);
+        }
+        // the block index of the next pair to load, read one iteration ahead of its use
+        int j_pre = n > 2 ? __ldg(idx + 2) : 0;
+        bool ok = issuer_wait(&bars[0], 0, ab, p.flag);
+        if (ok) f.waited[0] = 1;
+        ok = ok && issuer_wait(&bars[1], 0, ab, p.flag);
+        if (ok) ++f.waited[1];
+        ok = ok && issuer_wait(&bars[4], 0, ab, p.flag);
+        if (ok) {
+            ++f.waited[2];
+            tc_fence_after();
+            if (elect_one()) {
+                mma_rows<D>(tS, q_desc, kd(0));
+                mma_commit(&bars[6]);
+                mma_rows<D>(tP, g_desc, vd(0));
+                mma_commit(&bars[7]);
             }
             __syncwarp();
         }
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[3], c & 1, &abort_s, p.flag));
-        if (ok) {
+        for (int c = 0; ok && c < n; ++c) {
+            // S(c) has been read: S(c + 1) may overwrite it
+            if (!issuer_wait(&bars[8], c & 1, ab, p.flag)) { ok = false; break; }
+            if (c + 1 < n) {
+                const int ks = (c + 1) % 3;
+                if (!issuer_wait(&bars[1 + ks], ((c + 1) / 3) & 1, ab, p.flag)) { ok = false; break; }
+                ++f.waited[1];
+                tc_fence_after();
+                if (elect_one()) {
+                    mma_rows<D>(tS, q_desc, kd(ks));
+                    mma_commit(&bars[6]);
+                }
+                __syncwarp();
+            }
+            // dS(c) stored and dP(c) read: dQ += dS(c) K_c, then dP(c + 1) over it
+            if (!issuer_wait(&bars[9], c & 1, ab, p.flag)) { ok = false; break; }
             tc_fence_after();
-            // P = 2^(s scale_log2 + log2 w - L2) on the valid keys; dS = P (dP - D)
-            const int nvalid = p.N - j * 128;
-            const float bias = lw2 - L2r;
-            uint32_t pk[32];
+            if (elect_one()) {
+                mma_packed<D>(tAcc, tP, kd_mn(c % 3), c > 0);
+                if (c == n - 1) mma_commit(&bars[11]);
+            }
+            __syncwarp();
+            if (c + 1 < n) {
+                const int vs = (c + 1) & 1;
+                if (!issuer_wait(&bars[4 + vs], ((c + 1) >> 1) & 1, ab, p.flag)) { ok = false; break; }
+                ++f.waited[2];
+                tc_fence_after();
+                if (elect_one()) {
+                    mma_rows<D>(tP, g_desc, vd(vs));
+                    mma_commit(&bars[7]);
+                }
+                __syncwarp();
+            }
+            // K_{c-1} (read by dQ(c-1)) and V_c (read by dP(c)) are free: the compute warps
+            // saw dP(c) done, which the pipe ran after dQ(c-1)
+            if (c + 2 < n) {
+                if ((j_pre < 0 || j_pre >= p.nkb) && lane == 0) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
+                const int j2 = clamp_j(j_pre);
+                j_pre = c + 3 < n ? __ldg(idx + c + 3) : 0;
+                load_k(c + 2, j2);
+                load_v(c + 2, j2);
+            }
+        }
+        if (!ok) drain_issuer(bars, f, 3);
+    } else {
+        // ------------------------------ compute warps ------------------------------
+        const int grp = warp & 3, half = warp >> 2;
+        const uint32_t lane_off = (uint32_t)(32 * grp) << 16;
+        const int row = 32 * grp + lane;  // query row of the block (TMEM lane)
+        const float L2r = p.rowL2[row0 + row];
+        const float Dr = p.rowD[row0 + row];
+        volatile int *ab = &abort_s;
+        int j_cur = clamp_j(__ldg(idx));
+        float lw_cur = kW ? lw2_val(__ldg(wrow), p.flag, threadIdx.x == 0) : 0.f;
+        bool ok = true;
+        for (int c = 0; c < n; ++c) {
+            // the next plan entry: loaded here, used only after this pair's work
+            int j_raw = 0;
+            float w_raw = 1.f;
+            if (c + 1 < n) {
+                j_raw = __ldg(idx + c + 1);
+                if (kW) w_raw = __ldg(wrow + c + 1);
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[6], c & 1, ab, p.flag))) { ok = false; break; }
+            tc_fence_after();
+            // P = 2^(s scale_log2 + log2 w - L2) on the valid keys of block j
+            const int nvalid = p.N - j_cur * 128;
+            const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+            const uint64_t b2 = f2_pack(lw_cur - L2r, lw_cur - L2r);
+            float pv[64];
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
-                uint32_t sv[32], dv[32];
+                uint32_t sv[32];
                 tmem_ld32(tS + lane_off + half * 64 + ch * 32, sv);
-                tmem_ld32(tP + lane_off + half * 64 + ch * 32, dv);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int key = half * 64 + ch * 32 + e;
-                    const float p0 = key < nvalid ? fast_exp2(fmaf(__uint_as_float(sv[e]), p.scale_log2, bias)) : 0.f;
-                    const float p1 = key + 1 < nvalid ? fast_exp2(fmaf(__uint_as_float(sv[e + 1]), p.scale_log2, bias)) : 0.f;
-                    pk[ch * 16 + e / 2] = pack_bf16x2(p0 * (__uint_as_float(dv[e]) - Dr),
-                                                      p1 * (__uint_as_float(dv[e + 1]) - Dr));
+                    const float2 r = exp2_pair(
+                        f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, b2),
+                        (ch * 16 + e / 2) % 5 == 4);
+                    pv[ch * 32 + e] = key < nvalid ? r.x : 0.f;
+                    pv[ch * 32 + e + 1] = key + 1 < nvalid ? r.y : 0.f;
                 }
             }
-            tmem_st32(tS + lane_off + half * 64, pk);
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        if (__syncthreads_or(!ok || (threadIdx.x == 0 && !ok0))) {
-            failed = true;
-            break;
-        }
-        if (warp == 0) {
-            if (lane == 0) {
-                tc_fence_after();
-                mma_packed<D>(tAcc, tS, smem_desc_sw128(smem_u32(sK(s)), 16384, 1024), c > 0);
-                mma_commit(&bars[4]);
+            tc_fence_before();
+            mbar_arrive(&bars[8]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[7], c & 1, ab, p.flag))) { ok = false; break; }
+            tc_fence_after();
+            // dS = P (dP - D), packed to bf16 over the first 32 of this half's dP columns
+            uint32_t pk[32];
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t dv[32];
+                tmem_ld32(tP + lane_off + half * 64 + ch * 32, dv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; e += 2)
+                    pk[ch * 16 + e / 2] = pack_bf16x2(pv[ch * 32 + e] * (__uint_as_float(dv[e]) - Dr),
+                                                      pv[ch * 32 + e + 1] * (__uint_as_float(dv[e + 1]) - Dr));
             }
-            __syncwarp();
+            tmem_st32(tP + lane_off + half * 64, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[9]);
+            j_cur = clamp_j(j_raw);
+            lw_cur = kW ? lw2_val(w_raw, p.flag, threadIdx.x == 0) : 0.f;
         }
-    }
-    bool ok_end = !failed;
-    if (ok_end) ok_end = __all_sync(0xffffffffu, mbar_wait(&bars[4], (n - 1) & 1, &abort_s, p.flag));
-    if (ok_end) {
-        tc_fence_after();
-        store_acc_row<D>(tAcc + lane_off + half * (D / 2), p.dq + (row0 + row) * D + half * (D / 2),
-                         p.scale, qb * 128 + row < p.N);
-    }
-    if (threadIdx.x == 0 && (failed || !ok_end)) {
-        // let the copies and MMAs in flight land before the memory is released
-        mma_commit(&bars[5]);
-        drain_wait(&bars[5], 0);
-        if (!first_done) drain_wait(&bars[0], 0);
-        for (int k = kv_done; k < kv_issued; ++k) drain_wait(&bars[1 + (k & 1)], (k >> 1) & 1);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[11], 0, ab, p.flag));
+        if (ok) {
+            tc_fence_after();
+            store_acc_row<D>(tAcc + lane_off + half * (D / 2), p.dq + (row0 + row) * D + half * (D / 2),
+                             p.scale, qb * 128 + row < p.N);
+        }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kIssuerWarp) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kBwdTmemCols);
@@ -436,27 +564,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------
-// 4. dK, dV: one CTA per (b, h, key block).
+// 4. dK, dV: one CTA per (b, h, key block), over the kcount[bh][kb] query blocks that
+//    kept it, ascending, read from the mark column. Pipeline per pair c (Q_c with its
+//    rows' L2 and D, and dO_c, in slot c mod 2 of their rings):
+//      issuer: S^T(0), dP^T(0); then for each c: [P^T(c) stored] dV += P^T dO_c;
+//              [dS^T(c) stored] dK += dS^T Q_c, S^T(c+1), dP^T(c+1); [pair c done]
+//              loads for c + 2 into its slots;
+//      compute: [S^T(c)] P^T packed over S^T, arrive; [dP^T(c)] dS^T packed over dP^T,
+//               arrive.
+//    dV(c) runs while the warps form dS^T(c); dK(c), S^T(c+1) and dP^T(c+1) while they
+//    wait for S^T(c+1) and then form P^T(c+1).
 // ---------------------------------------------------------------------------------
-// The query blocks that kept this key block, in ascending order, from its mark column:
-// every warp walks the column in chunks of 32 (one ballot per chunk), so all warps see
-// the same sequence without talking to each other.
+// Every warp walks the mark column in chunks of 32 (one ballot per chunk, the next
+// chunk's entries already loaded), so all warps see the same sequence without talking
+// to each other.
 struct MarkWalk {
     const uint16_t *col;
     int nqb, base;
-    uint32_t mask, mv;
-    __device__ void load(int b)
+    uint32_t mask, mv, mv_next;
+    __device__ uint32_t raw(int b) const
     {
-        base = b;
         const int q = b + (int)(threadIdx.x & 31);
-        mv = q < nqb ? col[q] : 0u;
+        return q < nqb ? (uint32_t)col[q] : 0u;
+    }
+    __device__ void start()
+    {
+        base = 0;
+        mv = raw(0);
+        mv_next = raw(32);
         mask = __ballot_sync(0xffffffffu, mv != 0);
     }
     __device__ bool next(int &qb, int &c)
     {
         while (mask == 0) {
             if (base + 32 >= nqb) return false;
-            load(base + 32);
+            base += 32;
+            mv = mv_next;
+            mv_next = raw(base + 32);
+            mask = __ballot_sync(0xffffffffu, mv != 0);
         }
         const int l = __ffs(mask) - 1;
         mask &= mask - 1;
@@ -476,38 +621,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int item = blockIdx.x;
     const int bh = item / p.nkb, kb = item % p.nkb;
     const size_t row0 = (size_t)bh * p.N_pad + (size_t)kb * 128;
-    MarkWalk walk{p.mark + (size_t)item * p.nqb, p.nqb, 0, 0u, 0u};
-    walk.load(0);
-    int cur_qb = 0, cur_c = 0, nxt_qb = 0, nxt_c = 0;
-    bool have_cur = walk.next(cur_qb, cur_c);
-    if (!have_cur) {  // no query block kept this key block
+    const int n = (int)min(p.kcount[item], (uint32_t)p.nqb);
+    if (n == 0) {  // no query block kept this key block
         zero_rows<D>(p.dk, row0);
         zero_rows<D>(p.dv, row0);
         return;
     }
-    bool have_nxt = walk.next(nxt_qb, nxt_c);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem_1024(smem_raw);
     uint8_t *sK = smem, *sV = smem + kTileMax;
-    __shared__ __align__(8) uint64_t bars[6];
+    auto sQ = [&](int slot) { return smem + (2 + slot) * kTileMax; };
+    auto sG = [&](int slot) { return smem + (4 + slot) * kTileMax; };
+    __shared__ __align__(8) uint64_t bars[kBars];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_s;
-    __shared__ __align__(16) float sL2[2][128];
-    __shared__ __align__(16) float sD[2][128];
+    __shared__ __align__(16) float sLD[2][256];  // per slot: L2 of the 128 queries, then D
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int b = 0; b < 6; ++b) mbar_init(&bars[b], 1);
+        for (int b = 0; b < kBars; ++b) mbar_init(&bars[b], (b == 8 || b == 9) ? 256 : 1);
         abort_s = 0;
         fence_barrier_init();
     }
-    if (warp == 0) {
+    if (warp == kIssuerWarp) {
         tmem_alloc(&tmem_slot, kBwdTmemCols);
         tmem_relinquish();
-    }
-    if (threadIdx.x < 128) {
-        const size_t r = (size_t)bh * p.N_pad + (size_t)cur_qb * 128 + threadIdx.x;
-        sL2[0][threadIdx.x] = p.rowL2[r];
-        sD[0][threadIdx.x] = p.rowD[r];
     }
     tc_fence_before();
     __syncthreads();
@@ -515,139 +652,226 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t tmem = tmem_slot;
     // S^T then P^T, dP^T then dS^T, dV, dK
     const uint32_t tS = tmem, tP = tmem + 128, tV = tmem + 256, tK = tmem + 256 + D;
-    const BwdCta cta{bars, &abort_s, p.flag};
-    const int grp = warp & 3, half = warp >> 2;
-    const uint32_t lane_off = (uint32_t)(32 * grp) << 16;
-    const int key = 32 * grp + lane;  // key row of the block (TMEM lane)
-    const bool key_ok = kb * 128 + key < p.N;
-    auto sQ = [&](int s) { return smem + (2 + 2 * s) * kTileMax; };
-    auto sG = [&](int s) { return smem + (3 + 2 * s) * kTileMax; };
-    const uint64_t k_desc = smem_desc_sw128(smem_u32(sK), 16, 1024);
-    const uint64_t v_desc = smem_desc_sw128(smem_u32(sV), 16, 1024);
+    MarkWalk walk{p.mark + (size_t)item * p.nqb, p.nqb, 0, 0u, 0u, 0u};
+    walk.start();
+    volatile int *ab = &abort_s;
 
-    bool first_done = false;
-    int qg_issued = 0, qg_done = 0;
-    auto issue_qg = [&](int it, int qbl) {
-        const int s = it & 1;
-        mbar_arrive_expect_tx(&bars[1 + s], 2 * kTileBytes);
-        tma_tile<D>(sQ(s), &tmQ, &bars[1 + s], qbl, bh);
-        tma_tile<D>(sG(s), &tmG, &bars[1 + s], qbl, bh);
-        ++qg_issued;
-    };
-    bool ok0 = true;
-    if (threadIdx.x == 0) {
-        prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmK);
-        prefetch_tmap(&tmV);
-        prefetch_tmap(&tmG);
-        mbar_arrive_expect_tx(&bars[0], 2 * kTileBytes);
-        tma_tile<D>(sK, &tmK, &bars[0], kb, bh);
-        tma_tile<D>(sV, &tmV, &bars[0], kb, bh);
-        issue_qg(0, cur_qb);
-    }
-    bool failed = false;
-    int it = 0;
-    for (; have_cur; ++it) {
-        const int s = it & 1;
-        const float lw2 = kW ? lw2_of(p.w + ((size_t)bh * p.nqb + cur_qb) * p.nkb + cur_c, p.flag,
-                                      threadIdx.x == 0)
-                             : 0.f;
-        if (warp == 0) {
-            if (lane == 0) {
-                if (it == 0) ok0 = first_done = bwd_wait(cta, &bars[0], 0);
-                if (ok0) ok0 = bwd_wait(cta, &bars[1 + s], (it >> 1) & 1);
-                if (ok0) {
-                    ++qg_done;
-                    tc_fence_after();
-                    mma_rows<D>(tS, k_desc, smem_desc_sw128(smem_u32(sQ(s)), 16, 1024));
-                    mma_rows<D>(tP, v_desc, smem_desc_sw128(smem_u32(sG(s)), 16, 1024));
-                    mma_commit(&bars[3]);
-                }
-                // the other stage is free once dV, dK of pair it - 1 are done
-                if (ok0 && it >= 1) ok0 = bwd_wait(cta, &bars[4], (it - 1) & 1);
-                if (ok0 && have_nxt) issue_qg(it + 1, nxt_qb);
+    if (warp == kIssuerWarp) {
+        // ------------------------------ issuer warp ------------------------------
+        Inflight f;
+        auto next_qb = [&]() {
+            int q = 0, c = 0;
+            if (!walk.next(q, c) && lane == 0) raise_flag(p.flag, AB_FLAG_BAD_INDEX);
+            return q;
+        };
+        auto load_q = [&](int c, int q) {
+            const int slot = c & 1;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&bars[1 + slot], kTileBytes + 1024);
+                tma_tile<D>(sQ(slot), &tmQ, &bars[1 + slot], q, bh);
+                const size_t r = (size_t)bh * p.N_pad + (size_t)q * 128;
+                bulk_load(&sLD[slot][0], p.rowL2 + r, 512, &bars[1 + slot]);
+                bulk_load(&sLD[slot][128], p.rowD + r, 512, &bars[1 + slot]);
+            }
+            __syncwarp();
+            ++f.issued[1];
+        };
+        auto load_g = [&](int c, int q) {
+            const int slot = c & 1;
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&bars[4 + slot], kTileBytes);
+                tma_tile<D>(sG(slot), &tmG, &bars[4 + slot], q, bh);
+            }
+            __syncwarp();
+            ++f.issued[2];
+        };
+        auto qd = [&](int slot) { return smem_desc_sw128(smem_u32(sQ(slot)), 16, 1024); };
+        auto qd_mn = [&](int slot) { return smem_desc_sw128(smem_u32(sQ(slot)), 16384, 1024); };
+        auto gd = [&](int slot) { return smem_desc_sw128(smem_u32(sG(slot)), 16, 1024); };
+        auto gd_mn = [&](int slot) { return smem_desc_sw128(smem_u32(sG(slot)), 16384, 1024); };
+        const uint64_t k_desc = smem_desc_sw128(smem_u32(sK), 16, 1024);
+        const uint64_t v_desc = smem_desc_sw128(smem_u32(sV), 16, 1024);
+        if (elect_one()) {
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            prefetch_tmap(&tmG);
+            mbar_arrive_expect_tx(&bars[0], 2 * kTileBytes);
+            tma_tile<D>(sK, &tmK, &bars[0], kb, bh);
+            tma_tile<D>(sV, &tmV, &bars[0], kb, bh);
+        }
+        __syncwarp();
+        f.issued[0] = 1;
+        {
+            const int q0 = next_qb();
+            load_q(0, q0);
+            load_g(0, q0);
+        }
+        if (n > 1) {
+            const int q1 = next_qb();
+            load_q(1, q1);
+            load_g(1, q1);
+        }
+        bool ok = issuer_wait(&bars[0], 0, ab, p.flag);
+        if (ok) f.waited[0] = 1;
+        ok = ok && issuer_wait(&bars[1], 0, ab, p.flag);
+        if (ok) ++f.waited[1];
+        ok = ok && issuer_wait(&bars[4], 0, ab, p.flag);
+        if (ok) {
+            ++f.waited[2];
+            tc_fence_after();
+            if (elect_one()) {
+                mma_rows<D>(tS, k_desc, qd(0));
+                mma_commit(&bars[6]);
+                mma_rows<D>(tP, v_desc, gd(0));
+                mma_commit(&bars[7]);
             }
             __syncwarp();
         }
-        // the next pair's row statistics (stage s^1 was last read before the previous
-        // iteration's barrier)
-        if (have_nxt && threadIdx.x < 128) {
-            const size_t r = (size_t)bh * p.N_pad + (size_t)nxt_qb * 128 + threadIdx.x;
-            sL2[s ^ 1][threadIdx.x] = p.rowL2[r];
-            sD[s ^ 1][threadIdx.x] = p.rowD[r];
-        }
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[3], it & 1, &abort_s, p.flag));
-        if (ok) {
+        for (int c = 0; ok && c < n; ++c) {
+            const int s = c & 1, s1 = s ^ 1;
+            // P^T(c) stored and S^T(c) read: dV += P^T dO_c
+            if (!issuer_wait(&bars[8], c & 1, ab, p.flag)) { ok = false; break; }
             tc_fence_after();
-            // P^T and dS^T for this thread's key over the half's 64 queries
-            uint32_t pp[32], pd[32];
+            if (elect_one()) mma_packed<D>(tV, tS, gd_mn(s), c > 0);
+            __syncwarp();
+            // dS^T(c) stored and dP^T(c) read: dK += dS^T Q_c, then S^T(c + 1) and
+            // dP^T(c + 1) over the packed operands (the pipe runs them in order)
+            if (!issuer_wait(&bars[9], c & 1, ab, p.flag)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+                mma_packed<D>(tK, tP, qd_mn(s), c > 0);
+                mma_commit(&bars[10]);
+                if (c == n - 1) mma_commit(&bars[11]);
+            }
+            __syncwarp();
+            if (c + 1 < n) {
+                if (!issuer_wait(&bars[1 + s1], ((c + 1) >> 1) & 1, ab, p.flag)) { ok = false; break; }
+                ++f.waited[1];
+                tc_fence_after();
+                if (elect_one()) {
+                    mma_rows<D>(tS, k_desc, qd(s1));
+                    mma_commit(&bars[6]);
+                }
+                __syncwarp();
+                if (!issuer_wait(&bars[4 + s1], ((c + 1) >> 1) & 1, ab, p.flag)) { ok = false; break; }
+                ++f.waited[2];
+                tc_fence_after();
+                if (elect_one()) {
+                    mma_rows<D>(tP, v_desc, gd(s1));
+                    mma_commit(&bars[7]);
+                }
+                __syncwarp();
+            }
+            // pair c accumulated (dV(c), dK(c) and every earlier MMA done): its Q, rows and
+            // dO slots take pair c + 2
+            if (!issuer_wait(&bars[10], c & 1, ab, p.flag)) { ok = false; break; }
+            if (c + 2 < n) {
+                const int q2 = next_qb();
+                load_q(c + 2, q2);
+                load_g(c + 2, q2);
+            }
+        }
+        if (!ok) drain_issuer(bars, f, 2);
+    } else {
+        // ------------------------------ compute warps ------------------------------
+        const int grp = warp & 3, half = warp >> 2;
+        const uint32_t lane_off = (uint32_t)(32 * grp) << 16;
+        const int key = 32 * grp + lane;  // key row of the block (TMEM lane)
+        const bool key_ok = kb * 128 + key < p.N;
+        auto weight_ptr = [&](int q, int ce) { return p.w + ((size_t)bh * p.nqb + q) * p.nkb + ce; };
+        int q_cur = 0, ce_cur = 0;
+        walk.next(q_cur, ce_cur);
+        float lw_cur = kW ? lw2_val(__ldg(weight_ptr(q_cur, ce_cur)), p.flag, threadIdx.x == 0) : 0.f;
+        bool ok = true;
+        for (int c = 0; c < n; ++c) {
+            // the next pair's weight: loaded here, used only after this pair's work
+            float w_raw = 1.f;
+            if (c + 1 < n) {
+                int q_nx = 0, ce_nx = 0;
+                walk.next(q_nx, ce_nx);
+                if (kW) w_raw = __ldg(weight_ptr(q_nx, ce_nx));
+            }
+            const int slot = c & 1;
+            // the L2 and D rows arrive with Q_c
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[1 + slot], (c >> 1) & 1, ab, p.flag))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[6], c & 1, ab, p.flag))) { ok = false; break; }
+            tc_fence_after();
+            // P^T = 2^(s scale_log2 + log2 w - L2_i) for this key over the half's queries
+            float pv[64];
+            uint32_t pk[32];
+            const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+            uint32_t sv2[2][32];  // both 32-column halves of this warp's S^T columns, one wait
+            tmem_ld32(tS + lane_off + half * 64, sv2[0]);
+            tmem_ld32(tS + lane_off + half * 64 + 32, sv2[1]);
+            tmem_wait_ld();
 #pragma unroll
             for (int ch = 0; ch < 2; ++ch) {
-                uint32_t sv[32], dv[32];
-                tmem_ld32(tS + lane_off + half * 64 + ch * 32, sv);
-                tmem_ld32(tP + lane_off + half * 64 + ch * 32, dv);
-                tmem_wait_ld();
-                const float4 *l4 = reinterpret_cast<const float4 *>(&sL2[s][half * 64 + ch * 32]);
-                const float4 *d4 = reinterpret_cast<const float4 *>(&sD[s][half * 64 + ch * 32]);
+                const uint32_t (&sv)[32] = sv2[ch];
+                const float4 *l4 = reinterpret_cast<const float4 *>(&sLD[slot][half * 64 + ch * 32]);
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 lq = l4[e4], dq = d4[e4];
-                    const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
-                    const float dd[4] = {dq.x, dq.y, dq.z, dq.w};
-                    float pv[4], ds[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int e = e4 * 4 + u;
-                        pv[u] = key_ok ? fast_exp2(fmaf(__uint_as_float(sv[e]), p.scale_log2, lw2 - lv[u])) : 0.f;
-                        ds[u] = pv[u] * (__uint_as_float(dv[e]) - dd[u]);
-                    }
-                    pp[ch * 16 + e4 * 2] = pack_bf16x2(pv[0], pv[1]);
-                    pp[ch * 16 + e4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-                    pd[ch * 16 + e4 * 2] = pack_bf16x2(ds[0], ds[1]);
-                    pd[ch * 16 + e4 * 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                    const float4 lq = l4[e4];
+                    const int e = e4 * 4;
+                    const float2 r0 = exp2_pair(
+                        f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2,
+                               f2_pack(lw_cur - lq.x, lw_cur - lq.y)),
+                        (ch * 16 + e4 * 2) % 5 == 4);
+                    const float2 r1 = exp2_pair(
+                        f2_fma(f2_pack(__uint_as_float(sv[e + 2]), __uint_as_float(sv[e + 3])), sc2,
+                               f2_pack(lw_cur - lq.z, lw_cur - lq.w)),
+                        (ch * 16 + e4 * 2 + 1) % 5 == 4);
+                    pv[ch * 32 + e] = key_ok ? r0.x : 0.f;
+                    pv[ch * 32 + e + 1] = key_ok ? r0.y : 0.f;
+                    pv[ch * 32 + e + 2] = key_ok ? r1.x : 0.f;
+                    pv[ch * 32 + e + 3] = key_ok ? r1.y : 0.f;
+                    pk[ch * 16 + e4 * 2] = pack_bf16x2(pv[ch * 32 + e], pv[ch * 32 + e + 1]);
+                    pk[ch * 16 + e4 * 2 + 1] = pack_bf16x2(pv[ch * 32 + e + 2], pv[ch * 32 + e + 3]);
                 }
             }
-            tmem_st32(tS + lane_off + half * 64, pp);
-            tmem_st32(tP + lane_off + half * 64, pd);
+            tmem_st32(tS + lane_off + half * 64, pk);
             tmem_wait_st();
-        }
-        tc_fence_before();
-        if (__syncthreads_or(!ok || (threadIdx.x == 0 && !ok0))) {
-            failed = true;
-            break;
-        }
-        if (warp == 0) {
-            if (lane == 0) {
-                tc_fence_after();
-                mma_packed<D>(tV, tS, smem_desc_sw128(smem_u32(sG(s)), 16384, 1024), it > 0);
-                mma_packed<D>(tK, tP, smem_desc_sw128(smem_u32(sQ(s)), 16384, 1024), it > 0);
-                mma_commit(&bars[4]);
+            tc_fence_before();
+            mbar_arrive(&bars[8]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars[7], c & 1, ab, p.flag))) { ok = false; break; }
+            tc_fence_after();
+            // dS^T = P^T (dP^T - D_i)
+            uint32_t dv2[2][32];
+            tmem_ld32(tP + lane_off + half * 64, dv2[0]);
+            tmem_ld32(tP + lane_off + half * 64 + 32, dv2[1]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                const uint32_t (&dv)[32] = dv2[ch];
+                const float4 *d4 = reinterpret_cast<const float4 *>(&sLD[slot][128 + half * 64 + ch * 32]);
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 dq = d4[e4];
+                    const int e = ch * 32 + e4 * 4;
+                    pk[ch * 16 + e4 * 2] = pack_bf16x2(pv[e] * (__uint_as_float(dv[e4 * 4]) - dq.x),
+                                                       pv[e + 1] * (__uint_as_float(dv[e4 * 4 + 1]) - dq.y));
+                    pk[ch * 16 + e4 * 2 + 1] = pack_bf16x2(pv[e + 2] * (__uint_as_float(dv[e4 * 4 + 2]) - dq.z),
+                                                           pv[e + 3] * (__uint_as_float(dv[e4 * 4 + 3]) - dq.w));
+                }
             }
-            __syncwarp();
+            tmem_st32(tP + lane_off + half * 64, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[9]);
+            lw_cur = kW ? lw2_val(w_raw, p.flag, threadIdx.x == 0) : 0.f;
         }
-        cur_qb = nxt_qb;
-        cur_c = nxt_c;
-        have_cur = have_nxt;
-        if (have_cur) have_nxt = walk.next(nxt_qb, nxt_c);
-    }
-    bool ok_end = !failed;
-    if (ok_end) ok_end = __all_sync(0xffffffffu, mbar_wait(&bars[4], (it - 1) & 1, &abort_s, p.flag));
-    if (ok_end) {
-        tc_fence_after();
-        store_acc_row<D>(tV + lane_off + half * (D / 2), p.dv + (row0 + key) * D + half * (D / 2), 1.f,
-                         key_ok);
-        store_acc_row<D>(tK + lane_off + half * (D / 2), p.dk + (row0 + key) * D + half * (D / 2),
-                         p.scale, key_ok);
-    }
-    if (threadIdx.x == 0 && (failed || !ok_end)) {
-        mma_commit(&bars[5]);
-        drain_wait(&bars[5], 0);
-        if (!first_done) drain_wait(&bars[0], 0);
-        for (int k = qg_done; k < qg_issued; ++k) drain_wait(&bars[1 + (k & 1)], (k >> 1) & 1);
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[11], 0, ab, p.flag));
+        if (ok) {
+            tc_fence_after();
+            store_acc_row<D>(tV + lane_off + half * (D / 2), p.dv + (row0 + key) * D + half * (D / 2), 1.f,
+                             key_ok);
+            store_acc_row<D>(tK + lane_off + half * (D / 2), p.dk + (row0 + key) * D + half * (D / 2),
+                             p.scale, key_ok);
+        }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kIssuerWarp) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, kBwdTmemCols);
@@ -671,12 +895,14 @@ cudaError_t launch_bwd_t(const AttnBwdLaunch &a, cudaStream_t st)
     float *rowD = reinterpret_cast<float *>(ws + L.rowD);
     float *rowL2 = reinterpret_cast<float *>(ws + L.rowL2);
     uint16_t *mark = reinterpret_cast<uint16_t *>(ws + L.mark);
+    uint32_t *kcount = reinterpret_cast<uint32_t *>(ws + L.kcount);
     CUtensorMap tq, tk, tv, tg;
     if (!bwd_tmap(&tq, a.q, BH, a.N, a.N_pad, D) || !bwd_tmap(&tk, a.k, BH, a.N, a.N_pad, D) ||
         !bwd_tmap(&tv, a.v, BH, a.N, a.N_pad, D) || !bwd_tmap(&tg, a.dout, BH, a.N, a.N_pad, D))
         return cudaErrorInvalidValue;
     const size_t rows = (size_t)BH * a.N_pad;
-    cudaError_t e = cudaMemsetAsync(mark, 0, (size_t)BH * nb * nb * sizeof(uint16_t), st);
+    // the mark table and the per-key-block counts, one contiguous region
+    cudaError_t e = cudaMemsetAsync(mark, 0, L.total - L.mark, st);
     if (e != cudaSuccess) return e;
     const unsigned rs_grid = (unsigned)((rows + 15) / 16);
     if (a.out_f32)
@@ -687,8 +913,8 @@ cudaError_t launch_bwd_t(const AttnBwdLaunch &a, cudaStream_t st)
             a.out, static_cast<const __nv_bfloat16 *>(a.dout), a.lse, rowD, rowL2, rows, a.N, a.N_pad);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t plan_rows = (size_t)BH * nb;
-    attn_bwd_mark_kernel<<<(unsigned)((plan_rows + 7) / 8), 256, 0, st>>>(a.idx, a.cnt, mark, plan_rows,
-                                                                           nb, nb, a.flag);
+    attn_bwd_mark_kernel<<<(unsigned)((plan_rows + 7) / 8), 256, 0, st>>>(a.idx, a.cnt, mark, kcount,
+                                                                           plan_rows, nb, nb, a.flag);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     BwdParams p;
     p.idx = a.idx;
@@ -697,6 +923,7 @@ cudaError_t launch_bwd_t(const AttnBwdLaunch &a, cudaStream_t st)
     p.rowD = rowD;
     p.rowL2 = rowL2;
     p.mark = mark;
+    p.kcount = kcount;
     p.dq = a.dq;
     p.dk = a.dk;
     p.dv = a.dv;
@@ -707,13 +934,13 @@ cudaError_t launch_bwd_t(const AttnBwdLaunch &a, cudaStream_t st)
     p.nkb = nb;
     p.scale = (float)(1.0 / std::sqrt((double)D));
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-    e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem);
+    e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem);
+    e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDkdvSmem);
     if (e != cudaSuccess) return e;
-    attn_bwd_dq_kernel<D, kW><<<(unsigned)plan_rows, kBwdThreads, kBwdSmem, st>>>(tq, tk, tv, tg, p);
+    attn_bwd_dq_kernel<D, kW><<<(unsigned)plan_rows, kBwdThreads, kDqSmem, st>>>(tq, tk, tv, tg, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    attn_bwd_dkdv_kernel<D, kW><<<(unsigned)plan_rows, kBwdThreads, kBwdSmem, st>>>(tq, tk, tv, tg, p);
+    attn_bwd_dkdv_kernel<D, kW><<<(unsigned)plan_rows, kBwdThreads, kDkdvSmem, st>>>(tq, tk, tv, tg, p);
     return cudaGetLastError();
 }
 

@@ -295,8 +295,9 @@ ab_status ab_attn_topk_fwd(const void *q, const void *k, const void *v, ab_shape
 
 /*
  * ab_attn_bwd_workspace_size -- bytes of device scratch ab_attn_bwd() needs for shape s:
- * two fp32 values per query row and a uint16 table of n_qb x n_kb entries per head,
- * each region 256-byte aligned. Errors: AB_ERR_NULL and the shape errors of ab_attn_fwd.
+ * two fp32 values per query row, a uint16 table of n_qb x n_kb entries per head and a
+ * uint32 count per key block, each region 256-byte aligned. Errors: AB_ERR_NULL and the
+ * shape errors of ab_attn_fwd.
  */
 ab_status ab_attn_bwd_workspace_size(ab_shape s, size_t *bytes);
 
@@ -318,8 +319,8 @@ ab_status ab_attn_bwd_workspace_size(ab_shape s, size_t *bytes);
  *             empty selection (dq) and the rows of a key block no query block kept
  *             (dk, dv) are 0.
  * workspace : device scratch of ab_attn_bwd_workspace_size() bytes, owned by the
- *             caller, contents need not be initialised; the call clears its table with
- *             one memset on `stream`.
+ *             caller, contents need not be initialised; the call clears its table and
+ *             counts with one memset on `stream`.
  * Every sum runs in a fixed order: the result is the same on every run.
  * Device-side: an idx/cnt outside range or a block twice in one row sets
  * AB_FLAG_BAD_INDEX, a bad weight AB_FLAG_BAD_WEIGHT, a bounded wait that gave up

@@ -215,9 +215,10 @@ def test_attn_bwd_argument_checks(L):
     s = ab.Shape(1, 2, 1000, 1024, 128, ab.AB_BF16)
     n = ctypes.c_size_t(0)
     assert L.ab_attn_bwd_workspace_size(s, ctypes.byref(n)) == 0
-    # D_i and lse_i log2e per query row (fp32) and the n_kb x n_qb uint16 mark table per head
-    need = 2 * 2 * 1024 * 4 + 2 * 8 * 8 * 2
-    assert need <= n.value <= need + 3 * 256
+    # D_i and lse_i log2e per query row (fp32), the n_kb x n_qb uint16 mark table and a
+    # uint32 count per key block, per head
+    need = 2 * 2 * 1024 * 4 + 2 * 8 * 8 * 2 + 2 * 8 * 4
+    assert need <= n.value <= need + 4 * 256
     assert L.ab_attn_bwd_workspace_size(s, None) == 1
     assert L.ab_attn_bwd_workspace_size(ab.Shape(1, 2, 1000, 1024, 96, ab.AB_BF16), ctypes.byref(n)) == 4
     assert n.value == 0
