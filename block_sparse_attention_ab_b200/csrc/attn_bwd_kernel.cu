@@ -567,13 +567,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // 4. dK, dV: one CTA per (b, h, key block), over the kcount[bh][kb] query blocks that
 //    kept it, ascending, read from the mark column. Pipeline per pair c (Q_c with its
 //    rows' L2 and D, and dO_c, in slot c mod 2 of their rings):
-//      issuer: S^T(0), dP^T(0); then for each c: [P^T(c) stored] dV += P^T dO_c;
-//              [dS^T(c) stored] dK += dS^T Q_c, S^T(c+1), dP^T(c+1); [pair c done]
+//      issuer: S^T(0), dP^T(0); then for each c: [P^T(c) stored] dV += P^T dO_c,
+//              S^T(c+1); [dS^T(c) stored] dK += dS^T Q_c, dP^T(c+1); [pair c done]
 //              loads for c + 2 into its slots;
 //      compute: [S^T(c)] P^T packed over S^T, arrive; [dP^T(c)] dS^T packed over dP^T,
 //               arrive.
-//    dV(c) runs while the warps form dS^T(c); dK(c), S^T(c+1) and dP^T(c+1) while they
-//    wait for S^T(c+1) and then form P^T(c+1).
+//    dV(c) and S^T(c+1) run while the warps form dS^T(c); dK(c) and dP^T(c+1) while they
+//    form P^T(c+1).
 // ---------------------------------------------------------------------------------
 // Every warp walks the mark column in chunks of 32 (one ballot per chunk, the next
 // chunk's entries already loaded), so all warps see the same sequence without talking
@@ -730,20 +730,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         for (int c = 0; ok && c < n; ++c) {
             const int s = c & 1, s1 = s ^ 1;
-            // P^T(c) stored and S^T(c) read: dV += P^T dO_c
+            // P^T(c) stored and S^T(c) read: dV += P^T dO_c, then S^T(c + 1) over it (the
+            // pipe runs them in order; Q_{c+1} is the other slot of the ring)
             if (!issuer_wait(&bars[8], c & 1, ab, p.flag)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) mma_packed<D>(tV, tS, gd_mn(s), c > 0);
-            __syncwarp();
-            // dS^T(c) stored and dP^T(c) read: dK += dS^T Q_c, then S^T(c + 1) and
-            // dP^T(c + 1) over the packed operands (the pipe runs them in order)
-            if (!issuer_wait(&bars[9], c & 1, ab, p.flag)) { ok = false; break; }
-            tc_fence_after();
-            if (elect_one()) {
-                mma_packed<D>(tK, tP, qd_mn(s), c > 0);
-                mma_commit(&bars[10]);
-                if (c == n - 1) mma_commit(&bars[11]);
-            }
             __syncwarp();
             if (c + 1 < n) {
                 if (!issuer_wait(&bars[1 + s1], ((c + 1) >> 1) & 1, ab, p.flag)) { ok = false; break; }
@@ -754,6 +745,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     mma_commit(&bars[6]);
                 }
                 __syncwarp();
+            }
+            // dS^T(c) stored and dP^T(c) read: dK += dS^T Q_c, then dP^T(c + 1) over it
+            if (!issuer_wait(&bars[9], c & 1, ab, p.flag)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+                mma_packed<D>(tK, tP, qd_mn(s), c > 0);
+                mma_commit(&bars[10]);
+                if (c == n - 1) mma_commit(&bars[11]);
+            }
+            __syncwarp();
+            if (c + 1 < n) {
                 if (!issuer_wait(&bars[4 + s1], ((c + 1) >> 1) & 1, ab, p.flag)) { ok = false; break; }
                 ++f.waited[2];
                 tc_fence_after();
