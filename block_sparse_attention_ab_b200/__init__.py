@@ -79,6 +79,8 @@ def lib():
         L.ab_attn_bwd_workspace_size.argtypes = [S, ctypes.POINTER(ctypes.c_size_t)]
         L.ab_attn_bwd.argtypes = [P, P, P, S, P, P, P, P, I, P, P, P, P, P, P, ctypes.c_size_t,
                                   P, P]
+        L.ab_selftest_attn_bwd_wait_limit.argtypes = [P, P, P, S, P, P, P, P, I, P, P, P, P, P, P,
+                                                      ctypes.c_size_t, P, I, P]
         L.ab_score_units_workspace_size.argtypes = [S, I, I, ctypes.POINTER(ctypes.c_size_t)]
         L.ab_score_units.argtypes = [P, P, S, I, I, I, P, P, P, P, P, P, ctypes.c_size_t, P, P]
         L.ab_attn_units_fwd.argtypes = [P, P, P, S, I, P, P, P, P, I, P, P, P]
@@ -99,7 +101,8 @@ def lib():
                      "ab_attn_topk_fwd", "ab_check_flag", "ab_version", "ab_score_units_workspace_size",
                      "ab_score_units", "ab_attn_units_fwd", "ab_attn_units_topk_fwd",
                      "ab_selftest_bounded_wait", "ab_selftest_force_counter_slot",
-                     "ab_selftest_attn_wait_limit"):
+                     "ab_selftest_attn_wait_limit", "ab_attn_bwd_workspace_size", "ab_attn_bwd",
+                     "ab_selftest_attn_bwd_wait_limit"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -275,10 +278,12 @@ def attn_bwd_workspace_bytes(shape: Shape) -> int:
 
 
 def attn_bwd(q, k, v, N: int, idx, cnt, w, out, lse, dout,
-             dev_flag: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None):
+             dev_flag: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+             wait_limit_ns: Optional[int] = None):
     """Gradients (dq, dk, dv), fp32 [B,H,N_pad,d], of attn_fwd (w given) or attn_topk_fwd
     (w None) over key blocks, for the upstream gradient `dout` (bf16) of the output
-    `out` (bf16 or fp32) whose lse the forward returned."""
+    `out` (bf16 or fp32) whose lse the forward returned. wait_limit_ns (tests only) runs
+    ab_selftest_attn_bwd_wait_limit instead, with the kernels' waits limited to it."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
         _need(t, torch.bfloat16, n)
     _need(idx, torch.int32, "idx")
@@ -292,10 +297,14 @@ def attn_bwd(q, k, v, N: int, idx, cnt, w, out, lse, dout,
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     dq, dk, dv = (torch.empty(q.shape, device=q.device, dtype=torch.float32) for _ in range(3))
-    _check(lib().ab_attn_bwd(_ptr(q), _ptr(k), _ptr(v), shape, _ptr(idx), _ptr(cnt), _ptr(w),
-                             _ptr(out), _out_code(out.dtype), _ptr(lse), _ptr(dout), _ptr(dq),
-                             _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(),
-                             _ptr(dev_flag), _stream()), "ab_attn_bwd")
+    args = (_ptr(q), _ptr(k), _ptr(v), shape, _ptr(idx), _ptr(cnt), _ptr(w), _ptr(out),
+            _out_code(out.dtype), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+            _ptr(workspace), workspace.numel(), _ptr(dev_flag))
+    if wait_limit_ns is None:
+        _check(lib().ab_attn_bwd(*args, _stream()), "ab_attn_bwd")
+    else:
+        _check(lib().ab_selftest_attn_bwd_wait_limit(*args, int(wait_limit_ns), _stream()),
+               "ab_selftest_attn_bwd_wait_limit")
     return dq, dk, dv
 
 

@@ -81,6 +81,7 @@ struct AttnBwdLaunch {
     void *workspace;  // attn_bwd_layout(...).total bytes
     int *flag;
     int B, H, N, N_pad, d;
+    unsigned long long wait_ns;  // > 0: limit of the kernels' bounded waits (tests); 0: 2 s
 };
 
 constexpr int kBwdThreads = 288;  // 8 compute warps + 1 issuer warp
@@ -101,6 +102,7 @@ struct BwdParams {
     int *flag;
     int N, N_pad, nqb, nkb;
     float scale, scale_log2;
+    uint64_t wait_ns;  // limit of every bounded wait
 };
 
 // S (+)= A B^T over the head dimension: A, B are [128 rows][D] tiles, K-major, two
@@ -290,10 +292,39 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint3
                  : "memory");
 }
 
-// The issuer warp's bounded wait (all lanes agree).
-__device__ __forceinline__ bool issuer_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *flag)
+// The kernels' bounded wait. With the normal limit it is mbar_wait; with a limit below
+// 1 ms (the wait-limit test entry) it polls with the non-blocking test_wait and reads the
+// clock at every poll (try_wait may hold the thread until the phase completes), so that
+// even a wait of a few microseconds can run past the limit.
+__device__ __forceinline__ bool bwd_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *flag,
+                                         uint64_t limit_ns)
 {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, flag));
+    if (limit_ns >= 1000000ull) return mbar_wait(bar, parity, abort, flag, limit_ns);
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+            *abort = 1;
+            raise_flag(flag, AB_FLAG_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// The issuer warp's bounded wait (all lanes agree).
+__device__ __forceinline__ bool issuer_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *flag,
+                                            uint64_t limit_ns)
+{
+    return __all_sync(0xffffffffu, bwd_wait(bar, parity, abort, flag, limit_ns));
 }
 
 // Copies of the issuer still in flight after a failed wait: let them land before the CTA
@@ -423,11 +454,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // the block index of the next pair to load, read one iteration ahead of its use
         int j_pre = n > 2 ? __ldg(idx + 2) : 0;
-        bool ok = issuer_wait(&bars[0], 0, ab, p.flag);
+        bool ok = issuer_wait(&bars[0], 0, ab, p.flag, p.wait_ns);
         if (ok) f.waited[0] = 1;
-        ok = ok && issuer_wait(&bars[1], 0, ab, p.flag);
+        ok = ok && issuer_wait(&bars[1], 0, ab, p.flag, p.wait_ns);
         if (ok) ++f.waited[1];
-        ok = ok && issuer_wait(&bars[4], 0, ab, p.flag);
+        ok = ok && issuer_wait(&bars[4], 0, ab, p.flag, p.wait_ns);
         if (ok) {
             ++f.waited[2];
             tc_fence_after();
@@ -441,10 +472,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         for (int c = 0; ok && c < n; ++c) {
             // S(c) has been read: S(c + 1) may overwrite it
-            if (!issuer_wait(&bars[8], c & 1, ab, p.flag)) { ok = false; break; }
+            if (!issuer_wait(&bars[8], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             if (c + 1 < n) {
                 const int ks = (c + 1) % 3;
-                if (!issuer_wait(&bars[1 + ks], ((c + 1) / 3) & 1, ab, p.flag)) { ok = false; break; }
+                if (!issuer_wait(&bars[1 + ks], ((c + 1) / 3) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
                 ++f.waited[1];
                 tc_fence_after();
                 if (elect_one()) {
@@ -454,7 +485,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 __syncwarp();
             }
             // dS(c) stored and dP(c) read: dQ += dS(c) K_c, then dP(c + 1) over it
-            if (!issuer_wait(&bars[9], c & 1, ab, p.flag)) { ok = false; break; }
+            if (!issuer_wait(&bars[9], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) {
                 mma_packed<D>(tAcc, tP, kd_mn(c % 3), c > 0);
@@ -463,7 +494,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             __syncwarp();
             if (c + 1 < n) {
                 const int vs = (c + 1) & 1;
-                if (!issuer_wait(&bars[4 + vs], ((c + 1) >> 1) & 1, ab, p.flag)) { ok = false; break; }
+                if (!issuer_wait(&bars[4 + vs], ((c + 1) >> 1) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
                 ++f.waited[2];
                 tc_fence_after();
                 if (elect_one()) {
@@ -482,7 +513,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 load_v(c + 2, j2);
             }
         }
-        if (!ok) drain_issuer(bars, f, 3);
+        // the CTA frees its tensor memory only after every MMA is done: on a failed wait the
+        // drain, else the final commit (also when only the compute warps gave up)
+        if (!ok)
+            drain_issuer(bars, f, 3);
+        else
+            drain_wait(&bars[11], 0);
     } else {
         // ------------------------------ compute warps ------------------------------
         const int grp = warp & 3, half = warp >> 2;
@@ -502,7 +538,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 j_raw = __ldg(idx + c + 1);
                 if (kW) w_raw = __ldg(wrow + c + 1);
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[6], c & 1, ab, p.flag))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait(&bars[6], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
             tc_fence_after();
             // P = 2^(s scale_log2 + log2 w - L2) on the valid keys of block j
             const int nvalid = p.N - j_cur * 128;
@@ -526,7 +562,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             tc_fence_before();
             mbar_arrive(&bars[8]);
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[7], c & 1, ab, p.flag))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait(&bars[7], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
             tc_fence_after();
             // dS = P (dP - D), packed to bf16 over the first 32 of this half's dP columns
             uint32_t pk[32];
@@ -547,7 +583,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             j_cur = clamp_j(j_raw);
             lw_cur = kW ? lw2_val(w_raw, p.flag, threadIdx.x == 0) : 0.f;
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[11], 0, ab, p.flag));
+        if (ok) ok = __all_sync(0xffffffffu, bwd_wait(&bars[11], 0, ab, p.flag, p.wait_ns));
         if (ok) {
             tc_fence_after();
             store_acc_row<D>(tAcc + lane_off + half * (D / 2), p.dq + (row0 + row) * D + half * (D / 2),
@@ -712,11 +748,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             load_q(1, q1);
             load_g(1, q1);
         }
-        bool ok = issuer_wait(&bars[0], 0, ab, p.flag);
+        bool ok = issuer_wait(&bars[0], 0, ab, p.flag, p.wait_ns);
         if (ok) f.waited[0] = 1;
-        ok = ok && issuer_wait(&bars[1], 0, ab, p.flag);
+        ok = ok && issuer_wait(&bars[1], 0, ab, p.flag, p.wait_ns);
         if (ok) ++f.waited[1];
-        ok = ok && issuer_wait(&bars[4], 0, ab, p.flag);
+        ok = ok && issuer_wait(&bars[4], 0, ab, p.flag, p.wait_ns);
         if (ok) {
             ++f.waited[2];
             tc_fence_after();
@@ -732,12 +768,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int s = c & 1, s1 = s ^ 1;
             // P^T(c) stored and S^T(c) read: dV += P^T dO_c, then S^T(c + 1) over it (the
             // pipe runs them in order; Q_{c+1} is the other slot of the ring)
-            if (!issuer_wait(&bars[8], c & 1, ab, p.flag)) { ok = false; break; }
+            if (!issuer_wait(&bars[8], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) mma_packed<D>(tV, tS, gd_mn(s), c > 0);
             __syncwarp();
             if (c + 1 < n) {
-                if (!issuer_wait(&bars[1 + s1], ((c + 1) >> 1) & 1, ab, p.flag)) { ok = false; break; }
+                if (!issuer_wait(&bars[1 + s1], ((c + 1) >> 1) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
                 ++f.waited[1];
                 tc_fence_after();
                 if (elect_one()) {
@@ -747,7 +783,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 __syncwarp();
             }
             // dS^T(c) stored and dP^T(c) read: dK += dS^T Q_c, then dP^T(c + 1) over it
-            if (!issuer_wait(&bars[9], c & 1, ab, p.flag)) { ok = false; break; }
+            if (!issuer_wait(&bars[9], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) {
                 mma_packed<D>(tK, tP, qd_mn(s), c > 0);
@@ -756,7 +792,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             __syncwarp();
             if (c + 1 < n) {
-                if (!issuer_wait(&bars[4 + s1], ((c + 1) >> 1) & 1, ab, p.flag)) { ok = false; break; }
+                if (!issuer_wait(&bars[4 + s1], ((c + 1) >> 1) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
                 ++f.waited[2];
                 tc_fence_after();
                 if (elect_one()) {
@@ -767,14 +803,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             // pair c accumulated (dV(c), dK(c) and every earlier MMA done): its Q, rows and
             // dO slots take pair c + 2
-            if (!issuer_wait(&bars[10], c & 1, ab, p.flag)) { ok = false; break; }
+            if (!issuer_wait(&bars[10], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             if (c + 2 < n) {
                 const int q2 = next_qb();
                 load_q(c + 2, q2);
                 load_g(c + 2, q2);
             }
         }
-        if (!ok) drain_issuer(bars, f, 2);
+        if (!ok)
+            drain_issuer(bars, f, 2);
+        else
+            drain_wait(&bars[11], 0);
     } else {
         // ------------------------------ compute warps ------------------------------
         const int grp = warp & 3, half = warp >> 2;
@@ -796,8 +835,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             const int slot = c & 1;
             // the L2 and D rows arrive with Q_c
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[1 + slot], (c >> 1) & 1, ab, p.flag))) { ok = false; break; }
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[6], c & 1, ab, p.flag))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait(&bars[1 + slot], (c >> 1) & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait(&bars[6], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
             tc_fence_after();
             // P^T = 2^(s scale_log2 + log2 w - L2_i) for this key over the half's queries
             float pv[64];
@@ -835,7 +874,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[8]);
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars[7], c & 1, ab, p.flag))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait(&bars[7], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
             tc_fence_after();
             // dS^T = P^T (dP^T - D_i)
             uint32_t dv2[2][32];
@@ -862,7 +901,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_arrive(&bars[9]);
             lw_cur = kW ? lw2_val(w_raw, p.flag, threadIdx.x == 0) : 0.f;
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[11], 0, ab, p.flag));
+        if (ok) ok = __all_sync(0xffffffffu, bwd_wait(&bars[11], 0, ab, p.flag, p.wait_ns));
         if (ok) {
             tc_fence_after();
             store_acc_row<D>(tV + lane_off + half * (D / 2), p.dv + (row0 + key) * D + half * (D / 2), 1.f,
@@ -936,6 +975,7 @@ cudaError_t launch_bwd_t(const AttnBwdLaunch &a, cudaStream_t st)
     p.nkb = nb;
     p.scale = (float)(1.0 / std::sqrt((double)D));
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+    p.wait_ns = a.wait_ns > 0 ? a.wait_ns : kWaitLimitNs;
     e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDkdvSmem);
@@ -968,6 +1008,50 @@ ab_status bwd_check_shape(const ab_shape &s)
 
 bool bwd_aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Argument checks and launch shared by ab_attn_bwd and its wait-limit test entry.
+ab_status attn_bwd_common(const void *q, const void *k, const void *v, ab_shape s, const int32_t *idx,
+                          const int32_t *cnt, const float *w, const void *out, ab_dtype out_dtype,
+                          const float *lse, const void *dout, float *dq, float *dk, float *dv,
+                          void *workspace, size_t workspace_bytes, int *dev_flag, void *stream,
+                          unsigned long long wait_ns)
+{
+    if (!q || !k || !v || !idx || !cnt || !out || !lse || !dout || !dq || !dk || !dv)
+        return AB_ERR_NULL;
+    const ab_status st = bwd_check_shape(s);
+    if (st != AB_OK) return st;
+    if (out_dtype != AB_BF16 && out_dtype != AB_F32) return AB_ERR_DTYPE;
+    if (!bwd_aligned16(q) || !bwd_aligned16(k) || !bwd_aligned16(v) || !bwd_aligned16(idx) ||
+        !bwd_aligned16(cnt) || (w && !bwd_aligned16(w)) || !bwd_aligned16(out) ||
+        !bwd_aligned16(lse) || !bwd_aligned16(dout) || !bwd_aligned16(dq) || !bwd_aligned16(dk) ||
+        !bwd_aligned16(dv) || (workspace && !bwd_aligned16(workspace)))
+        return AB_ERR_ALIGN;
+    const AttnBwdLayout L = attn_bwd_layout((size_t)s.B * s.H, (size_t)s.N_pad);
+    if (!workspace || workspace_bytes < L.total) return AB_ERR_WORKSPACE;
+    AttnBwdLaunch a;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.out = out;
+    a.out_f32 = out_dtype == AB_F32;
+    a.dout = dout;
+    a.lse = lse;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.w = w;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.workspace = workspace;
+    a.flag = dev_flag;
+    a.B = s.B;
+    a.H = s.H;
+    a.N = s.N;
+    a.N_pad = s.N_pad;
+    a.d = s.d;
+    a.wait_ns = wait_ns;
+    return status_of(launch_attn_bwd(a, (cudaStream_t)stream));
+}
+
 }  // namespace
 
 }  // namespace ab
@@ -993,41 +1077,25 @@ ab_status ab_attn_bwd(const void *q, const void *k, const void *v, ab_shape s, c
     struct Pop {
         ~Pop() { nvtxRangePop(); }
     } pop;
-    using ab::bwd_aligned16;
-    if (!q || !k || !v || !idx || !cnt || !out || !lse || !dout || !dq || !dk || !dv)
-        return AB_ERR_NULL;
-    const ab_status st = ab::bwd_check_shape(s);
-    if (st != AB_OK) return st;
-    if (out_dtype != AB_BF16 && out_dtype != AB_F32) return AB_ERR_DTYPE;
-    if (!bwd_aligned16(q) || !bwd_aligned16(k) || !bwd_aligned16(v) || !bwd_aligned16(idx) ||
-        !bwd_aligned16(cnt) || (w && !bwd_aligned16(w)) || !bwd_aligned16(out) ||
-        !bwd_aligned16(lse) || !bwd_aligned16(dout) || !bwd_aligned16(dq) || !bwd_aligned16(dk) ||
-        !bwd_aligned16(dv) || (workspace && !bwd_aligned16(workspace)))
-        return AB_ERR_ALIGN;
-    const ab::AttnBwdLayout L = ab::attn_bwd_layout((size_t)s.B * s.H, (size_t)s.N_pad);
-    if (!workspace || workspace_bytes < L.total) return AB_ERR_WORKSPACE;
-    ab::AttnBwdLaunch a;
-    a.q = q;
-    a.k = k;
-    a.v = v;
-    a.out = out;
-    a.out_f32 = out_dtype == AB_F32;
-    a.dout = dout;
-    a.lse = lse;
-    a.idx = idx;
-    a.cnt = cnt;
-    a.w = w;
-    a.dq = dq;
-    a.dk = dk;
-    a.dv = dv;
-    a.workspace = workspace;
-    a.flag = dev_flag;
-    a.B = s.B;
-    a.H = s.H;
-    a.N = s.N;
-    a.N_pad = s.N_pad;
-    a.d = s.d;
-    return ab::status_of(ab::launch_attn_bwd(a, (cudaStream_t)stream));
+    return ab::attn_bwd_common(q, k, v, s, idx, cnt, w, out, out_dtype, lse, dout, dq, dk, dv, workspace,
+                               workspace_bytes, dev_flag, stream, 0);
+}
+
+ab_status ab_selftest_attn_bwd_wait_limit(const void *q, const void *k, const void *v, ab_shape s,
+                                          const int32_t *idx, const int32_t *cnt, const float *w,
+                                          const void *out, ab_dtype out_dtype, const float *lse,
+                                          const void *dout, float *dq, float *dk, float *dv,
+                                          void *workspace, size_t workspace_bytes, int *dev_flag,
+                                          int limit_ns, void *stream)
+{
+    nvtxRangePushA("ab_selftest_attn_bwd_wait_limit");
+    struct Pop {
+        ~Pop() { nvtxRangePop(); }
+    } pop;
+    if (!dev_flag) return AB_ERR_NULL;
+    if (limit_ns < 1 || limit_ns > 1000000000) return AB_ERR_RANGE;
+    return ab::attn_bwd_common(q, k, v, s, idx, cnt, w, out, out_dtype, lse, dout, dq, dk, dv, workspace,
+                               workspace_bytes, dev_flag, stream, (unsigned long long)limit_ns);
 }
 
 }  // extern "C"

@@ -334,6 +334,24 @@ ab_status ab_attn_bwd(const void *q, const void *k, const void *v, ab_shape s, c
                       void *workspace, size_t workspace_bytes, int *dev_flag, void *stream);
 
 /*
+ * ab_selftest_attn_bwd_wait_limit -- test entry point with no counterpart on the method's
+ * pages: ab_attn_bwd with every bounded wait inside its two tensor-core kernels limited to
+ * limit_ns nanoseconds (1..1e9) instead of 2 s, so that a test can make their own waits
+ * give up (below 1 ms the waits poll without blocking and read the clock at every
+ * poll). A wait that gives up ORs AB_FLAG_TIMEOUT into *dev_flag (required here); the
+ * issuer warp lets its copies and MMAs in flight land, the compute warps leave their
+ * loops, and the CTA frees its tensor memory and returns, leaving the context usable.
+ * The gradients of such a call are undefined. Arguments and errors otherwise as
+ * ab_attn_bwd.
+ */
+ab_status ab_selftest_attn_bwd_wait_limit(const void *q, const void *k, const void *v, ab_shape s,
+                                          const int32_t *idx, const int32_t *cnt, const float *w,
+                                          const void *out, ab_dtype out_dtype, const float *lse,
+                                          const void *dout, float *dq, float *dk, float *dv,
+                                          void *workspace, size_t workspace_bytes, int *dev_flag,
+                                          int limit_ns, void *stream);
+
+/*
  * ab_attn_units_fwd, ab_attn_units_topk_fwd -- the attention of ab_attn_fwd /
  * ab_attn_topk_fwd over selected key units of key_unit tokens (AB_BLOCK, or AB_UNIT4:
  * the page's 4-token units, third technique). idx / cnt / w come from ab_select run on

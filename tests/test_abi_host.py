@@ -248,3 +248,12 @@ def test_attn_bwd_argument_checks(L):
     assert with_(ws=None) == 10
     assert with_(wsb=need - 1) == 10
     assert "ab_attn_bwd" in declared_functions()
+    # the wait-limit test entry: a device flag and a limit in 1..1e9 ns are required
+    sw = L.ab_selftest_attn_bwd_wait_limit
+    base = args[:16]
+    assert sw(*base, None, 1000, None) == 1
+    assert sw(*base, FAKE, 0, None) == 5
+    assert sw(*base, FAKE, 1_000_000_001, None) == 5
+    bad = list(base)
+    bad[0] = None
+    assert sw(*bad, FAKE, 1000, None) == 1

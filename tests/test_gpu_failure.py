@@ -128,3 +128,50 @@ def test_attention_wait_limit_argument_checks():
     p = ab._ptr(z)
     assert L.ab_selftest_attn_wait_limit(p, p, p, s, 128, p, p, p, p, ab.AB_F32, None, None, 1000, None) == 1
     assert L.ab_selftest_attn_wait_limit(p, p, p, s, 128, p, p, p, p, ab.AB_F32, None, p, 0, None) == 5
+
+
+def test_backward_wait_limit_runs_out(orc):
+    # the attention backward's own waits (TMA tiles, MMAs, the compute warps' handovers)
+    # given 1 ns: a wait not satisfied at its first poll gives up at the next tick of the
+    # GPU's global timer; the flag reports it, every CTA lets its copies and MMAs land,
+    # frees its tensor memory and returns, and the next call on the same context gives
+    # the result it gave before, which matches the oracle's gradient
+    g = torch.Generator().manual_seed(5)
+    N, H, d = 2000, 4, 128
+    N_pad = (N + 127) // 128 * 128
+    nb = N_pad // 128
+    q, k, v, do = (torch.zeros(1, H, N_pad, d, dtype=torch.bfloat16) for _ in range(4))
+    for t in (q, k, v, do):
+        t[:, :, :N] = torch.randn(1, H, N, d, generator=g).to(torch.bfloat16)
+    rng = np.random.default_rng(3)
+    idx = np.full((1, H, nb, nb), -1, dtype=np.int32)
+    cnt = np.zeros((1, H, nb), dtype=np.int32)
+    w = np.zeros((1, H, nb, nb), dtype=np.float32)
+    for h in range(H):
+        for qb in range(nb):
+            c = int(rng.integers(3, 9))
+            idx[0, h, qb, :c] = np.sort(rng.choice(nb, c, replace=False))
+            cnt[0, h, qb] = c
+            w[0, h, qb, :c] = rng.uniform(1.0, 3.0, c)
+    qc, kc, vc, gc = (t.cuda() for t in (q, k, v, do))
+    ic, cc, wc = (torch.from_numpy(a).cuda() for a in (idx, cnt, w))
+    out, lse = ab.attn_fwd(qc, kc, vc, N, ic, cc, wc, want_lse=True)
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    good = ab.attn_bwd(qc, kc, vc, N, ic, cc, wc, out, lse, gc, dev_flag=flag,
+                       wait_limit_ns=1_000_000_000)
+    assert ab.check_flag(flag) == 0
+    t0 = time.perf_counter()
+    flag.zero_()
+    ab.attn_bwd(qc, kc, vc, N, ic, cc, wc, out, lse, gc, dev_flag=flag, wait_limit_ns=1)
+    bits = ab.check_flag(flag)
+    assert time.perf_counter() - t0 < 10.0
+    assert bits & ab.FLAG_TIMEOUT and not bits & ~ab.FLAG_TIMEOUT
+    flag.zero_()
+    again = ab.attn_bwd(qc, kc, vc, N, ic, cc, wc, out, lse, gc, dev_flag=flag)
+    assert ab.check_flag(flag) == 0
+    for a, b in zip(again, good):
+        assert torch.equal(a, b)
+    ref = orc.attn_bwd(q, k, v, do, N, idx, cnt, w)
+    for got, r in zip(good, ref):
+        got = got.double().cpu().numpy()
+        assert np.linalg.norm(got - r) <= 1e-2 * np.linalg.norm(r)
