@@ -296,10 +296,13 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *src, uint3
 // 1 ms (the wait-limit test entry) it polls with the non-blocking test_wait and reads the
 // clock at every poll (try_wait may hold the thread until the phase completes), so that
 // even a wait of a few microseconds can run past the limit.
+// The polling form is a separate instantiation of the kernels (kPoll), launched only by
+// the test entry, so that it adds nothing to the normal kernels' code.
+template <bool kPoll>
 __device__ __forceinline__ bool bwd_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *flag,
                                          uint64_t limit_ns)
 {
-    if (limit_ns >= 1000000ull) return mbar_wait(bar, parity, abort, flag, limit_ns);
+    if constexpr (!kPoll) return mbar_wait(bar, parity, abort, flag, limit_ns);
     const uint64_t t0 = global_timer_ns();
     for (;;) {
         uint32_t done;
@@ -321,10 +324,11 @@ __device__ __forceinline__ bool bwd_wait(uint64_t *bar, uint32_t parity, volatil
 }
 
 // The issuer warp's bounded wait (all lanes agree).
+template <bool kPoll>
 __device__ __forceinline__ bool issuer_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *flag,
                                             uint64_t limit_ns)
 {
-    return __all_sync(0xffffffffu, bwd_wait(bar, parity, abort, flag, limit_ns));
+    return __all_sync(0xffffffffu, bwd_wait<kPoll>(bar, parity, abort, flag, limit_ns));
 }
 
 // Copies of the issuer still in flight after a failed wait: let them land before the CTA
@@ -353,7 +357,7 @@ __device__ __forceinline__ void drain_issuer(uint64_t *bars, const Inflight &f, 
 //    the next P step. (Issuing dP(c+1) ahead of dQ(c), with dS in two buffers of the spare
 //    TMEM columns, measured 10% slower.)
 // ---------------------------------------------------------------------------------
-template <int D, bool kW>
+template <int D, bool kW, bool kPoll>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
@@ -454,11 +458,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // the block index of the next pair to load, read one iteration ahead of its use
         int j_pre = n > 2 ? __ldg(idx + 2) : 0;
-        bool ok = issuer_wait(&bars[0], 0, ab, p.flag, p.wait_ns);
+        bool ok = issuer_wait<kPoll>(&bars[0], 0, ab, p.flag, p.wait_ns);
         if (ok) f.waited[0] = 1;
-        ok = ok && issuer_wait(&bars[1], 0, ab, p.flag, p.wait_ns);
+        ok = ok && issuer_wait<kPoll>(&bars[1], 0, ab, p.flag, p.wait_ns);
         if (ok) ++f.waited[1];
-        ok = ok && issuer_wait(&bars[4], 0, ab, p.flag, p.wait_ns);
+        ok = ok && issuer_wait<kPoll>(&bars[4], 0, ab, p.flag, p.wait_ns);
         if (ok) {
             ++f.waited[2];
             tc_fence_after();
@@ -472,10 +476,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         for (int c = 0; ok && c < n; ++c) {
             // S(c) has been read: S(c + 1) may overwrite it
-            if (!issuer_wait(&bars[8], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
+            if (!issuer_wait<kPoll>(&bars[8], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             if (c + 1 < n) {
                 const int ks = (c + 1) % 3;
-                if (!issuer_wait(&bars[1 + ks], ((c + 1) / 3) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
+                if (!issuer_wait<kPoll>(&bars[1 + ks], ((c + 1) / 3) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
                 ++f.waited[1];
                 tc_fence_after();
                 if (elect_one()) {
@@ -485,7 +489,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 __syncwarp();
             }
             // dS(c) stored and dP(c) read: dQ += dS(c) K_c, then dP(c + 1) over it
-            if (!issuer_wait(&bars[9], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
+            if (!issuer_wait<kPoll>(&bars[9], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) {
                 mma_packed<D>(tAcc, tP, kd_mn(c % 3), c > 0);
@@ -494,7 +498,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             __syncwarp();
             if (c + 1 < n) {
                 const int vs = (c + 1) & 1;
-                if (!issuer_wait(&bars[4 + vs], ((c + 1) >> 1) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
+                if (!issuer_wait<kPoll>(&bars[4 + vs], ((c + 1) >> 1) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
                 ++f.waited[2];
                 tc_fence_after();
                 if (elect_one()) {
@@ -538,7 +542,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 j_raw = __ldg(idx + c + 1);
                 if (kW) w_raw = __ldg(wrow + c + 1);
             }
-            if (!__all_sync(0xffffffffu, bwd_wait(&bars[6], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait<kPoll>(&bars[6], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
             tc_fence_after();
             // P = 2^(s scale_log2 + log2 w - L2) on the valid keys of block j
             const int nvalid = p.N - j_cur * 128;
@@ -562,7 +566,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             tc_fence_before();
             mbar_arrive(&bars[8]);
-            if (!__all_sync(0xffffffffu, bwd_wait(&bars[7], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait<kPoll>(&bars[7], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
             tc_fence_after();
             // dS = P (dP - D), packed to bf16 over the first 32 of this half's dP columns
             uint32_t pk[32];
@@ -583,7 +587,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             j_cur = clamp_j(j_raw);
             lw_cur = kW ? lw2_val(w_raw, p.flag, threadIdx.x == 0) : 0.f;
         }
-        if (ok) ok = __all_sync(0xffffffffu, bwd_wait(&bars[11], 0, ab, p.flag, p.wait_ns));
+        if (ok) ok = __all_sync(0xffffffffu, bwd_wait<kPoll>(&bars[11], 0, ab, p.flag, p.wait_ns));
         if (ok) {
             tc_fence_after();
             store_acc_row<D>(tAcc + lane_off + half * (D / 2), p.dq + (row0 + row) * D + half * (D / 2),
@@ -647,7 +651,7 @@ struct MarkWalk {
     }
 };
 
-template <int D, bool kW>
+template <int D, bool kW, bool kPoll>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmG,
@@ -748,11 +752,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             load_q(1, q1);
             load_g(1, q1);
         }
-        bool ok = issuer_wait(&bars[0], 0, ab, p.flag, p.wait_ns);
+        bool ok = issuer_wait<kPoll>(&bars[0], 0, ab, p.flag, p.wait_ns);
         if (ok) f.waited[0] = 1;
-        ok = ok && issuer_wait(&bars[1], 0, ab, p.flag, p.wait_ns);
+        ok = ok && issuer_wait<kPoll>(&bars[1], 0, ab, p.flag, p.wait_ns);
         if (ok) ++f.waited[1];
-        ok = ok && issuer_wait(&bars[4], 0, ab, p.flag, p.wait_ns);
+        ok = ok && issuer_wait<kPoll>(&bars[4], 0, ab, p.flag, p.wait_ns);
         if (ok) {
             ++f.waited[2];
             tc_fence_after();
@@ -768,12 +772,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int s = c & 1, s1 = s ^ 1;
             // P^T(c) stored and S^T(c) read: dV += P^T dO_c, then S^T(c + 1) over it (the
             // pipe runs them in order; Q_{c+1} is the other slot of the ring)
-            if (!issuer_wait(&bars[8], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
+            if (!issuer_wait<kPoll>(&bars[8], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) mma_packed<D>(tV, tS, gd_mn(s), c > 0);
             __syncwarp();
             if (c + 1 < n) {
-                if (!issuer_wait(&bars[1 + s1], ((c + 1) >> 1) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
+                if (!issuer_wait<kPoll>(&bars[1 + s1], ((c + 1) >> 1) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
                 ++f.waited[1];
                 tc_fence_after();
                 if (elect_one()) {
@@ -783,7 +787,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 __syncwarp();
             }
             // dS^T(c) stored and dP^T(c) read: dK += dS^T Q_c, then dP^T(c + 1) over it
-            if (!issuer_wait(&bars[9], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
+            if (!issuer_wait<kPoll>(&bars[9], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             tc_fence_after();
             if (elect_one()) {
                 mma_packed<D>(tK, tP, qd_mn(s), c > 0);
@@ -792,7 +796,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             __syncwarp();
             if (c + 1 < n) {
-                if (!issuer_wait(&bars[4 + s1], ((c + 1) >> 1) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
+                if (!issuer_wait<kPoll>(&bars[4 + s1], ((c + 1) >> 1) & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
                 ++f.waited[2];
                 tc_fence_after();
                 if (elect_one()) {
@@ -803,7 +807,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             // pair c accumulated (dV(c), dK(c) and every earlier MMA done): its Q, rows and
             // dO slots take pair c + 2
-            if (!issuer_wait(&bars[10], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
+            if (!issuer_wait<kPoll>(&bars[10], c & 1, ab, p.flag, p.wait_ns)) { ok = false; break; }
             if (c + 2 < n) {
                 const int q2 = next_qb();
                 load_q(c + 2, q2);
@@ -835,8 +839,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             const int slot = c & 1;
             // the L2 and D rows arrive with Q_c
-            if (!__all_sync(0xffffffffu, bwd_wait(&bars[1 + slot], (c >> 1) & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
-            if (!__all_sync(0xffffffffu, bwd_wait(&bars[6], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait<kPoll>(&bars[1 + slot], (c >> 1) & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait<kPoll>(&bars[6], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
             tc_fence_after();
             // P^T = 2^(s scale_log2 + log2 w - L2_i) for this key over the half's queries
             float pv[64];
@@ -874,7 +878,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[8]);
-            if (!__all_sync(0xffffffffu, bwd_wait(&bars[7], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, bwd_wait<kPoll>(&bars[7], c & 1, ab, p.flag, p.wait_ns))) { ok = false; break; }
             tc_fence_after();
             // dS^T = P^T (dP^T - D_i)
             uint32_t dv2[2][32];
@@ -901,7 +905,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_arrive(&bars[9]);
             lw_cur = kW ? lw2_val(w_raw, p.flag, threadIdx.x == 0) : 0.f;
         }
-        if (ok) ok = __all_sync(0xffffffffu, bwd_wait(&bars[11], 0, ab, p.flag, p.wait_ns));
+        if (ok) ok = __all_sync(0xffffffffu, bwd_wait<kPoll>(&bars[11], 0, ab, p.flag, p.wait_ns));
         if (ok) {
             tc_fence_after();
             store_acc_row<D>(tV + lane_off + half * (D / 2), p.dv + (row0 + key) * D + half * (D / 2), 1.f,
@@ -927,7 +931,7 @@ bool bwd_tmap(CUtensorMap *tm, const void *base, int BH, int N, int N_pad, int d
                              (uint64_t)N_pad * d * 2, 64, 128);
 }
 
-template <int D, bool kW>
+template <int D, bool kW, bool kPoll>
 cudaError_t launch_bwd_t(const AttnBwdLaunch &a, cudaStream_t st)
 {
     const int BH = a.B * a.H, nb = a.N_pad / 128;
@@ -976,21 +980,32 @@ cudaError_t launch_bwd_t(const AttnBwdLaunch &a, cudaStream_t st)
     p.scale = (float)(1.0 / std::sqrt((double)D));
     p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
     p.wait_ns = a.wait_ns > 0 ? a.wait_ns : kWaitLimitNs;
-    e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem);
+    e = cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kW, kPoll>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kDqSmem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, kW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDkdvSmem);
+    e = cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, kW, kPoll>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kDkdvSmem);
     if (e != cudaSuccess) return e;
-    attn_bwd_dq_kernel<D, kW><<<(unsigned)plan_rows, kBwdThreads, kDqSmem, st>>>(tq, tk, tv, tg, p);
+    attn_bwd_dq_kernel<D, kW, kPoll><<<(unsigned)plan_rows, kBwdThreads, kDqSmem, st>>>(tq, tk, tv, tg, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    attn_bwd_dkdv_kernel<D, kW><<<(unsigned)plan_rows, kBwdThreads, kDkdvSmem, st>>>(tq, tk, tv, tg, p);
+    attn_bwd_dkdv_kernel<D, kW, kPoll><<<(unsigned)plan_rows, kBwdThreads, kDkdvSmem, st>>>(tq, tk, tv, tg, p);
     return cudaGetLastError();
 }
 
-cudaError_t launch_attn_bwd(const AttnBwdLaunch &a, cudaStream_t st)
+template <bool kPoll>
+cudaError_t launch_attn_bwd_p(const AttnBwdLaunch &a, cudaStream_t st)
 {
     const bool weighted = a.w != nullptr;
-    if (a.d == 128) return weighted ? launch_bwd_t<128, true>(a, st) : launch_bwd_t<128, false>(a, st);
-    return weighted ? launch_bwd_t<64, true>(a, st) : launch_bwd_t<64, false>(a, st);
+    if (a.d == 128)
+        return weighted ? launch_bwd_t<128, true, kPoll>(a, st) : launch_bwd_t<128, false, kPoll>(a, st);
+    return weighted ? launch_bwd_t<64, true, kPoll>(a, st) : launch_bwd_t<64, false, kPoll>(a, st);
+}
+
+// A wait limit below 1 ms (the test entry) takes the polling instantiation.
+cudaError_t launch_attn_bwd(const AttnBwdLaunch &a, cudaStream_t st)
+{
+    if (a.wait_ns > 0 && a.wait_ns < 1000000ull) return launch_attn_bwd_p<true>(a, st);
+    return launch_attn_bwd_p<false>(a, st);
 }
 
 // The shape rules of the forward calls (include/ab_attn.h): 128-token blocks, d in
