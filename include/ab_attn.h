@@ -17,7 +17,8 @@
  *     is a DEVICE pointer on the current device, allocated and owned by the caller,
  *     16-byte aligned. The calls allocate no device memory; the host-side work is
  *     argument validation, building TMA tensor maps and enqueueing kernels (and, for
- *     the attention calls, one 16-byte memset; for ab_forward_host, the copies).
+ *     the attention calls, one 16-byte memset; for ab_attn_bwd, one memset of part of
+ *     its workspace; for ab_forward_host, the copies).
  *   - Library-owned device state: two file-scope __device__ arrays exist once on every
  *     GPU that loads the library, from load until process exit: the attention
  *     kernels' 4096 claim slots (16 bytes each; see "Scheduling" at ab_attn_fwd) and
