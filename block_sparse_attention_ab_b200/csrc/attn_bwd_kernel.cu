@@ -30,8 +30,9 @@
 // tensor core runs the next pair's products while the warps work on the current one.
 // Tiles arrive by TMA in 64-column boxes with the 128-byte swizzle, as in the forward
 // kernel. Every wait is bounded; a wait that gives up raises AB_FLAG_TIMEOUT, and the
-// CTA lets its copies and MMAs land and frees its tensor memory before it returns. The C entry points ab_attn_bwd and ab_attn_bwd_workspace_size
-// are at the end of this file.
+// CTA lets its copies and MMAs land and frees its tensor memory before it returns. The C
+// entry points ab_attn_bwd, ab_attn_bwd_workspace_size and the wait-limit test entry
+// ab_selftest_attn_bwd_wait_limit are at the end of this file.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
