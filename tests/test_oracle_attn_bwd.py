@@ -7,7 +7,9 @@ oracle's hand-written backward is checked against torch autograd in fp64 of the 
 function written densely (a log-weight bias on kept blocks, -inf elsewhere), and against
 two closed forms: the softmax is invariant to a shift of a row's logits, so the key
 gradients of a head sum to zero, and each row's probabilities sum to one, so the value
-gradients of a head sum to the sum of the upstream gradient rows.
+gradients of a head sum to the sum of the upstream gradient rows. The value gradient is
+also tied to the separately written forward oracle: O is linear in V, so an exact change
+of one value changes the loss by exactly that change times its gradient.
 """
 
 import math
@@ -139,3 +141,34 @@ def test_bwd_weight_is_block_multiplicity(orc):
     np.testing.assert_allclose(dq, qf.grad.numpy(), rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(dk, kf.grad.numpy(), rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(dv, vf.grad.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_bwd_dv_is_the_forward_oracles_derivative(orc):
+    """O is linear in V, so doubling one value v of V (exact in bf16) changes the loss
+    L = sum_i dO_i . O_i by exactly v * dL/dv. The separately written forward oracle
+    gives both losses; the backward oracle's dV must equal their difference over v."""
+    N, H, d = 3 * 128 + 40, 1, 64
+    q, k, v, do = _inputs(N, H, d, seed=21)
+    nb = q.shape[2] // 128
+    idx, cnt, w = _plan(1, H, nb, 2, seed=9, weighted=True)
+    _, _, dv = orc.attn_bwd(q, k, v, do, N, idx, cnt, w)
+    g = do.double().numpy()[0, 0]
+
+    def loss(vv):
+        out, _, _, _ = orc.attn_rows(q, k, vv, N, idx, cnt, w)
+        o = out.reshape(nb * 128, d)
+        return float((o[:N] * g[:N]).sum())
+
+    base = loss(v)
+    checked = 0
+    for t, e in ((5, 3), (130, 17), (300, 63), (N - 1, 0)):
+        val = float(v[0, 0, t, e].float())
+        if val == 0.0:
+            continue
+        v2 = v.clone()
+        v2[0, 0, t, e] = torch.tensor(2.0 * val).to(torch.bfloat16)
+        assert float(v2[0, 0, t, e].float()) == 2.0 * val
+        fd = (loss(v2) - base) / val
+        assert abs(fd - dv[0, 0, t, e]) <= 1e-9 * max(1.0, abs(dv[0, 0, t, e]))
+        checked += 1
+    assert checked >= 3
