@@ -35,7 +35,8 @@ median and min; "cold" = a 256 MB buffer written before each call to flush L2):
   e2e            the headline step through the public API with host buffers (pinned
                  H2D of Q, K, V and D2H of O inside the timed region);
   cpu_baseline   the CPU oracle on a bounded sample of the headline workload,
-                 extrapolated to a whole step.
+                 extrapolated to a whole step (and cpu_baseline_backward: the oracle's
+                 attention gradient on sampled pairs of HunyuanVideo-720p);
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Profiling runs: --config NAME --heads H --headline-only (the headline step only),
@@ -576,6 +577,14 @@ def run_ours(args, rank, world, local_rank):
         res["workloads"] = other_workloads(ab, dev, args, peaks, calls)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, K, seconds=args.cpu_seconds)
+        if not args.headline_only:
+            # the oracle beside the attention backward (HunyuanVideo-720p at 10%); a
+            # failure here is reported in the line, never fatal to it
+            try:
+                wb = workload("hunyuan720")
+                res["cpu_baseline_backward"] = cpu_baseline_backward(wb, wb.budget_blocks(wb.budgets[0]))
+            except Exception as e:  # noqa: BLE001
+                res["cpu_baseline_backward"] = {"unavailable": f"{type(e).__name__}: {e}"}
     return res
 
 
@@ -824,6 +833,63 @@ def cpu_baseline(w, K, seconds: float = 15.0, n_items: int = 64):
                        f"blocks plus the mean keys of 1 of {w.B * w.H} heads, extrapolated to one "
                        f"whole step: {detail}"),
             "est_step_s": round(step_s, 2)}
+
+
+def cpu_baseline_backward(w, K, n_items: int = 3, seed: int = 777):
+    """The oracle's attention gradient, as it stands, on a bounded sample of workload w at
+    budget K: for `n_items` query blocks of head 0 (their plan rows from the oracle's own
+    k-means, score and SIP), the gradient of a problem that holds only that block's
+    queries and its kept key blocks (the same work per kept pair as the whole backward),
+    timed and extrapolated to the B*H*n_qb*K pairs of the workload."""
+    import oracle
+
+    rng = np.random.default_rng(seed)
+    nb, d = w.n_blocks, w.d
+    q, k, v = _head_data(w, 0)
+    kbar = oracle.mean_key(k, w.N)
+    gen = torch.Generator().manual_seed(seed)
+    t_bwd, pairs = 0.0, 0
+    for qb in rng.choice(nb, size=n_items, replace=False):
+        qb = int(qb)
+        nv = min(128, w.N - qb * 128)
+        qblk = torch.zeros(1, 1, 128, d, dtype=q.dtype)
+        qblk[0, 0, :nv] = q[0, 0, qb * 128: qb * 128 + nv]
+        cent, wts, _, _, _ = oracle.kmeans(qblk, nv, w.n_clusters, w.iters)
+        sc = oracle.score(cent, wts, kbar)
+        i_, c_, w_, _, _ = oracle.sip(sc.astype(np.float32), K, w.sip_seed, with_p=False)
+        c = int(c_[0, 0, 0])
+        if c == 0:
+            continue
+        sel = [int(j) for j in i_[0, 0, 0, :c]]
+        nb2 = c + 1  # block 0: the query block; blocks 1..c: its kept key blocks
+        Q2 = torch.zeros(1, 1, nb2 * 128, d, dtype=torch.bfloat16)
+        K2, V2, G2 = torch.zeros_like(Q2), torch.zeros_like(Q2), torch.zeros_like(Q2)
+        Q2[0, 0, :nv] = q[0, 0, qb * 128: qb * 128 + nv]
+        G2[0, 0, :nv] = torch.randn(nv, d, generator=gen).to(torch.bfloat16)
+        for m, j in enumerate(sel):
+            K2[0, 0, (m + 1) * 128:(m + 2) * 128] = k[0, 0, j * 128:(j + 1) * 128]
+            V2[0, 0, (m + 1) * 128:(m + 2) * 128] = v[0, 0, j * 128:(j + 1) * 128]
+        N2 = nb2 * 128 - ((w.N_pad - w.N) if sel[-1] == nb - 1 else 0)
+        idx2 = np.full((1, 1, nb2, nb2), -1, dtype=np.int32)
+        cnt2 = np.zeros((1, 1, nb2), dtype=np.int32)
+        w2 = np.zeros((1, 1, nb2, nb2), dtype=np.float32)
+        idx2[0, 0, 0, :c] = np.arange(1, c + 1)
+        cnt2[0, 0, 0] = c
+        w2[0, 0, 0, :c] = w_[0, 0, 0, :c]
+        t0 = time.perf_counter()
+        oracle.attn_bwd(Q2, K2, V2, G2, N2, idx2, cnt2, w2)
+        t_bwd += time.perf_counter() - t0
+        pairs += c
+    per_pair = t_bwd / max(1, pairs)
+    total = w.B * w.H * nb * K
+    est_s = per_pair * total
+    return {"value": round(10 * 128 * 128 * d * total / est_s / 1e12, 6),
+            "unit": "TFLOP/s (5 products of 128x128xd per kept pair)", "cores": 1,
+            "kind": "oracle", "extrapolated": True,
+            "sample": (f"{pairs} kept (query block, key block) pairs of {n_items} query blocks of "
+                       f"head 0 of {w.name} at {K}/{nb} blocks (one thread: one head), "
+                       f"{per_pair * 1e3:.1f} ms per pair, extrapolated to {total} pairs"),
+            "est_s": round(est_s, 1)}
 
 
 def run_reference(args, rank, world):
