@@ -290,6 +290,8 @@ def attn_bwd(q, k, v, N: int, idx, cnt, w, out, lse, dout,
     _need(cnt, torch.int32, "cnt")
     if w is not None:
         _need(w, torch.float32, "w")
+    if not isinstance(out, torch.Tensor) or out.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out must be the forward's bf16 or fp32 output")
     _need(out, out.dtype, "out")
     _need(lse, torch.float32, "lse")
     shape = make_shape(q, N)
